@@ -1,0 +1,368 @@
+"""CPU oracle for the LRMoE pruned MoE expert backward -- TEST INFRASTRUCTURE ONLY.
+
+Plain, slow, obviously-correct numpy restatement of what the hot path computes.
+Only the tests, the package smoke check and the benchmark's CPU-baseline leg may
+import it; the product path never does.  It shares no code with the CUDA
+library (only the seeded input generator, which holds none of this arithmetic).
+
+Source of the method: the three news pages on LRMoE.  Citations name the page
+title and section:
+  [RU-B]  "LRMoE урезает обратный проход MoE ...", section "Что делает LRMoE:
+          полный прямой проход, обрезанный обратный" (bullets 1-5 and the note
+          after them); [FR-B] is the same section of the French page
+          ("Ce que fait LRMoE : passe avant complète, passe arrière élaguée").
+  [RU-C]  same page, section "Что показали эксперименты и где подвох".
+  [DE]    "LRMoE führt eine Nachkalibrierung der Last ...", paragraphs 3-4.
+
+What each function follows
+--------------------------
+lrm_score        [RU-B] bullet 3 / [FR-B] bullet 3 / [DE] para 3: a pair's
+                 contribution to the expert weight update is the outer product
+                 of the incoming gradient (w * dY) and the saved projection
+                 input a; its squared Frobenius norm factorises into
+                 w^2 * ||dY||^2 * ||a||^2, so no gradient matrix is formed.
+select_quota     [RU-B] bullet 3 (last sentence) / [DE] para 3: within the
+                 per-expert quota the pairs with the highest score stay.
+pack             [RU-B] bullet 5 / [DE] para 4: retained gradient and
+                 activation rows are gathered into dense per-expert blocks;
+                 [RU-B] note: masking rows inside full tensors gives nothing,
+                 only physically smaller matrices do.
+expert_backward  [RU-B] bullet 5: variable-size grouped GEMMs on those blocks
+                 with no zero padding (here: plain fp64 matmuls per expert).
+unpack           [RU-B] bullet 5, last sentence: the result goes back to the
+                 original layout.
+dense_backward   the ordinary unpruned SwiGLU MoE expert backward (textbook
+                 calculus); used only to pin the pruned functions.
+forward          the ordinary SwiGLU MoE forward in fp64, used only by the
+                 finite-difference pin ([RU-B] bullet 1: the forward stays full).
+
+Readings where the pages are silent:
+  R1  "saved projection input" = a = silu(g)*u, the input of the down
+      projection, because the incoming gradient there is w*dY.
+  R2  one retained set serves dW_down, dW_gate, dW_up and dX.
+  R3  canonical fp32 score order (below) so that selection is bit-comparable.
+  R4  key = (score bits descending, pair index ascending); blocks in ascending
+      expert id, rows inside a block in ascending pair index; NaN scores are
+      canonicalised to 0x7FFFFFFF (rank above +Inf).
+  R5  quotas are integers given as input; m_e = min(max(q_e, 0), c_e).
+  R6  the packed gradient row is RNE_storage(fp32(w) * fp32(dY_t)); all
+      gradient arithmetic afterwards is fp64 here.
+  R7  topk_idx < 0 = not routed; idx >= E = invalid (skipped, status bit).
+
+Canonical score order (R3), for one row v of D = V * VEC elements
+(VEC = 8 for bf16 storage, 4 for fp32):
+  1. 32 fp32 partials start at +0.  Partial l takes vectors c = l, l+32, ...
+  2. inside a vector, elements in index order: acc = fl(acc + fl(x*x))
+     (two RNE roundings, no fused multiply-add).
+  3. butterfly: for o in 16, 8, 4, 2, 1: acc[l] = fl(acc[l] + acc[l ^ o]).
+  4. the norm is acc[0].
+  score = fl(fl(fl(w*w) * n_dY) * n_a).
+
+Parity with the pages themselves is unpinned for R1 and R2 (the pages print no
+worked example); every function below is pinned to closed forms, brute force,
+library routines or finite differences by the tests under tests/.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+ST_BAD_EXPERT = 1
+ST_BAD_QUOTA = 2
+ST_NONFINITE = 4
+
+NAN_SCORE_BITS = np.uint32(0x7FFFFFFF)
+VEC = {"bf16": 8, "f32": 4}
+
+
+# ----------------------------------------------------------------------------
+# storage helpers (bf16 kept as uint16 bit patterns)
+# ----------------------------------------------------------------------------
+def decode(arr: np.ndarray, dtype: str) -> np.ndarray:
+    """Storage values -> float32.  bf16 bits b are the upper half of an fp32."""
+    if dtype == "bf16":
+        return (arr.astype(np.uint32) << np.uint32(16)).view(np.float32)
+    if dtype in ("f32", "f64"):
+        return np.asarray(arr)
+    raise ValueError(dtype)
+
+
+def encode_rne(v32: np.ndarray, dtype: str) -> np.ndarray:
+    """float32 -> storage dtype with round-to-nearest-even; NaN -> 0x7FFF (bf16)."""
+    if dtype in ("f32", "f64"):
+        return np.asarray(v32)
+    bits = np.ascontiguousarray(v32, dtype=np.float32).view(np.uint32)
+    lsb = (bits >> np.uint32(16)) & np.uint32(1)
+    rounded = (bits.astype(np.uint64) + np.uint64(0x7FFF) + lsb.astype(np.uint64)) >> np.uint64(16)
+    out = rounded.astype(np.uint16)
+    out[np.isnan(v32)] = np.uint16(0x7FFF)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# a1: LRM score
+# ----------------------------------------------------------------------------
+def row_sq_norm(rows32: np.ndarray, vec: int) -> np.ndarray:
+    """Squared L2 norm of each row in the canonical fp32 order (R3)."""
+    rows32 = np.ascontiguousarray(rows32, dtype=np.float32)
+    n, D = rows32.shape
+    assert D % vec == 0
+    V = D // vec
+    v = rows32.reshape(n, V, vec)
+    acc = np.zeros((n, 32), dtype=np.float32)
+    for r in range(0, V, 32):             # round r: lane l holds vector r + l
+        nl = min(32, V - r)
+        for j in range(vec):
+            x = v[:, r:r + nl, j]
+            acc[:, :nl] = acc[:, :nl] + x * x
+    lane = np.arange(32)
+    for o in (16, 8, 4, 2, 1):
+        acc = acc + acc[:, lane ^ o]
+    return acc[:, 0].copy()
+
+
+def lrm_score(topk_idx, topk_w, dY, a, dtype: str, E: int):
+    """score[p] = w_p^2 * ||dY_t||^2 * ||a_p||^2 for every routed pair p = t*k + j.
+
+    Non-routed (idx < 0) and invalid (idx >= E) slots get +0 and are never
+    selected; invalid ones set ST_BAD_EXPERT.  NaN scores set ST_NONFINITE.
+    """
+    T, k = topk_idx.shape
+    idx = topk_idx.reshape(-1)
+    w = topk_w.reshape(-1).astype(np.float32)
+    status = 0
+    if np.any(idx >= E):
+        status |= ST_BAD_EXPERT
+    routed = (idx >= 0) & (idx < E)
+    vec = VEC[dtype]
+    n_dy = row_sq_norm(decode(dY, dtype), vec)                 # [T]
+    n_a = row_sq_norm(decode(a, dtype), vec)                   # [P]
+    n_dy_p = np.repeat(n_dy, k)
+    s = ((w * w) * n_dy_p) * n_a
+    s = np.where(routed, s, np.float32(0.0)).astype(np.float32)
+    bits = s.view(np.uint32).copy()
+    nan = np.isnan(s)
+    if np.any(nan):
+        status |= ST_NONFINITE
+        bits[nan] = NAN_SCORE_BITS
+    if np.any(np.isinf(s)):
+        status |= ST_NONFINITE
+    return bits.view(np.float32), status
+
+
+def lrm_score_f64(topk_idx, topk_w, dY64, a64):
+    """Same factorised score in fp64 (no canonical order); used by pins only."""
+    T, k = topk_idx.shape
+    w = topk_w.reshape(-1).astype(np.float64)
+    n_dy = np.repeat((dY64.astype(np.float64) ** 2).sum(1), k)
+    n_a = (a64.astype(np.float64) ** 2).sum(1)
+    return w * w * n_dy * n_a
+
+
+# ----------------------------------------------------------------------------
+# a2: per-expert top-quota selection
+# ----------------------------------------------------------------------------
+def select_quota(topk_idx, score, quota, E: int):
+    """Keep, per expert, the m_e = min(max(q_e,0), c_e) pairs with the largest key.
+
+    Returns counts[E], kept[E], offsets[E+1], perm[M], pos[P], status.
+    perm lists the retained pairs, expert blocks in ascending e and pairs in
+    ascending index inside a block; pos[p] is p's packed row or -1.
+    """
+    idx = topk_idx.reshape(-1)
+    P = idx.size
+    bits = np.ascontiguousarray(score, dtype=np.float32).view(np.uint32)
+    quota = np.asarray(quota, dtype=np.int64)
+    status = 0
+    if np.any(quota < 0):
+        status |= ST_BAD_QUOTA
+    if np.any(idx >= E):
+        status |= ST_BAD_EXPERT
+    counts = np.zeros(E, dtype=np.int32)
+    kept = np.zeros(E, dtype=np.int32)
+    offsets = np.zeros(E + 1, dtype=np.int32)
+    pos = np.full(P, -1, dtype=np.int32)
+    blocks = []
+    for e in range(E):
+        pairs = np.nonzero(idx == e)[0]                        # ascending p
+        c = pairs.size
+        m = int(min(max(int(quota[e]), 0), c))
+        counts[e] = c
+        kept[e] = m
+        offsets[e + 1] = offsets[e] + m
+        # sort by (bits descending, p ascending); lexsort keys: last is primary
+        order = np.lexsort((pairs, np.uint32(0xFFFFFFFF) - bits[pairs]))
+        chosen = np.sort(pairs[order[:m]])
+        blocks.append(chosen)
+    perm = np.concatenate(blocks).astype(np.int32) if blocks else np.zeros(0, np.int32)
+    pos[perm] = np.arange(perm.size, dtype=np.int32)
+    return counts, kept, offsets, perm, pos, status
+
+
+# ----------------------------------------------------------------------------
+# a3: physical compaction
+# ----------------------------------------------------------------------------
+def pack(perm, topk_w, k: int, x, dY, a, g, u, dtype: str):
+    """Gather retained rows into dense blocks (storage dtype).
+
+    X_p[r] = x[t], DY_p[r] = RNE(fp32(w_p) * fp32(dY[t])), A_p/G_p/U_p[r] = a/g/u[p],
+    with p = perm[r], t = p // k.
+    """
+    perm = np.asarray(perm, dtype=np.int64)
+    t = perm // k
+    w = topk_w.reshape(-1)[perm].astype(np.float32)
+    if dtype == "f64":
+        DYp = w.astype(np.float64)[:, None] * dY[t]
+    else:
+        DYp = encode_rne(w[:, None] * decode(dY, dtype)[t], dtype)
+    return x[t].copy(), DYp, a[perm].copy(), g[perm].copy(), u[perm].copy()
+
+
+# ----------------------------------------------------------------------------
+# a4: expert backward on the compacted blocks
+# ----------------------------------------------------------------------------
+def sigmoid64(g):
+    return 1.0 / (1.0 + np.exp(-g))
+
+
+def expert_backward(Xp, DYp, Ap, Gp, Up, offsets, W_gu, W_down, dtype: str, experts=None):
+    """fp64 SwiGLU expert backward over each expert's packed rows.
+
+    For rows R_e = [offsets[e], offsets[e+1]):
+      dA      = DY_p W_down[e]                      (m_e x I)
+      dG      = dA * u * s * (1 + g (1 - s)),  s = sigmoid(g)
+      dU      = dA * g * s
+      dW_down = DY_p^T A_p                          (H x I)
+      dW_gu   = [dG | dU]^T X_p                     (2I x H)
+      dX_p    = [dG | dU] W_gu[e]                   (m_e x H)
+    Returns (dW_down [E,H,I] or dict, dW_gu, dXp [M,H], dGUp [M,2I]) in fp64.
+    `experts` restricts the weight gradients to a subset (dict keyed by e).
+    """
+    E = offsets.size - 1
+    f = lambda arr: decode(arr, dtype).astype(np.float64)
+    M = int(offsets[-1])
+    H = W_down.shape[1]
+    I = W_down.shape[2]
+    dXp = np.zeros((M, H), dtype=np.float64)
+    dGUp = np.zeros((M, 2 * I), dtype=np.float64)
+    sel = range(E) if experts is None else experts
+    dW_down = {}
+    dW_gu = {}
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        want_w = e in sel
+        if hi == lo:
+            if want_w:
+                dW_down[e] = np.zeros((H, I))
+                dW_gu[e] = np.zeros((2 * I, H))
+            continue
+        dy = f(DYp[lo:hi])
+        g = f(Gp[lo:hi])
+        u = f(Up[lo:hi])
+        Wd = f(W_down[e])
+        Wgu = f(W_gu[e])
+        dA = dy @ Wd
+        s = sigmoid64(g)
+        dG = dA * u * s * (1.0 + g * (1.0 - s))
+        dU = dA * g * s
+        dGU = np.concatenate([dG, dU], axis=1)
+        dGUp[lo:hi] = dGU
+        dXp[lo:hi] = dGU @ Wgu
+        if want_w:
+            dW_down[e] = dy.T @ f(Ap[lo:hi])
+            dW_gu[e] = dGU.T @ f(Xp[lo:hi])
+    if experts is None:
+        dW_down = np.stack([dW_down[e] for e in range(E)])
+        dW_gu = np.stack([dW_gu[e] for e in range(E)])
+    return dW_down, dW_gu, dXp, dGUp
+
+
+# ----------------------------------------------------------------------------
+# a5: back to the token layout
+# ----------------------------------------------------------------------------
+def unpack(dXp, pos, T: int, k: int):
+    """dX[t] = sum over j ascending of dX_p[pos[t*k+j]] for retained pairs; else 0."""
+    H = dXp.shape[1]
+    dX = np.zeros((T, H), dtype=np.float64)
+    pos = np.asarray(pos).reshape(T, k)
+    for j in range(k):
+        r = pos[:, j]
+        keep = r >= 0
+        dX[keep] += dXp[r[keep]]
+    return dX
+
+
+# ----------------------------------------------------------------------------
+# whole path
+# ----------------------------------------------------------------------------
+def pruned_backward(layer, experts=None):
+    """Run a1..a5 on a generated layer.  Returns a dict of every intermediate."""
+    s = layer.spec
+    dt = s.dtype
+    score, st1 = lrm_score(layer.topk_idx, layer.topk_w, layer.dY, layer.a, dt, s.E)
+    counts, kept, offsets, perm, pos, st2 = select_quota(layer.topk_idx, score, layer.quota, s.E)
+    Xp, DYp, Ap, Gp, Up = pack(perm, layer.topk_w, s.k, layer.x, layer.dY, layer.a, layer.g, layer.u, dt)
+    dW_down, dW_gu, dXp, dGUp = expert_backward(Xp, DYp, Ap, Gp, Up, offsets, layer.W_gu,
+                                                layer.W_down, dt, experts=experts)
+    dX = unpack(dXp, pos, s.T, s.k)
+    return dict(score=score, status=st1 | st2, counts=counts, kept=kept, offsets=offsets,
+                perm=perm, pos=pos, Xp=Xp, DYp=DYp, Ap=Ap, Gp=Gp, Up=Up,
+                dW_down=dW_down, dW_gu=dW_gu, dXp=dXp, dGUp=dGUp, dX=dX)
+
+
+# ----------------------------------------------------------------------------
+# unpruned references (pins only)
+# ----------------------------------------------------------------------------
+def dense_backward(topk_idx, grad_rows, x, g, u, a, W_gu, W_down):
+    """Unpruned expert backward, one pair at a time, in fp64.
+
+    grad_rows[p] is the gradient arriving at expert output y_p (w_p * dY_t,
+    already in the precision the caller chose).  Pairs with idx < 0 or idx >= E
+    are skipped.  Returns dW_down [E,H,I], dW_gu [E,2I,H], dX [T,H].
+    """
+    T, k = topk_idx.shape
+    E, H, I = W_down.shape
+    dW_down = np.zeros((E, H, I))
+    dW_gu = np.zeros((E, 2 * I, H))
+    dX = np.zeros((T, H))
+    for t in range(T):
+        for j in range(k):
+            e = int(topk_idx[t, j])
+            if e < 0 or e >= E:
+                continue
+            p = t * k + j
+            gy = grad_rows[p]                                  # dL/dy_p      [H]
+            dW_down[e] += np.outer(gy, a[p])                   # dL/dW_down
+            da = W_down[e].T @ gy                              # dL/da        [I]
+            sg = 1.0 / (1.0 + np.exp(-g[p]))
+            silu = g[p] * sg
+            dsilu = sg * (1.0 + g[p] * (1.0 - sg))
+            dg = da * u[p] * dsilu
+            du = da * silu
+            dW_gu[e, :I] += np.outer(dg, x[t])
+            dW_gu[e, I:] += np.outer(du, x[t])
+            dX[t] += W_gu[e, :I].T @ dg + W_gu[e, I:].T @ du
+    return dW_down, dW_gu, dX
+
+
+def forward(topk_idx, topk_w, x, W_gu, W_down):
+    """Y_t = sum_j w_tj * W_down[e] (silu(W_gate[e] x_t) * (W_up[e] x_t)), fp64.
+
+    Also returns the saved per-pair g, u, a.
+    """
+    T, k = topk_idx.shape
+    E, H, I = W_down.shape
+    Y = np.zeros((T, H))
+    g = np.zeros((T * k, I))
+    u = np.zeros((T * k, I))
+    a = np.zeros((T * k, I))
+    for t in range(T):
+        for j in range(k):
+            e = int(topk_idx[t, j])
+            if e < 0 or e >= E:
+                continue
+            p = t * k + j
+            g[p] = W_gu[e, :I] @ x[t]
+            u[p] = W_gu[e, I:] @ x[t]
+            a[p] = g[p] / (1.0 + np.exp(-g[p])) * u[p]
+            Y[t] += topk_w[t, j] * (W_down[e] @ a[p])
+    return Y, g, u, a

@@ -1,0 +1,387 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties one oracle function to a closed form, brute force, a library
+routine, finite differences or a hand-worked example, so that a dropped term,
+a wrong sign or index, or a transposed operand in the oracle fails here.
+No GPU is needed.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lrmoe_oracle as O
+from pruned_expert_backward_lrmoe_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+U = 2.0 ** -24
+
+
+# ----------------------------------------------------------------------------
+# helpers local to the tests
+# ----------------------------------------------------------------------------
+def brute_force_contribution_norm(w, dy_row, a_row):
+    """||(w dY) a^T||_F^2 by forming the full H x I matrix in fp64."""
+    G = np.outer(np.float64(w) * dy_row.astype(np.float64), a_row.astype(np.float64))
+    return float((G * G).sum())
+
+
+def small_layer(name="tiny", seed=0, **over):
+    return inputs.make_layer(inputs.spec(name, **over), seed=seed)
+
+
+# ----------------------------------------------------------------------------
+# worked example from the golden fixture
+# ----------------------------------------------------------------------------
+def _read_golden(fname):
+    rows = {}
+    with open(os.path.join(GOLDEN, fname)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            rows.setdefault(key, []).append([float(v) for v in vals])
+    return rows
+
+
+def test_golden_worked_example():
+    g = _read_golden("score_worked_example.txt")
+    idx = np.array(g["topk_idx"][0], np.int32).reshape(2, 2)
+    w = np.array(g["topk_w"][0], np.float32).reshape(2, 2)
+    dY = np.array(g["dY"], np.float32)
+    a = np.array(g["a"], np.float32)
+    quota = np.array(g["quota"][0], np.int32)
+    score, st = O.lrm_score(idx, w, dY, a, "f32", 2)
+    assert st == 0
+    np.testing.assert_array_equal(score, np.array(g["score"][0], np.float32))
+    counts, kept, offsets, perm, pos, st = O.select_quota(idx, score, quota, 2)
+    np.testing.assert_array_equal(counts, g["counts"][0])
+    np.testing.assert_array_equal(kept, g["kept"][0])
+    np.testing.assert_array_equal(offsets, g["offsets"][0])
+    np.testing.assert_array_equal(perm, g["perm"][0])
+    np.testing.assert_array_equal(pos, g["pos"][0])
+
+
+# ----------------------------------------------------------------------------
+# T1: factorisation of the contribution norm
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_t1_factorisation_dyadic_exact(dtype):
+    """Dyadic inputs: brute-force outer-product norm == fp64 factorised == canonical fp32, bitwise."""
+    rng = np.random.default_rng(1)
+    T, k, E, H, I = 12, 3, 4, 64, 128
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    w = rng.choice(np.array([0.5, 0.25, 0.75, 1.0, 0.125], np.float32), size=(T, k))
+    dY32 = (rng.integers(-4, 5, size=(T, H)) / 8.0).astype(np.float32)
+    a32 = (rng.integers(-4, 5, size=(T * k, I)) / 8.0).astype(np.float32)
+    dY = O.encode_rne(dY32, dtype)
+    a = O.encode_rne(a32, dtype)
+    s32, st = O.lrm_score(idx, w, dY, a, dtype, E)
+    s64 = O.lrm_score_f64(idx, w, dY32, a32)
+    for p in range(T * k):
+        t = p // k
+        bf = brute_force_contribution_norm(w.reshape(-1)[p], dY32[t], a32[p])
+        assert bf == s64[p]
+        assert float(s32[p]) == bf
+    assert st == 0
+
+
+@pytest.mark.parametrize("dtype,H,I", [("f32", 64, 128), ("bf16", 2048, 768), ("bf16", 4096, 1408),
+                                       ("f32", 36, 20)])
+def test_t1_factorisation_random_within_bound(dtype, H, I):
+    """Random inputs: fp64 factorised vs brute force <= 1e-12, canonical fp32 within its bound."""
+    rng = np.random.default_rng(2)
+    T, k, E = 16, 2, 3
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    w = rng.random((T, k)).astype(np.float32)
+    dY = O.encode_rne(rng.standard_normal((T, H)).astype(np.float32), dtype)
+    a = O.encode_rne(rng.standard_normal((T * k, I)).astype(np.float32), dtype)
+    dY32, a32 = O.decode(dY, dtype), O.decode(a, dtype)
+    s32, _ = O.lrm_score(idx, w, dY, a, dtype, E)
+    s64 = O.lrm_score_f64(idx, w, dY32, a32)
+    # error of the canonical order: per norm, ceil(D/32) sequential adds + 5 butterfly
+    # levels + 1 product rounding; three final multiplies.
+    bound = ((math.ceil(H / 32) + 6) + (math.ceil(I / 32) + 6) + 4) * U * 1.01
+    for p in range(T * k):
+        t = p // k
+        if H * I <= 64 * 128:
+            bf = brute_force_contribution_norm(w.reshape(-1)[p], dY32[t], a32[p])
+            assert abs(bf - s64[p]) <= 1e-12 * bf
+        assert abs(float(s32[p]) - s64[p]) <= bound * s64[p]
+
+
+@pytest.mark.parametrize("dtype,D", [("f32", 64), ("bf16", 64), ("bf16", 776), ("f32", 20)])
+def test_row_norm_every_element_counted(dtype, D):
+    """A row with one nonzero element at position i has norm x_i^2 exactly, for every i."""
+    vals = np.zeros((D, D), np.float32)
+    vals[np.arange(D), np.arange(D)] = 1.5 + np.arange(D, dtype=np.float32) / 4
+    enc = O.encode_rne(vals, dtype)
+    n = O.row_sq_norm(O.decode(enc, dtype), O.VEC[dtype])
+    x = O.decode(enc, dtype)[np.arange(D), np.arange(D)].astype(np.float64)
+    np.testing.assert_array_equal(n.astype(np.float64), x * x)
+
+
+def test_score_nonrouted_invalid_and_nonfinite():
+    T, k, E, H, I = 4, 2, 3, 8, 8
+    idx = np.array([[0, -1], [5, 1], [2, 2], [1, 0]], np.int32)
+    w = np.full((T, k), 0.5, np.float32)
+    dY = np.ones((T, H), np.float32)
+    a = np.ones((T * k, I), np.float32)
+    a[6, 0] = np.inf            # pair (3,0): score inf
+    a[7, 1] = np.nan            # pair (3,1): score NaN
+    s, st = O.lrm_score(idx, w, dY, a, "f32", E)
+    bits = s.view(np.uint32)
+    assert bits[1] == 0 and bits[2] == 0                # not routed / invalid -> +0
+    assert st & O.ST_BAD_EXPERT and st & O.ST_NONFINITE
+    assert np.isinf(s[6]) and bits[7] == 0x7FFFFFFF
+    assert s[0] == 0.25 * 8 * 8
+
+
+# ----------------------------------------------------------------------------
+# bf16 rounding against torch's conversion
+# ----------------------------------------------------------------------------
+def test_encode_rne_matches_torch():
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal(200000).astype(np.float32) * np.float32(10.0) ** rng.integers(-40, 39, 200000)
+    # exact midpoints (ties) between neighbouring bf16 values, both parities
+    base = rng.integers(0, 0x7F00, 20000).astype(np.uint32) << 16
+    ties = (base | np.uint32(0x8000)).view(np.float32)
+    special = np.array([0.0, -0.0, np.inf, -np.inf, 3.3895313892515355e38, 1e-45, -1e-40,
+                        np.float32(3.4028235e38)], np.float32)
+    with np.errstate(over="ignore"):
+        allv = np.concatenate([v, ties, -ties, special]).astype(np.float32)
+    ref = torch.from_numpy(allv).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(O.encode_rne(allv, "bf16"), ref)
+    assert O.encode_rne(np.array([np.nan], np.float32), "bf16")[0] == 0x7FFF
+    back = O.decode(ref, "bf16")
+    np.testing.assert_array_equal(back, torch.from_numpy(allv).to(torch.bfloat16).float().numpy())
+
+
+# ----------------------------------------------------------------------------
+# T3: selection equals a brute-force sort
+# ----------------------------------------------------------------------------
+def brute_force_select(idx_flat, bits, quota, E):
+    P = idx_flat.size
+    perm = []
+    for e in range(E):
+        pairs = [p for p in range(P) if idx_flat[p] == e]
+        q = min(max(int(quota[e]), 0), len(pairs))
+        ranked = sorted(pairs, key=lambda p: (-int(bits[p]), p))
+        perm.extend(sorted(ranked[:q]))
+    return perm
+
+
+SCORE_KINDS = ["random", "ties", "all_equal", "all_zero", "nan_inf"]
+
+
+@pytest.mark.parametrize("kind", SCORE_KINDS)
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_t3_selection_brute_force(kind, seed):
+    rng = np.random.default_rng(100 + seed)
+    T, k, E = 97, 3, 7
+    idx = rng.integers(-1, E, size=(T, k)).astype(np.int32)
+    P = T * k
+    if kind == "random":
+        s = rng.random(P).astype(np.float32)
+    elif kind == "ties":
+        s = rng.integers(0, 4, P).astype(np.float32) * np.float32(0.5)
+    elif kind == "all_equal":
+        s = np.full(P, 1.25, np.float32)
+    elif kind == "all_zero":
+        s = np.zeros(P, np.float32)
+    else:
+        s = rng.random(P).astype(np.float32)
+        s[rng.integers(0, P, 20)] = np.inf
+        s.view(np.uint32)[rng.integers(0, P, 20)] = 0x7FFFFFFF
+    quota = rng.integers(-2, 40, size=E).astype(np.int32)
+    counts, kept, offsets, perm, pos, st = O.select_quota(idx, s, quota, E)
+    ref = brute_force_select(idx.reshape(-1), s.view(np.uint32), quota, E)
+    assert perm.tolist() == ref
+    assert bool(st & O.ST_BAD_QUOTA) == bool((quota < 0).any())
+
+
+# ----------------------------------------------------------------------------
+# T6 / T7: invariants and nested retained sets
+# ----------------------------------------------------------------------------
+def check_invariants(idx, score, quota, E, out):
+    counts, kept, offsets, perm, pos = out
+    flat = idx.reshape(-1)
+    bits = score.view(np.uint32)
+    for e in range(E):
+        c = int(((flat == e)).sum())
+        assert counts[e] == c
+        assert kept[e] == min(max(int(quota[e]), 0), c)
+    assert offsets[0] == 0 and (np.diff(offsets) == kept).all()
+    for e in range(E):
+        blk = perm[offsets[e]:offsets[e + 1]]
+        assert (np.diff(blk) > 0).all()
+        assert (flat[blk] == e).all()
+        dropped = np.setdiff1d(np.nonzero(flat == e)[0], blk)
+        if blk.size and dropped.size:
+            assert bits[blk].min() >= bits[dropped].max()
+    assert (pos[perm] == np.arange(perm.size)).all()
+    mask = np.ones(flat.size, bool)
+    mask[perm] = False
+    assert (pos[mask] == -1).all()
+
+
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("qwen", dict(T=256, E=16, H=64, I=64)),
+                                       ("skew", dict(T=512, E=32, H=64, I=64))])
+def test_t6_invariants(name, over):
+    L = small_layer(name, **over)
+    s, _ = O.lrm_score(L.topk_idx, L.topk_w, L.dY, L.a, L.dtype, L.spec.E)
+    out = O.select_quota(L.topk_idx, s, L.quota, L.spec.E)
+    check_invariants(L.topk_idx, s, L.quota, L.spec.E, out[:5])
+    r = O.pruned_backward(L)
+    for e in range(L.spec.E):
+        if r["kept"][e] == 0:
+            assert not r["dW_down"][e].any() and not r["dW_gu"][e].any()
+    pos = r["pos"].reshape(L.spec.T, L.spec.k)
+    none_kept = (pos < 0).all(axis=1)
+    assert not r["dX"][none_kept].any()
+
+
+def test_t7_monotone_quota():
+    L = small_layer("tiny")
+    E = L.spec.E
+    s, _ = O.lrm_score(L.topk_idx, L.topk_w, L.dY, L.a, L.dtype, E)
+    prev = set()
+    for q in range(0, int(L.counts.max()) + 2, 3):
+        quota = np.full(E, q, np.int32)
+        perm = O.select_quota(L.topk_idx, s, quota, E)[3]
+        cur = set(perm.tolist())
+        assert prev <= cur
+        prev = cur
+
+
+# ----------------------------------------------------------------------------
+# T2: full quota reproduces the unpruned dense backward
+# ----------------------------------------------------------------------------
+def _dense_inputs(L):
+    """fp64 views of a layer plus the rounded per-pair upstream gradients."""
+    dt = L.dtype
+    k = L.spec.k
+    f = lambda arr: O.decode(arr, dt).astype(np.float64)
+    w = L.topk_w.reshape(-1).astype(np.float32)
+    t = np.arange(L.spec.P) // k
+    grad = f(O.encode_rne(w[:, None] * O.decode(L.dY, dt)[t], dt))
+    return grad, f(L.x), f(L.g), f(L.u), f(L.a), f(L.W_gu), f(L.W_down)
+
+
+def rel_fro(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    d = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (d if d > 0 else 1.0)
+
+
+@pytest.mark.parametrize("name,over", [("tiny", dict(quota="full")),
+                                       ("qwen", dict(T=64, E=8, H=64, I=32, quota="full"))])
+def test_t2_full_quota_equals_dense(name, over):
+    L = small_layer(name, **over)
+    r = O.pruned_backward(L)
+    assert r["perm"].size == (L.topk_idx >= 0).sum()
+    grad, x, g, u, a, Wgu, Wd = _dense_inputs(L)
+    dWd, dWgu, dX = O.dense_backward(L.topk_idx, grad, x, g, u, a, Wgu, Wd)
+    assert rel_fro(r["dW_down"], dWd) <= 1e-12
+    assert rel_fro(r["dW_gu"], dWgu) <= 1e-12
+    assert rel_fro(r["dX"], dX) <= 1e-12
+
+
+# ----------------------------------------------------------------------------
+# T4: dropped pairs contribute exactly zero
+# ----------------------------------------------------------------------------
+def test_t4_dropped_equals_dense_with_zero_weight():
+    L = small_layer("tiny")
+    r = O.pruned_backward(L)
+    grad, x, g, u, a, Wgu, Wd = _dense_inputs(L)
+    dropped = r["pos"] < 0
+    grad[dropped] = 0.0
+    dWd, dWgu, dX = O.dense_backward(L.topk_idx, grad, x, g, u, a, Wgu, Wd)
+    assert rel_fro(r["dW_down"], dWd) <= 1e-12
+    assert rel_fro(r["dW_gu"], dWgu) <= 1e-12
+    assert rel_fro(r["dX"], dX) <= 1e-12
+
+
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("qwen", dict(T=128, E=8, H=64, I=32))])
+def test_t4_dropped_rows_never_read(name, over):
+    """NaN in the a, g, u rows of dropped pairs (after selection) changes nothing."""
+    L = small_layer(name, **over)
+    s = L.spec
+    r = O.pruned_backward(L)
+    dropped = np.nonzero(r["pos"] < 0)[0]
+    nan = O.encode_rne(np.full((1, s.I), np.nan, np.float32), s.dtype)
+    a2, g2, u2 = L.a.copy(), L.g.copy(), L.u.copy()
+    a2[dropped] = nan
+    g2[dropped] = nan
+    u2[dropped] = nan
+    Xp, DYp, Ap, Gp, Up = O.pack(r["perm"], L.topk_w, s.k, L.x, L.dY, a2, g2, u2, s.dtype)
+    dWd, dWgu, dXp, _ = O.expert_backward(Xp, DYp, Ap, Gp, Up, r["offsets"], L.W_gu, L.W_down, s.dtype)
+    dX = O.unpack(dXp, r["pos"], s.T, s.k)
+    for got, ref in ((dWd, r["dW_down"]), (dWgu, r["dW_gu"]), (dX, r["dX"])):
+        assert np.isfinite(got).all()
+        np.testing.assert_array_equal(got, ref)
+
+
+# ----------------------------------------------------------------------------
+# T5: the dense backward equals finite differences of the forward
+# ----------------------------------------------------------------------------
+def test_t5_finite_differences():
+    rng = np.random.default_rng(5)
+    T, E, k, H, I = 5, 3, 2, 6, 4
+    idx = np.array([[0, 1], [2, 0], [1, 1], [2, -1], [0, 2]], np.int32)
+    w = rng.random((T, k))
+    x = rng.standard_normal((T, H))
+    Wgu = rng.standard_normal((E, 2 * I, H)) * 0.5
+    Wd = rng.standard_normal((E, H, I)) * 0.5
+    dY = rng.standard_normal((T, H))
+
+    def loss(x_, Wgu_, Wd_):
+        Y, *_ = O.forward(idx, w, x_, Wgu_, Wd_)
+        return float((dY * Y).sum())
+
+    _, g, u, a = O.forward(idx, w, x, Wgu, Wd)
+    grad = (w.reshape(-1)[:, None] * dY[np.arange(T * k) // k])
+    dWd, dWgu, dX = O.dense_backward(idx, grad, x, g, u, a, Wgu, Wd)
+
+    h = 1e-6
+
+    def fd(arr, setter):
+        out = np.zeros_like(arr)
+        for i in np.ndindex(arr.shape):
+            plus, minus = arr.copy(), arr.copy()
+            plus[i] += h
+            minus[i] -= h
+            out[i] = (setter(plus) - setter(minus)) / (2 * h)
+        return out
+
+    fd_Wd = fd(Wd, lambda v: loss(x, Wgu, v))
+    fd_Wgu = fd(Wgu, lambda v: loss(x, v, Wd))
+    fd_x = fd(x, lambda v: loss(v, Wgu, Wd))
+    assert rel_fro(dWd, fd_Wd) < 1e-7
+    assert rel_fro(dWgu, fd_Wgu) < 1e-7
+    assert rel_fro(dX, fd_x) < 1e-7
+
+    # the pruned path in fp64 at full quota gives the same gradients
+    score = O.lrm_score_f64(idx, w, dY, a)
+    quota = np.full(E, 99, np.int32)
+    counts, kept, offsets, perm, pos, _ = O.select_quota(idx, score.astype(np.float32), quota, E)
+    Xp, DYp, Ap, Gp, Up = O.pack(perm, w.astype(np.float32), k, x, dY, a, g, u, "f64")
+    dWd2, dWgu2, dXp, _ = O.expert_backward(Xp, DYp, Ap, Gp, Up, offsets, Wgu, Wd, "f64")
+    dX2 = O.unpack(dXp, pos, T, k)
+    assert rel_fro(dWd2, fd_Wd) < 1e-7
+    assert rel_fro(dWgu2, fd_Wgu) < 1e-7
+    assert rel_fro(dX2, fd_x) < 1e-7
+
+
+def test_swiglu_derivative_closed_form():
+    """d/dg [silu(g) u] = u s (1 + g (1 - s)) against the central difference of silu."""
+    g = np.linspace(-8, 8, 401)
+    s = O.sigmoid64(g)
+    h = 1e-6
+    silu = lambda v: v / (1 + np.exp(-v))
+    fd = (silu(g + h) - silu(g - h)) / (2 * h)
+    np.testing.assert_allclose(s * (1 + g * (1 - s)), fd, rtol=1e-7, atol=1e-9)
