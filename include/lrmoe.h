@@ -1,0 +1,246 @@
+/*
+ * lrmoe.h -- C ABI of the B200 (sm_100a) pruned MoE expert backward (LRMoE).
+ *
+ * The method (three news pages on LRMoE; sections cited per entry point):
+ *   RU-B  = "LRMoE урезает обратный проход MoE и ускоряет обучение на 21–45%",
+ *           section "Что делает LRMoE: полный прямой проход, обрезанный обратный"
+ *   FR-B  = "LRMoE élague la passe arrière des MoE ...", section
+ *           "Ce que fait LRMoE : passe avant complète, passe arrière élaguée"
+ *   DE    = "LRMoE führt eine Nachkalibrierung der Last auf der Nachfrageseite ...",
+ *           paragraphs 3 and 4
+ *
+ * Notation: T tokens, E experts, k routed experts per token, H hidden size,
+ * I SwiGLU intermediate size.  Pair p = t*k + j is slot j of token t
+ * (token-major).  c_e = routed count of expert e, q_e = quota,
+ * m_e = min(max(q_e, 0), c_e) retained pairs, M = sum m_e.
+ * Expert FFN: g = x W_gate^T, u = x W_up^T, a = silu(g) * u, y = a W_down^T,
+ * layer output Y_t = sum_j w_tj y_{e(t,j)}.  Weights are stored row-major as
+ * W_gu[E][2I][H] (gate rows 0..I-1, up rows I..2I-1) and W_down[E][H][I].
+ *
+ * Conventions shared by every entry point
+ *   - Every data pointer is a DEVICE pointer, 16-byte aligned, rows contiguous
+ *     and row-major.  `stream` is a cudaStream_t passed as void* (NULL = the
+ *     legacy default stream).
+ *   - The caller owns all memory.  The library allocates nothing and keeps no
+ *     state between calls; calls are re-entrant.
+ *   - Calls only enqueue work on `stream` and never synchronise the host.
+ *     Counts and offsets stay on the device; later kernels read them there.
+ *   - Errors a host can see (null pointer, size <= 0, feature size not a
+ *     multiple of 8 elements for bf16 or 4 for fp32, too small workspace, a
+ *     failed launch) return a nonzero lrmoe_status before or instead of
+ *     launching; nothing is written then.  lrmoe_last_error() describes it.
+ *   - Errors that depend on data set bits in the optional device status word
+ *     (`status`, uint32, may be NULL) with atomicOr; kernels then continue
+ *     safely: an expert id >= E is skipped as a pair, a negative quota counts
+ *     as 0.  The caller clears the word and reads it after its own sync.
+ *   - topk_idx < 0 marks an empty slot (no pair).
+ *   - Feature sizes H, I (and the GEMM sizes K, N, N1, N2) are multiples of 8
+ *     elements for bf16 and of 4 for fp32.
+ */
+#ifndef LRMOE_H
+#define LRMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LRMOE_OK = 0,
+  LRMOE_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or enum */
+  LRMOE_ERR_UNSUPPORTED = 2,  /* valid but outside what this build handles (e.g. E > 1024) */
+  LRMOE_ERR_CUDA = 3,         /* a CUDA runtime/driver call or a launch failed */
+  LRMOE_ERR_WORKSPACE = 4     /* workspace pointer NULL or smaller than required */
+} lrmoe_status;
+
+/* Storage type of activations, gradients and weights.  Arithmetic is fp32
+ * (score, pack, unpack, fp32 GEMMs) or bf16 x bf16 -> fp32 (tensor-core GEMMs). */
+typedef enum { LRMOE_F32 = 0, LRMOE_BF16 = 1 } lrmoe_dtype;
+
+/* Epilogue of lrmoe_grouped_dgrad. */
+typedef enum {
+  LRMOE_EPI_STORE = 0,       /* out = rows . W[e], stored in the storage dtype */
+  LRMOE_EPI_SWIGLU_BWD = 1   /* out = [dG | dU] from dA = rows . W[e] and saved g, u */
+} lrmoe_epilogue;
+
+/* Device status word bits. */
+#define LRMOE_ST_BAD_EXPERT 1u /* some topk_idx >= E (that pair was skipped) */
+#define LRMOE_ST_BAD_QUOTA  2u /* some quota < 0 (treated as 0) */
+#define LRMOE_ST_NONFINITE  4u /* some score was +Inf or NaN */
+#define LRMOE_ST_TIMEOUT    8u /* a bounded device-side wait gave up; outputs invalid */
+#define LRMOE_ST_BAD_INDEX 16u /* a perm/pos entry was out of range and was skipped */
+
+/* Library version, (major << 16) | minor. */
+int lrmoe_version(void);
+
+/* Static text for a status code. */
+const char* lrmoe_status_string(int code);
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char* lrmoe_last_error(void);
+
+/* ---------------------------------------------------------------------------
+ * a1  LRM score.  RU-B bullet 3, FR-B bullet 3, DE paragraph 3: a pair's
+ * contribution to its expert's weight update is the outer product of the
+ * incoming gradient and the projection's saved input, so the squared norm of
+ * that contribution factorises into routing weight^2 * ||gradient||^2 *
+ * ||saved input||^2 and no gradient matrix is formed.
+ *
+ *   score[p] = w_p^2 * ||dY_t||^2 * ||a_p||^2     (p = t*k + j, e = topk_idx[p] in [0,E))
+ *
+ * topk_idx [T*k] int32, topk_w [T*k] fp32, dY [T][H] and a_saved [T*k][D] in
+ * dtype `dt` (a_saved is the saved input of the down projection, D = I; any
+ * other [T*k][D] saved input may be passed).  Output score [T*k] fp32; slots
+ * with topk_idx < 0 or >= E get +0.
+ * Arithmetic (bit-reproducible): each squared norm uses 32 fp32 partials, lane
+ * l summing 16-byte vectors l, l+32, ... element by element as
+ * fl(acc + fl(x*x)), then a butterfly fl(acc[l] + acc[l^o]) for o = 16..1;
+ * score = fl(fl(fl(w*w) * n_dY) * n_a).  NaN scores are written as 0x7FFFFFFF
+ * and, like +Inf, set LRMOE_ST_NONFINITE.  No fused multiply-add, no FTZ.
+ * ------------------------------------------------------------------------- */
+int lrmoe_score(const int32_t* topk_idx, const float* topk_w, int T, int k, int E,
+                const void* dY, int H, const void* a_saved, int D, lrmoe_dtype dt,
+                float* score, uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a2  Per-expert top-quota selection.  RU-B bullets 2-3, FR-B bullets 2-3,
+ * DE paragraph 3: a quota per expert is fixed for the layer call before the
+ * backward, and within it the pairs with the highest score stay.
+ *
+ * For each expert e keep the m_e = min(max(q_e,0), c_e) pairs that are
+ * largest under the key (score bit pattern as uint32 descending, p ascending).
+ * Outputs (int32, device):
+ *   counts[E]   = c_e            kept[E] = m_e
+ *   offsets[E+1]= exclusive prefix sum of m_e (offsets[E] = M)
+ *   perm[T*k]   = first M entries: packed row r holds pair perm[r]; expert
+ *                 blocks in ascending e, pairs ascending inside a block
+ *   pos[T*k]    = packed row of pair p, or -1 (dropped, empty or invalid slot)
+ * quota [E] int32 on the device.  Deterministic: integer/bitwise work only.
+ * workspace: device scratch of at least lrmoe_select_workspace_bytes(T,k,E)
+ * bytes, 256-byte aligned; its contents on entry do not matter.
+ * E <= 4096 (else LRMOE_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------- */
+size_t lrmoe_select_workspace_bytes(int T, int k, int E);
+
+int lrmoe_select_quota(const int32_t* topk_idx, const float* score, int T, int k, int E,
+                       const int32_t* quota, int32_t* counts, int32_t* kept, int32_t* offsets,
+                       int32_t* perm, int32_t* pos, void* workspace, size_t workspace_bytes,
+                       uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a3  Physical compaction.  RU-B bullet 5 and the note after it, FR-B bullet
+ * 5, DE paragraph 4: the retained gradient and activation rows are gathered
+ * into dense blocks per expert; masking rows inside full-size tensors would
+ * save neither time nor memory.
+ *
+ * For packed rows r < offsets[E] (read on the device), p = perm[r], t = p / k:
+ *   Xp[r] = x[t] (H)      DYp[r] = RNE_dt(fl(topk_w[p] * dY[t])) (H)
+ *   Ap[r] = a[p] (I)      Gp[r] = g[p] (I)       Up[r] = u[p] (I)
+ * x, dY [T][H]; a, g, u [T*k][I]; outputs [rows_cap][.] with rows_cap >= M
+ * (T*k always suffices).  Rows >= M are not touched.  A perm entry outside
+ * [0, T*k) is skipped and sets LRMOE_ST_BAD_INDEX.
+ * ------------------------------------------------------------------------- */
+int lrmoe_pack(const int32_t* perm, const int32_t* offsets, const float* topk_w, int T, int k, int E,
+               const void* x, const void* dY, int H, const void* a, const void* g, const void* u,
+               int I, lrmoe_dtype dt, void* Xp, void* DYp, void* Ap, void* Gp, void* Up,
+               int rows_cap, uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a4  Variable-size grouped GEMMs without zero padding.  RU-B bullet 5, FR-B
+ * bullet 5, DE paragraph 4 ("gruppierte GEMMs variabler Größe").  Expert e
+ * owns packed rows R_e = [offsets[e], offsets[e+1]) (offsets read on the
+ * device; m_e may be 0).
+ *
+ * lrmoe_grouped_dgrad: for each e, D = rows[R_e] (m_e x K) . W[e] (K x N)
+ *   rows [rows_cap][K], W [E][K][N] row-major, accumulate fp32.
+ *   LRMOE_EPI_STORE:      out[R_e] = D                  out [rows_cap][N]
+ *   LRMOE_EPI_SWIGLU_BWD: with s = sigmoid(g), g = Gp[R_e], u = Up[R_e] ([rows_cap][N]):
+ *       dG = D * u * s * (1 + g (1 - s)),   dU = D * g * s,
+ *       out[R_e] = [dG | dU]                            out [rows_cap][2N]
+ *   (D = dA, the gradient of the down projection's input, is never stored.)
+ *   Rows outside every R_e are not written.
+ *
+ * lrmoe_grouped_wgrad: for each e, dW[e] (N1 x N2) = grad_rows[R_e]^T . in_rows[R_e]
+ *   grad_rows [rows_cap][N1], in_rows [rows_cap][N2], dW [E][N1][N2] fp32.
+ *   accumulate = 0 overwrites dW (zeros for m_e = 0); 1 adds to it.
+ *
+ * Uses: dA/dGU  = dgrad(DYp, W_down, K=H, N=I, SWIGLU_BWD)
+ *       dW_down = wgrad(DYp, Ap, N1=H, N2=I)
+ *       dW_gu   = wgrad(dGUp, Xp, N1=2I, N2=H)
+ *       dXp     = dgrad(dGUp, W_gu, K=2I, N=H, STORE)
+ * bf16 runs on the tensor cores (bf16 operands, fp32 accumulation, bf16
+ * outputs for dgrad); fp32 runs in fp32 FFMA.  E <= 1024.
+ * ------------------------------------------------------------------------- */
+int lrmoe_grouped_dgrad(const void* rows, int rows_cap, const void* W, const int32_t* offsets,
+                        int E, int K, int N, lrmoe_dtype dt, lrmoe_epilogue epi,
+                        const void* Gp, const void* Up, void* out, uint32_t* status, void* stream);
+
+int lrmoe_grouped_wgrad(const void* grad_rows, const void* in_rows, int rows_cap,
+                        const int32_t* offsets, int E, int N1, int N2, lrmoe_dtype dt,
+                        float* dW, int accumulate, uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a5  Back to the original layout.  RU-B bullet 5, last sentence; FR-B
+ * bullet 5, last sentence.
+ *
+ *   dX[t] = RNE_dt( sum_{j ascending, pos[t*k+j] >= 0} dXp[pos[t*k+j]] )
+ * summed in fp32 and rounded once; a token with no retained pair gets 0.
+ * dXp [rows_cap][H], pos [T*k], dX [T][H].  A gather: no atomics,
+ * deterministic.  pos >= rows_cap is skipped and sets LRMOE_ST_BAD_INDEX.
+ * ------------------------------------------------------------------------- */
+int lrmoe_unpack(const void* dXp, int rows_cap, const int32_t* pos, int T, int k, int H,
+                 lrmoe_dtype dt, void* dX, uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * The whole path a1..a5 on one stream (RU-B bullets 3-5): score, selection,
+ * compaction, the four grouped GEMMs and the return to the token layout, as
+ * one enqueue with no host synchronisation.  All buffers are caller-owned
+ * device memory; rows_cap >= M (T*k always suffices).
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  /* inputs */
+  const int32_t* topk_idx;  /* [T*k] */
+  const float* topk_w;      /* [T*k] */
+  const int32_t* quota;     /* [E] */
+  const void* x;            /* [T][H] */
+  const void* dY;           /* [T][H] */
+  const void* g;            /* [T*k][I] saved gate pre-activation */
+  const void* u;            /* [T*k][I] saved up projection */
+  const void* a;            /* [T*k][I] saved down-projection input */
+  const void* W_gu;         /* [E][2I][H] */
+  const void* W_down;       /* [E][H][I] */
+  /* selection outputs */
+  float* score;             /* [T*k] */
+  int32_t* counts;          /* [E] */
+  int32_t* kept;            /* [E] */
+  int32_t* offsets;         /* [E+1] */
+  int32_t* perm;            /* [T*k] */
+  int32_t* pos;             /* [T*k] */
+  /* packed blocks and intermediates, rows_cap rows each */
+  void* Xp;                 /* [rows_cap][H] */
+  void* DYp;                /* [rows_cap][H] */
+  void* Ap;                 /* [rows_cap][I] */
+  void* Gp;                 /* [rows_cap][I] */
+  void* Up;                 /* [rows_cap][I] */
+  void* dGUp;               /* [rows_cap][2I] */
+  void* dXp;                /* [rows_cap][H] */
+  /* gradients */
+  float* dW_gu;             /* [E][2I][H] fp32 */
+  float* dW_down;           /* [E][H][I] fp32 */
+  void* dX;                 /* [T][H] */
+  /* scratch and status */
+  void* workspace;          /* >= lrmoe_select_workspace_bytes(T,k,E) */
+  size_t workspace_bytes;
+  uint32_t* status;         /* may be NULL */
+} lrmoe_buffers;
+
+int lrmoe_pruned_backward(const lrmoe_buffers* b, int T, int k, int E, int H, int I,
+                          int rows_cap, lrmoe_dtype dt, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LRMOE_H */

@@ -235,7 +235,8 @@ def expert_backward(Xp, DYp, Ap, Gp, Up, offsets, W_gu, W_down, dtype: str, expe
       dW_gu   = [dG | dU]^T X_p                     (2I x H)
       dX_p    = [dG | dU] W_gu[e]                   (m_e x H)
     Returns (dW_down [E,H,I] or dict, dW_gu, dXp [M,H], dGUp [M,2I]) in fp64.
-    `experts` restricts the weight gradients to a subset (dict keyed by e).
+    `experts` restricts the work to a subset: weight gradients come back as a
+    dict keyed by e, and the dXp / dGUp rows of other experts stay zero.
     """
     E = offsets.size - 1
     f = lambda arr: decode(arr, dtype).astype(np.float64)
@@ -250,6 +251,8 @@ def expert_backward(Xp, DYp, Ap, Gp, Up, offsets, W_gu, W_down, dtype: str, expe
     for e in range(E):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         want_w = e in sel
+        if not want_w:
+            continue
         if hi == lo:
             if want_w:
                 dW_down[e] = np.zeros((H, I))
@@ -276,9 +279,47 @@ def expert_backward(Xp, DYp, Ap, Gp, Up, offsets, W_gu, W_down, dtype: str, expe
     return dW_down, dW_gu, dXp, dGUp
 
 
+def expert_backward_rows(rows, offsets, DYp, Gp, Up, W_gu, W_down, dtype: str):
+    """dGU_p and dX_p of selected packed rows only (same formulas as expert_backward).
+
+    Each output row depends only on its own packed row and its expert's weights.
+    Returns dicts row -> fp64 vector.
+    """
+    f = lambda arr: decode(arr, dtype).astype(np.float64)
+    I = W_down.shape[2]
+    rows = np.asarray(sorted(set(int(r) for r in rows)), dtype=np.int64)
+    owner = np.searchsorted(np.asarray(offsets), rows, side="right") - 1
+    dgu, dxp = {}, {}
+    for e in np.unique(owner):
+        rs = rows[owner == e]
+        dy = f(DYp[rs])
+        g = f(Gp[rs])
+        u = f(Up[rs])
+        dA = dy @ f(W_down[e])
+        s = sigmoid64(g)
+        dGU = np.concatenate([dA * u * s * (1.0 + g * (1.0 - s)), dA * g * s], axis=1)
+        dX = dGU @ f(W_gu[e])
+        for i, r in enumerate(rs):
+            dgu[int(r)] = dGU[i]
+            dxp[int(r)] = dX[i]
+    return dgu, dxp
+
+
 # ----------------------------------------------------------------------------
 # a5: back to the token layout
 # ----------------------------------------------------------------------------
+def unpack_tokens(tokens, dxp_rows, pos, k: int, H: int):
+    """dX for selected tokens from a row -> dX_p mapping (same rule as unpack)."""
+    pos = np.asarray(pos).reshape(-1, k)
+    out = np.zeros((len(tokens), H))
+    for i, t in enumerate(tokens):
+        for j in range(k):
+            r = int(pos[t, j])
+            if r >= 0:
+                out[i] += dxp_rows[r]
+    return out
+
+
 def unpack(dXp, pos, T: int, k: int):
     """dX[t] = sum over j ascending of dX_p[pos[t*k+j]] for retained pairs; else 0."""
     H = dXp.shape[1]

@@ -1,0 +1,274 @@
+// extern "C" entry points of liblrmoe.so: argument checks, then the launchers.
+// Host-visible problems return a status code before anything is enqueued.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/lrmoe.h"
+#include "launch.h"
+
+namespace lrmoe {
+
+static thread_local char g_last_error[512] = "";
+
+static int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+static int cuda_fail(cudaError_t e, const char* where) {
+  return fail(LRMOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int elem_multiple(lrmoe_dtype dt) { return dt == LRMOE_BF16 ? 8 : 4; }
+
+static bool valid_dtype(lrmoe_dtype dt) { return dt == LRMOE_F32 || dt == LRMOE_BF16; }
+
+#define REQUIRE(cond, ...)                                 \
+  do {                                                     \
+    if (!(cond)) return fail(LRMOE_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+#define REQUIRE_PTR(p) REQUIRE((p) != nullptr && aligned16(p), "%s is null or not 16-byte aligned", #p)
+
+static int check_feature(int n, lrmoe_dtype dt, const char* name) {
+  if (n <= 0 || n % elem_multiple(dt))
+    return fail(LRMOE_ERR_INVALID_ARG, "%s=%d must be a positive multiple of %d", name, n,
+                elem_multiple(dt));
+  return LRMOE_OK;
+}
+
+static int check_pairs(int T, int k, int E) {
+  REQUIRE(T > 0 && k > 0 && E > 0, "T, k, E must be positive (T=%d k=%d E=%d)", T, k, E);
+  REQUIRE(k <= 32, "k=%d > 32 is not supported", k);
+  REQUIRE((long long)T * k < (1LL << 31) - 1, "T*k overflows int32");
+  return LRMOE_OK;
+}
+
+}  // namespace lrmoe
+
+using namespace lrmoe;
+
+extern "C" {
+
+int lrmoe_version(void) { return (1 << 16) | 0; }
+
+const char* lrmoe_status_string(int code) {
+  switch (code) {
+    case LRMOE_OK: return "ok";
+    case LRMOE_ERR_INVALID_ARG: return "invalid argument";
+    case LRMOE_ERR_UNSUPPORTED: return "unsupported";
+    case LRMOE_ERR_CUDA: return "CUDA error";
+    case LRMOE_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+const char* lrmoe_last_error(void) { return g_last_error; }
+
+int lrmoe_score(const int32_t* topk_idx, const float* topk_w, int T, int k, int E,
+                const void* dY, int H, const void* a_saved, int D, lrmoe_dtype dt,
+                float* score, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  if (int r = check_pairs(T, k, E)) return r;
+  if (int r = check_feature(H, dt, "H")) return r;
+  if (int r = check_feature(D, dt, "D")) return r;
+  REQUIRE_PTR(topk_idx);
+  REQUIRE_PTR(topk_w);
+  REQUIRE_PTR(dY);
+  REQUIRE_PTR(a_saved);
+  REQUIRE_PTR(score);
+  cudaError_t e = launch_score(topk_idx, topk_w, T, k, E, dY, H, a_saved, D, dt, score, status,
+                               static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_score launch");
+}
+
+size_t lrmoe_select_workspace_bytes(int T, int k, int E) {
+  if (T <= 0 || k <= 0 || E <= 0) return 0;
+  return select_ws_layout(T, k, E).total;
+}
+
+int lrmoe_select_quota(const int32_t* topk_idx, const float* score, int T, int k, int E,
+                       const int32_t* quota, int32_t* counts, int32_t* kept, int32_t* offsets,
+                       int32_t* perm, int32_t* pos, void* workspace, size_t workspace_bytes,
+                       uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  if (int r = check_pairs(T, k, E)) return r;
+  if (E > 4096) return fail(LRMOE_ERR_UNSUPPORTED, "E=%d > 4096", E);
+  REQUIRE_PTR(topk_idx);
+  REQUIRE_PTR(score);
+  REQUIRE_PTR(quota);
+  REQUIRE_PTR(counts);
+  REQUIRE_PTR(kept);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(perm);
+  REQUIRE_PTR(pos);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(LRMOE_ERR_WORKSPACE, "workspace is null or not 256-byte aligned");
+  const size_t need = select_ws_layout(T, k, E).total;
+  if (workspace_bytes < need)
+    return fail(LRMOE_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, need);
+  cudaError_t e = launch_select(topk_idx, score, T, k, E, quota, counts, kept, offsets, perm, pos,
+                                workspace, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_select_quota launch");
+}
+
+int lrmoe_pack(const int32_t* perm, const int32_t* offsets, const float* topk_w, int T, int k, int E,
+               const void* x, const void* dY, int H, const void* a, const void* g, const void* u,
+               int I, lrmoe_dtype dt, void* Xp, void* DYp, void* Ap, void* Gp, void* Up,
+               int rows_cap, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  if (int r = check_pairs(T, k, E)) return r;
+  if (int r = check_feature(H, dt, "H")) return r;
+  if (int r = check_feature(I, dt, "I")) return r;
+  REQUIRE(rows_cap > 0, "rows_cap must be positive");
+  REQUIRE_PTR(perm);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(topk_w);
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(dY);
+  REQUIRE_PTR(a);
+  REQUIRE_PTR(g);
+  REQUIRE_PTR(u);
+  REQUIRE_PTR(Xp);
+  REQUIRE_PTR(DYp);
+  REQUIRE_PTR(Ap);
+  REQUIRE_PTR(Gp);
+  REQUIRE_PTR(Up);
+  cudaError_t e = launch_pack(perm, offsets, topk_w, T, k, E, x, dY, H, a, g, u, I, dt, Xp, DYp, Ap,
+                              Gp, Up, rows_cap, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_pack launch");
+}
+
+int lrmoe_grouped_dgrad(const void* rows, int rows_cap, const void* W, const int32_t* offsets,
+                        int E, int K, int N, lrmoe_dtype dt, lrmoe_epilogue epi,
+                        const void* Gp, const void* Up, void* out, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  REQUIRE(epi == LRMOE_EPI_STORE || epi == LRMOE_EPI_SWIGLU_BWD, "unknown epilogue %d", (int)epi);
+  REQUIRE(E > 0 && rows_cap > 0, "E and rows_cap must be positive");
+  if (E > kMaxGroupedExperts) return fail(LRMOE_ERR_UNSUPPORTED, "E=%d > %d", E, kMaxGroupedExperts);
+  if (int r = check_feature(K, dt, "K")) return r;
+  if (int r = check_feature(N, dt, "N")) return r;
+  REQUIRE_PTR(rows);
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(out);
+  if (epi == LRMOE_EPI_SWIGLU_BWD) {
+    REQUIRE_PTR(Gp);
+    REQUIRE_PTR(Up);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dt == LRMOE_BF16) {
+    const char* why = "launch failed";
+    e = launch_dgrad_tc(rows, rows_cap, W, offsets, E, K, N, epi, Gp, Up, out, status, s, &why);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+  } else {
+    e = launch_dgrad_simt(rows, rows_cap, W, offsets, E, K, N, dt, epi, Gp, Up, out, status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "lrmoe_grouped_dgrad launch");
+  }
+  return LRMOE_OK;
+}
+
+int lrmoe_grouped_wgrad(const void* grad_rows, const void* in_rows, int rows_cap,
+                        const int32_t* offsets, int E, int N1, int N2, lrmoe_dtype dt, float* dW,
+                        int accumulate, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  REQUIRE(E > 0 && rows_cap > 0, "E and rows_cap must be positive");
+  if (E > kMaxGroupedExperts) return fail(LRMOE_ERR_UNSUPPORTED, "E=%d > %d", E, kMaxGroupedExperts);
+  if (int r = check_feature(N1, dt, "N1")) return r;
+  if (int r = check_feature(N2, dt, "N2")) return r;
+  REQUIRE_PTR(grad_rows);
+  REQUIRE_PTR(in_rows);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(dW);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dt == LRMOE_BF16) {
+    const char* why = "launch failed";
+    e = launch_wgrad_tc(grad_rows, in_rows, rows_cap, offsets, E, N1, N2, dW, accumulate, status, s,
+                        &why);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+  } else {
+    e = launch_wgrad_simt(grad_rows, in_rows, rows_cap, offsets, E, N1, N2, dt, dW, accumulate,
+                          status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "lrmoe_grouped_wgrad launch");
+  }
+  return LRMOE_OK;
+}
+
+int lrmoe_unpack(const void* dXp, int rows_cap, const int32_t* pos, int T, int k, int H,
+                 lrmoe_dtype dt, void* dX, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  REQUIRE(T > 0 && k > 0 && rows_cap > 0, "T, k, rows_cap must be positive");
+  REQUIRE(k <= 32, "k=%d > 32 is not supported", k);
+  if (int r = check_feature(H, dt, "H")) return r;
+  REQUIRE_PTR(dXp);
+  REQUIRE_PTR(pos);
+  REQUIRE_PTR(dX);
+  cudaError_t e = launch_unpack(dXp, rows_cap, pos, T, k, H, dt, dX, status,
+                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_unpack launch");
+}
+
+int lrmoe_pruned_backward(const lrmoe_buffers* b, int T, int k, int E, int H, int I,
+                          int rows_cap, lrmoe_dtype dt, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(b != nullptr, "buffers is null");
+  REQUIRE(rows_cap > 0, "rows_cap must be positive");
+  int r;
+  if ((r = lrmoe_score(b->topk_idx, b->topk_w, T, k, E, b->dY, H, b->a, I, dt, b->score, b->status,
+                       stream)))
+    return r;
+  if ((r = lrmoe_select_quota(b->topk_idx, b->score, T, k, E, b->quota, b->counts, b->kept,
+                              b->offsets, b->perm, b->pos, b->workspace, b->workspace_bytes,
+                              b->status, stream)))
+    return r;
+  if ((r = lrmoe_pack(b->perm, b->offsets, b->topk_w, T, k, E, b->x, b->dY, H, b->a, b->g, b->u, I,
+                      dt, b->Xp, b->DYp, b->Ap, b->Gp, b->Up, rows_cap, b->status, stream)))
+    return r;
+  // dA -> [dG | dU]  (m_e x H) . (H x I), SwiGLU backward in the epilogue
+  if ((r = lrmoe_grouped_dgrad(b->DYp, rows_cap, b->W_down, b->offsets, E, H, I, dt,
+                               LRMOE_EPI_SWIGLU_BWD, b->Gp, b->Up, b->dGUp, b->status, stream)))
+    return r;
+  // dW_down = DY_p^T A_p
+  if ((r = lrmoe_grouped_wgrad(b->DYp, b->Ap, rows_cap, b->offsets, E, H, I, dt, b->dW_down, 0,
+                               b->status, stream)))
+    return r;
+  // dW_gu = dGU_p^T X_p
+  if ((r = lrmoe_grouped_wgrad(b->dGUp, b->Xp, rows_cap, b->offsets, E, 2 * I, H, dt, b->dW_gu, 0,
+                               b->status, stream)))
+    return r;
+  // dX_p = dGU_p W_gu
+  if ((r = lrmoe_grouped_dgrad(b->dGUp, rows_cap, b->W_gu, b->offsets, E, 2 * I, H, dt,
+                               LRMOE_EPI_STORE, nullptr, nullptr, b->dXp, b->status, stream)))
+    return r;
+  return lrmoe_unpack(b->dXp, rows_cap, b->pos, T, k, H, dt, b->dX, b->status, stream);
+}
+
+}  // extern "C"

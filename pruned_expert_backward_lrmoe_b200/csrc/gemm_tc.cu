@@ -1,0 +1,483 @@
+// a4 for bf16 storage: variable-size grouped GEMMs on the sm_100a tensor cores.
+//
+// "LRMoE урезает обратный проход MoE ...", section "Что делает LRMoE", bullet 5
+// (German page, paragraph 4: "gruppierte GEMMs variabler Größe"): the expert
+// gradients are computed as grouped GEMMs over the compacted per-expert blocks
+// with no zero padding.
+//
+// One persistent, warp-specialised kernel serves both shapes:
+//   dgrad (variable M): D[R_e, :] = rows[R_e] (m_e x K) . W[e] (K x N)
+//          A = rows, K-major;   B = W[e], N-major;  epilogue STORE or SwiGLU-bwd
+//   wgrad (variable K): D = grad[R_e]^T (N1 x m_e) . in[R_e] (m_e x N2)
+//          A = grad, M-major;   B = in, N-major;    epilogue fp32 store / add
+// Roles (192 threads): warp 0 issues TMA loads into a ring of shared-memory
+// stages; warp 1 owns tensor memory and one lane issues tcgen05.mma (128 x BN
+// x 16 per instruction, fp32 accumulators in TMEM, two accumulator buffers so
+// that the epilogue of one tile overlaps the main loop of the next); warps 2-5
+// drain TMEM with tcgen05.ld and store.  Group sizes are read on the device.
+// In wgrad the last K block of an expert may reach into the next expert's
+// rows: those rows are zeroed in shared memory before the MMAs read them.
+// Every mbarrier wait is bounded (LRMOE_ST_TIMEOUT, then a clean exit).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "grouped.cuh"
+#include "launch.h"
+
+namespace lrmoe {
+namespace {
+
+constexpr int BM = 128;        // tile rows = TMEM lanes
+constexpr int BK = 64;         // 64 bf16 = one 128-byte swizzle row
+constexpr int UK = 16;         // K of one kind::f16 MMA
+constexpr int kThreads = 192;  // TMA warp, MMA warp, 4 epilogue warps
+constexpr int kEpiThreads = 128;
+
+enum Mode : int { kDgradStore = 0, kDgradSwiglu = 1, kWgrad = 2 };
+
+template <int BN, int STAGES>
+struct Layout {
+  static constexpr int kABytes = BM * BK * 2;                 // 16 KB
+  static constexpr int kBBytes = BN * BK * 2;                 // 32 KB at BN = 256
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTilesBytes = STAGES * kStageBytes;
+  static constexpr int kTableInts = 2 * (kMaxExperts + 1) + 33;
+  static constexpr int kBarOff = kTilesBytes;                 // 8-byte barriers
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;     // tmem base, abort flag
+  static constexpr int kTableOff = kMiscOff + 16;
+  static constexpr int kBytes = kTableOff + kTableInts * 4;
+  static constexpr int kAlloc = kBytes + 1024;                // slack for 1024-B alignment
+};
+
+struct TileInfo {
+  int e;       // expert
+  int row0;    // dgrad: first packed row of the tile; wgrad: first packed row of the expert
+  int row_end; // end of the expert's rows
+  int m0, n0;  // output tile origin (dgrad: m0 unused)
+  int nk;      // number of K blocks
+};
+
+template <int MODE, int BN>
+__device__ __forceinline__ TileInfo decode_tile(int t, const int32_t* __restrict__ offsets,
+                                                const int* tab0, int E, int K, int n_tiles,
+                                                int m_tiles) {
+  TileInfo ti;
+  if constexpr (MODE == kWgrad) {
+    const int per_e = m_tiles * n_tiles;
+    const int oi = t / per_e, local = t - oi * per_e;
+    ti.e = tab0[oi];
+    ti.m0 = (local / n_tiles) * BM;
+    ti.n0 = (local % n_tiles) * BN;
+    ti.row0 = offsets[ti.e];
+    ti.row_end = offsets[ti.e + 1];
+    ti.nk = (ti.row_end - ti.row0 + BK - 1) / BK;
+  } else {
+    const int e = find_group(tab0, E, t);
+    const int local = t - tab0[e];
+    ti.e = e;
+    ti.m0 = 0;
+    ti.n0 = (local % n_tiles) * BN;
+    ti.row0 = offsets[e] + (local / n_tiles) * BM;
+    ti.row_end = offsets[e + 1];
+    ti.nk = (K + BK - 1) / BK;
+  }
+  return ti;
+}
+
+__device__ __forceinline__ float sigmoid_fast(float x) { return 1.0f / (1.0f + __expf(-x)); }
+
+template <int MODE, int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const int32_t* __restrict__ offsets, int E, int K, int N /* dgrad N or wgrad N2 */,
+    int N1 /* wgrad only */, const uint16_t* __restrict__ Gp, const uint16_t* __restrict__ Up,
+    void* __restrict__ out, int accumulate, uint32_t* __restrict__ status) {
+  using L = Layout<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;      // [2]
+  uint64_t* tempty = bars + 2 * STAGES + 2; // [2]
+  uint64_t* mma_done = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  int* tab0 = reinterpret_cast<int*>(smem + L::kTableOff);
+  int* tab1 = tab0 + (kMaxExperts + 1);
+  int* scratch = tab1 + (kMaxExperts + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], kEpiThreads);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * BN);
+    tmem_relinquish();
+  }
+  // tile table
+  const int n_tiles = (N + BN - 1) / BN;
+  int m_tiles = 0, total;
+  if constexpr (MODE == kWgrad) {
+    m_tiles = (N1 + BM - 1) / BM;
+    build_wgrad_order(offsets, E, tab0, tab1);
+    total = E * m_tiles * n_tiles;
+  } else {
+    total = build_dgrad_tiles(offsets, E, BM, n_tiles, tab0, scratch);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+        const TileInfo ti = decode_tile<MODE, BN>(t, offsets, tab0, E, K, n_tiles, m_tiles);
+        for (int kb = 0; kb < ti.nk; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status)) break;
+          uint8_t* sa = smem + stage * L::kStageBytes;
+          uint8_t* sb = sa + L::kABytes;
+          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+          if constexpr (MODE == kWgrad) {
+            const int r = ti.row0 + kb * BK;
+            tma_load_2d(sa, &tmA, &full[stage], ti.m0, r);
+            tma_load_2d(sa + 8192, &tmA, &full[stage], ti.m0 + 64, r);
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(sb + c * 8192, &tmB, &full[stage], ti.n0 + c * 64, r);
+          } else {
+            tma_load_2d(sa, &tmA, &full[stage], kb * BK, ti.row0);
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_3d(sb + c * 8192, &tmB, &full[stage], ti.n0 + c * 64, kb * BK, ti.e);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, MODE == kWgrad, true);
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t acc_iter = 0;
+    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+      const TileInfo ti = decode_tile<MODE, BN>(t, offsets, tab0, E, K, n_tiles, m_tiles);
+      if (ti.nk == 0) continue;
+      const uint32_t b = acc_iter & 1u, bphase = (acc_iter >> 1) & 1u;
+      if (!__all_sync(kFull, mbar_wait_bounded(&tempty[b], bphase ^ 1u, abort_flag, status)))
+        break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + b * BN;
+      bool ok = true;
+      for (int kb = 0; kb < ti.nk; ++kb) {
+        if (!__all_sync(kFull, mbar_wait_bounded(&full[stage], phase, abort_flag, status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint8_t* sa = smem + stage * L::kStageBytes;
+        uint8_t* sb = sa + L::kABytes;
+        if constexpr (MODE == kWgrad) {
+          const int valid = ti.row_end - (ti.row0 + kb * BK);
+          if (valid < BK) {
+            // zero the K rows that belong to the next expert (or lie past the data)
+            const int nchunk = 2 + BN / 64;
+            const int rows_bad = BK - valid;
+            const int n16 = nchunk * rows_bad * 8;  // 16-byte pieces
+            for (int i = lane; i < n16; i += 32) {
+              const int ch = i / (rows_bad * 8);
+              const int rem = i - ch * rows_bad * 8;
+              const int row = valid + rem / 8;
+              const int piece = rem & 7;
+              uint8_t* base = ch < 2 ? sa + ch * 8192 : sb + (ch - 2) * 8192;
+              *reinterpret_cast<uint4*>(base + row * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+        }
+        if (lane == 0) {
+          const uint32_t a_addr = smem_u32(sa), b_addr = smem_u32(sb);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk) {
+            uint64_t adesc, bdesc;
+            if constexpr (MODE == kWgrad)
+              adesc = smem_desc_sw128(a_addr + kk * 2048, 8192, 1024);
+            else
+              adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+            bdesc = smem_desc_sw128(b_addr + kk * 2048, 8192, 1024);
+            tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(&tfull[b]);
+      __syncwarp();
+      ++acc_iter;
+    }
+    // make sure every issued MMA has finished before tensor memory is released
+    if (lane == 0) tc_commit(mma_done);
+    __syncwarp();
+    mbar_wait_bounded(mma_done, 0, abort_flag, status);
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = q * 32 + lane;
+    uint32_t acc_iter = 0;
+    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+      const TileInfo ti = decode_tile<MODE, BN>(t, offsets, tab0, E, K, n_tiles, m_tiles);
+      if constexpr (MODE == kWgrad) {
+        float* dW = static_cast<float*>(out) + (size_t)ti.e * N1 * N;
+        const int m = ti.m0 + row_in_tile;
+        if (ti.nk == 0) {
+          if (!accumulate && m < N1) {
+            for (int c = 0; c < BN; c += 4) {
+              const int n = ti.n0 + c;
+              if (n < N)
+                *reinterpret_cast<uint4*>(dW + (size_t)m * N + n) = make_uint4(0, 0, 0, 0);
+            }
+          }
+          continue;
+        }
+        const uint32_t b = acc_iter & 1u, bphase = (acc_iter >> 1) & 1u;
+        if (!__all_sync(kFull, mbar_wait_bounded(&tfull[b], bphase, abort_flag, status))) break;
+        tc_fence_after();
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + b * BN + ch * 32, r);
+          tmem_wait_ld();
+          if (m < N1) {
+            float* dst = dW + (size_t)m * N + ti.n0 + ch * 32;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              if (ti.n0 + ch * 32 + v * 4 < N) {
+                float4 o = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                       __uint_as_float(r[4 * v + 2]),
+                                       __uint_as_float(r[4 * v + 3]));
+                if (accumulate) {
+                  const float4 old = *reinterpret_cast<const float4*>(dst + 4 * v);
+                  o.x += old.x;
+                  o.y += old.y;
+                  o.z += old.z;
+                  o.w += old.w;
+                }
+                *reinterpret_cast<float4*>(dst + 4 * v) = o;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[b]);
+        ++acc_iter;
+      } else {
+        const uint32_t b = acc_iter & 1u, bphase = (acc_iter >> 1) & 1u;
+        if (!__all_sync(kFull, mbar_wait_bounded(&tfull[b], bphase, abort_flag, status))) break;
+        tc_fence_after();
+        const int row = ti.row0 + row_in_tile;
+        const bool row_ok = row < ti.row_end;
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + b * BN + ch * 32, r);
+          tmem_wait_ld();
+          if (!row_ok) continue;
+          const int nb = ti.n0 + ch * 32;
+          if constexpr (MODE == kDgradStore) {
+            uint16_t* o = static_cast<uint16_t*>(out) + (size_t)row * N + nb;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (nb + v * 8 < N) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+                w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+                w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+                w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+                *reinterpret_cast<uint4*>(o + v * 8) = w;
+              }
+            }
+          } else {
+            const uint16_t* gp = Gp + (size_t)row * N + nb;
+            const uint16_t* up = Up + (size_t)row * N + nb;
+            uint16_t* og = static_cast<uint16_t*>(out) + (size_t)row * 2 * N + nb;
+            uint16_t* ou = og + N;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (nb + v * 8 < N) {
+                const uint4 gv = *reinterpret_cast<const uint4*>(gp + v * 8);
+                const uint4 uv = *reinterpret_cast<const uint4*>(up + v * 8);
+                const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+                const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
+                uint32_t dg[4], du[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  float res_g[2], res_u[2];
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {
+                    const float da = __uint_as_float(r[8 * v + 2 * i + h]);
+                    const float g = bf16_bits_to_f32(h ? (gw[i] >> 16) : (gw[i] & 0xffffu));
+                    const float u = bf16_bits_to_f32(h ? (uw[i] >> 16) : (uw[i] & 0xffffu));
+                    const float s = sigmoid_fast(g);
+                    res_g[h] = da * u * s * (1.0f + g * (1.0f - s));
+                    res_u[h] = da * g * s;
+                  }
+                  dg[i] = pack_bf16x2(res_g[0], res_g[1]);
+                  du[i] = pack_bf16x2(res_u[0], res_u[1]);
+                }
+                *reinterpret_cast<uint4*>(og + v * 8) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+                *reinterpret_cast<uint4*>(ou + v * 8) = make_uint4(du[0], du[1], du[2], du[3]);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[b]);
+        ++acc_iter;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, 2 * BN);
+}
+
+// ---------------------------------------------------------------------------
+// host: tensor maps
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 map over a row-major [rows][cols] matrix, box = box_cols x box_rows, 128-B swizzle.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                 uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D bf16 map over [E][K][N], box = 64 (N) x 64 (K) x 1, 128-B swizzle.
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t N) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {N, K, E};
+  cuuint64_t strides[2] = {N * 2, K * N * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kBN = 256;
+constexpr int kStages = 4;
+
+template <int MODE>
+cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const int32_t* offsets,
+                        int E, int K, int N, int N1, const void* Gp, const void* Up, void* out,
+                        int accumulate, uint32_t* status, cudaStream_t s, int grid) {
+  using L = Layout<kBN, kStages>;
+  static unsigned long long attr_done = 0;  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tc<MODE, kBN, kStages>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (err != cudaSuccess) return err;
+    attr_done |= 1ull << dev;
+  }
+  grouped_gemm_tc<MODE, kBN, kStages><<<grid, kThreads, L::kAlloc, s>>>(
+      ta, tb, offsets, E, K, N, N1, static_cast<const uint16_t*>(Gp),
+      static_cast<const uint16_t*>(Up), out, accumulate, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
+                            const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
+                            const void* Gp, const void* Up, void* out, uint32_t* status,
+                            cudaStream_t s, const char** why) {
+  CUtensorMap ta, tb;
+  if (!make_map_2d(&ta, rows, (uint64_t)rows_cap, (uint64_t)K, 64, 128) ||
+      !make_map_3d(&tb, W, (uint64_t)E, (uint64_t)K, (uint64_t)N)) {
+    *why = "cuTensorMapEncodeTiled failed for a dgrad operand";
+    return cudaErrorInvalidValue;
+  }
+  const int grid = num_sms();
+  if (epi == LRMOE_EPI_SWIGLU_BWD)
+    return launch_mode<kDgradSwiglu>(ta, tb, offsets, E, K, N, 0, Gp, Up, out, 0, status, s, grid);
+  return launch_mode<kDgradStore>(ta, tb, offsets, E, K, N, 0, nullptr, nullptr, out, 0, status, s,
+                                  grid);
+}
+
+cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows_cap,
+                            const int32_t* offsets, int E, int N1, int N2, float* dW,
+                            int accumulate, uint32_t* status, cudaStream_t s, const char** why) {
+  CUtensorMap ta, tb;
+  if (!make_map_2d(&ta, grad_rows, (uint64_t)rows_cap, (uint64_t)N1, 64, 64) ||
+      !make_map_2d(&tb, in_rows, (uint64_t)rows_cap, (uint64_t)N2, 64, 64)) {
+    *why = "cuTensorMapEncodeTiled failed for a wgrad operand";
+    return cudaErrorInvalidValue;
+  }
+  const long long total =
+      (long long)E * ((N1 + BM - 1) / BM) * ((N2 + kBN - 1) / kBN);
+  int grid = num_sms();
+  if (total < grid) grid = (int)total;
+  return launch_mode<kWgrad>(ta, tb, offsets, E, 0, N2, N1, nullptr, nullptr, dW, accumulate,
+                             status, s, grid);
+}
+
+}  // namespace lrmoe

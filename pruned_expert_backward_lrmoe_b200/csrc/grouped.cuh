@@ -1,0 +1,91 @@
+// Device-side tile bookkeeping of the variable-size grouped GEMMs.
+//
+// Expert e owns packed rows [offsets[e], offsets[e+1]).  The group sizes stay
+// on the device, so every persistent CTA rebuilds the tile table from
+// `offsets` in shared memory at start-up (E <= kMaxExperts) and walks the
+// same tile sequence; no host synchronisation and no zero padding.
+#pragma once
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace lrmoe {
+
+constexpr int kMaxExperts = kMaxGroupedExperts;
+
+// Exclusive scan of v[0..n) in place (shared memory), block-wide; returns total.
+__device__ __forceinline__ int block_scan_inplace(int* v, int n, int* scratch /*[33]*/) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int b = tid * per;
+  int s = 0;
+  for (int i = 0; i < per; ++i)
+    if (b + i < n) s += v[b + i];
+  const int incl = warp_incl_scan(s);
+  if (lane == 31) scratch[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    const int x = lane < nw ? scratch[lane] : 0;
+    const int xi = warp_incl_scan(x);
+    if (lane < nw) scratch[lane] = xi - x;
+    if (lane == 31) scratch[32] = xi;
+  }
+  __syncthreads();
+  int run = scratch[wid] + incl - s;
+  for (int i = 0; i < per; ++i)
+    if (b + i < n) {
+      const int t = v[b + i];
+      v[b + i] = run;
+      run += t;
+    }
+  const int total = scratch[32];
+  __syncthreads();
+  return total;
+}
+
+// dgrad (variable M): tiles of expert e = ceil(m_e / BM) * n_tiles, experts in order.
+// tstart[0..E] receives the exclusive prefix; returns the total tile count.
+__device__ __forceinline__ int build_dgrad_tiles(const int32_t* __restrict__ offsets, int E,
+                                                 int BM, int n_tiles, int* tstart,
+                                                 int* scratch) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int m = offsets[e + 1] - offsets[e];
+    tstart[e] = m > 0 ? ((m + BM - 1) / BM) * n_tiles : 0;
+  }
+  __syncthreads();
+  const int total = block_scan_inplace(tstart, E, scratch);
+  if (threadIdx.x == 0) tstart[E] = total;
+  __syncthreads();
+  return total;
+}
+
+// Largest e with tstart[e] <= t (tstart non-decreasing, tstart[0] = 0).
+__device__ __forceinline__ int find_group(const int* tstart, int E, int t) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tstart[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// wgrad (variable K): every expert has the same tiles; experts are visited in
+// descending m_e (ties by ascending e) so that the longest K loops start first.
+// order[0..E) receives the expert sequence.
+__device__ __forceinline__ void build_wgrad_order(const int32_t* __restrict__ offsets, int E,
+                                                  int* order, int* msz) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) msz[e] = offsets[e + 1] - offsets[e];
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int me = msz[e];
+    int rank = 0;
+    for (int f = 0; f < E; ++f) {
+      const int mf = msz[f];
+      rank += (mf > me) || (mf == me && f < e);
+    }
+    order[rank] = e;
+  }
+  __syncthreads();
+}
+
+}  // namespace lrmoe

@@ -1,0 +1,61 @@
+// Internal launchers behind the C ABI (host side).  Arguments are already
+// validated by abi.cu; each launcher only enqueues kernels on `s`.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/lrmoe.h"
+
+namespace lrmoe {
+
+// Largest expert count the grouped GEMMs build their tile table for.
+constexpr int kMaxGroupedExperts = 1024;
+
+int num_sms();
+
+cudaError_t launch_score(const int32_t* idx, const float* w, int T, int k, int E, const void* dY,
+                         int H, const void* a, int D, lrmoe_dtype dt, float* score,
+                         uint32_t* status, cudaStream_t s);
+
+struct SelectWs {
+  int chunk;        // pairs per chunk
+  int nchunks;
+  size_t off_cc, off_seg_start, off_seg_p, off_seg_key, total;
+};
+SelectWs select_ws_layout(int T, int k, int E);
+
+cudaError_t launch_select(const int32_t* idx, const float* score, int T, int k, int E,
+                          const int32_t* quota, int32_t* counts, int32_t* kept, int32_t* offsets,
+                          int32_t* perm, int32_t* pos, void* ws, uint32_t* status,
+                          cudaStream_t s);
+
+cudaError_t launch_pack(const int32_t* perm, const int32_t* offsets, const float* w, int T,
+                        int k, int E, const void* x, const void* dY, int H, const void* a,
+                        const void* g, const void* u, int I, lrmoe_dtype dt, void* Xp, void* DYp,
+                        void* Ap, void* Gp, void* Up, int rows_cap, uint32_t* status,
+                        cudaStream_t s);
+
+cudaError_t launch_unpack(const void* dXp, int rows_cap, const int32_t* pos, int T, int k, int H,
+                          lrmoe_dtype dt, void* dX, uint32_t* status, cudaStream_t s);
+
+// fp32 FFMA grouped GEMMs (fp32 storage)
+cudaError_t launch_dgrad_simt(const void* rows, int rows_cap, const void* W,
+                              const int32_t* offsets, int E, int K, int N, lrmoe_dtype dt,
+                              lrmoe_epilogue epi, const void* Gp, const void* Up, void* out,
+                              uint32_t* status, cudaStream_t s);
+cudaError_t launch_wgrad_simt(const void* grad_rows, const void* in_rows, int rows_cap,
+                              const int32_t* offsets, int E, int N1, int N2, lrmoe_dtype dt,
+                              float* dW, int accumulate, uint32_t* status, cudaStream_t s);
+
+// tcgen05 grouped GEMMs (bf16 storage)
+cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
+                            const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
+                            const void* Gp, const void* Up, void* out, uint32_t* status,
+                            cudaStream_t s, const char** why);
+cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows_cap,
+                            const int32_t* offsets, int E, int N1, int N2, float* dW,
+                            int accumulate, uint32_t* status, cudaStream_t s, const char** why);
+
+}  // namespace lrmoe

@@ -1,0 +1,197 @@
+// a3  Physical compaction and a5  return to the token layout.
+//
+// "LRMoE урезает обратный проход MoE ...", section "Что делает LRMoE", bullet 5
+// and the note after it: retained gradient and activation rows are gathered
+// into dense per-expert blocks (masking rows inside full-size tensors would
+// save nothing), and the result then goes back to the original layout.
+//
+// Both are HBM-bound row gathers.  One warp per row, 16 bytes per lane per
+// access; persistent grid-stride loops, since the retained-row count M lives
+// on the device (offsets[E]) and is never read back by the host.
+#include "common.cuh"
+#include "launch.h"
+
+namespace lrmoe {
+namespace {
+
+__device__ __forceinline__ void copy_row(uint4* __restrict__ dst, const uint4* __restrict__ src,
+                                         int V, int lane) {
+  int c = lane;
+  for (; c + 96 < V; c += 128) {
+    const uint4 v0 = __ldg(src + c), v1 = __ldg(src + c + 32), v2 = __ldg(src + c + 64),
+                v3 = __ldg(src + c + 96);
+    dst[c] = v0;
+    dst[c + 32] = v1;
+    dst[c + 64] = v2;
+    dst[c + 96] = v3;
+  }
+  for (; c < V; c += 32) dst[c] = __ldg(src + c);
+}
+
+template <lrmoe_dtype DT>
+__device__ __forceinline__ uint4 scale_vec(uint4 v, float w) {
+  if constexpr (DT == LRMOE_BF16) {
+    uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = f32_to_bf16_bits_rne(__fmul_rn(w, bf16_bits_to_f32(in[i] & 0xffffu)));
+      const uint32_t hi = f32_to_bf16_bits_rne(__fmul_rn(w, bf16_bits_to_f32(in[i] >> 16)));
+      out[i] = lo | (hi << 16);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+  } else {
+    return make_uint4(__float_as_uint(__fmul_rn(w, __uint_as_float(v.x))),
+                      __float_as_uint(__fmul_rn(w, __uint_as_float(v.y))),
+                      __float_as_uint(__fmul_rn(w, __uint_as_float(v.z))),
+                      __float_as_uint(__fmul_rn(w, __uint_as_float(v.w))));
+  }
+}
+
+template <lrmoe_dtype DT>
+__device__ __forceinline__ void scale_row(uint4* __restrict__ dst, const uint4* __restrict__ src,
+                                          int V, float w, int lane) {
+  int c = lane;
+  for (; c + 96 < V; c += 128) {
+    const uint4 v0 = __ldg(src + c), v1 = __ldg(src + c + 32), v2 = __ldg(src + c + 64),
+                v3 = __ldg(src + c + 96);
+    dst[c] = scale_vec<DT>(v0, w);
+    dst[c + 32] = scale_vec<DT>(v1, w);
+    dst[c + 64] = scale_vec<DT>(v2, w);
+    dst[c + 96] = scale_vec<DT>(v3, w);
+  }
+  for (; c < V; c += 32) dst[c] = scale_vec<DT>(__ldg(src + c), w);
+}
+
+template <lrmoe_dtype DT>
+__global__ void __launch_bounds__(256) pack_kernel(
+    const int32_t* __restrict__ perm, const int32_t* __restrict__ offsets, int E,
+    const float* __restrict__ w, int P, int k, const uint4* __restrict__ x,
+    const uint4* __restrict__ dY, int VH, const uint4* __restrict__ a,
+    const uint4* __restrict__ g, const uint4* __restrict__ u, int VI, uint4* __restrict__ Xp,
+    uint4* __restrict__ DYp, uint4* __restrict__ Ap, uint4* __restrict__ Gp,
+    uint4* __restrict__ Up, int rows_cap, uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  int M = offsets[E];
+  if (M > rows_cap) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
+    M = rows_cap;
+  }
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < M; r += gridDim.x * wpb) {
+    const int p = perm[r];
+    if (p < 0 || p >= P) {
+      if (lane == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
+      continue;
+    }
+    const int t = p / k;
+    const float wp = __ldg(w + p);
+    const size_t rr = (size_t)r;
+    copy_row(Xp + rr * VH, x + (size_t)t * VH, VH, lane);
+    scale_row<DT>(DYp + rr * VH, dY + (size_t)t * VH, VH, wp, lane);
+    copy_row(Ap + rr * VI, a + (size_t)p * VI, VI, lane);
+    copy_row(Gp + rr * VI, g + (size_t)p * VI, VI, lane);
+    copy_row(Up + rr * VI, u + (size_t)p * VI, VI, lane);
+  }
+}
+
+// dX[t] = sum over retained slots j (ascending) of dXp[pos[t*k+j]], fp32, rounded once.
+template <lrmoe_dtype DT>
+__global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ dXp, int rows_cap,
+                                                     const int32_t* __restrict__ pos, int T,
+                                                     int k, int VH, uint4* __restrict__ dX,
+                                                     uint32_t* __restrict__ status) {
+  constexpr int PER = DT == LRMOE_BF16 ? 8 : 4;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    // retained rows of this token, in ascending slot order (k <= 32)
+    int r = lane < k ? pos[(size_t)t * k + lane] : -1;
+    if (r >= rows_cap) {
+      raise_status(status, LRMOE_ST_BAD_INDEX);
+      r = -1;
+    }
+    const unsigned have = __ballot_sync(kFull, r >= 0);
+    for (int c = lane; c < VH; c += 32) {
+      float acc[PER];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
+      unsigned todo = have;
+      while (todo) {
+        const int j = __ffs(todo) - 1;
+        todo &= todo - 1;
+        const int row = __shfl_sync(kFull, r, j);
+        const uint4 v = __ldg(dXp + (size_t)row * VH + c);
+        if constexpr (DT == LRMOE_BF16) {
+          const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] = __fadd_rn(acc[2 * i], bf16_bits_to_f32(ww[i] & 0xffffu));
+            acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], bf16_bits_to_f32(ww[i] >> 16));
+          }
+        } else {
+          acc[0] = __fadd_rn(acc[0], __uint_as_float(v.x));
+          acc[1] = __fadd_rn(acc[1], __uint_as_float(v.y));
+          acc[2] = __fadd_rn(acc[2], __uint_as_float(v.z));
+          acc[3] = __fadd_rn(acc[3], __uint_as_float(v.w));
+        }
+      }
+      uint4 o;
+      if constexpr (DT == LRMOE_BF16) {
+        o = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+      } else {
+        o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
+                       __float_as_uint(acc[3]));
+      }
+      dX[(size_t)t * VH + c] = o;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const int32_t* perm, const int32_t* offsets, const float* w, int T,
+                        int k, int E, const void* x, const void* dY, int H, const void* a,
+                        const void* g, const void* u, int I, lrmoe_dtype dt, void* Xp, void* DYp,
+                        void* Ap, void* Gp, void* Up, int rows_cap, uint32_t* status,
+                        cudaStream_t s) {
+  const int per = dt == LRMOE_BF16 ? 8 : 4;
+  const int VH = H / per, VI = I / per;
+  const int blocks = num_sms() * 8;
+  auto X = static_cast<const uint4*>(x);
+  auto D = static_cast<const uint4*>(dY);
+  auto A = static_cast<const uint4*>(a);
+  auto G = static_cast<const uint4*>(g);
+  auto U = static_cast<const uint4*>(u);
+  if (dt == LRMOE_BF16)
+    pack_kernel<LRMOE_BF16><<<blocks, 256, 0, s>>>(
+        perm, offsets, E, w, T * k, k, X, D, VH, A, G, U, VI, static_cast<uint4*>(Xp),
+        static_cast<uint4*>(DYp), static_cast<uint4*>(Ap), static_cast<uint4*>(Gp),
+        static_cast<uint4*>(Up), rows_cap, status);
+  else
+    pack_kernel<LRMOE_F32><<<blocks, 256, 0, s>>>(
+        perm, offsets, E, w, T * k, k, X, D, VH, A, G, U, VI, static_cast<uint4*>(Xp),
+        static_cast<uint4*>(DYp), static_cast<uint4*>(Ap), static_cast<uint4*>(Gp),
+        static_cast<uint4*>(Up), rows_cap, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack(const void* dXp, int rows_cap, const int32_t* pos, int T, int k, int H,
+                          lrmoe_dtype dt, void* dX, uint32_t* status, cudaStream_t s) {
+  const int per = dt == LRMOE_BF16 ? 8 : 4;
+  const int VH = H / per;
+  const int wpb = 8;
+  int blocks = (T + wpb - 1) / wpb;
+  const int maxb = num_sms() * 8;
+  if (blocks > maxb) blocks = maxb;
+  if (dt == LRMOE_BF16)
+    unpack_kernel<LRMOE_BF16><<<blocks, 256, 0, s>>>(static_cast<const uint4*>(dXp), rows_cap,
+                                                      pos, T, k, VH, static_cast<uint4*>(dX),
+                                                      status);
+  else
+    unpack_kernel<LRMOE_F32><<<blocks, 256, 0, s>>>(static_cast<const uint4*>(dXp), rows_cap, pos,
+                                                     T, k, VH, static_cast<uint4*>(dX), status);
+  return cudaGetLastError();
+}
+
+}  // namespace lrmoe

@@ -1,0 +1,421 @@
+// a2  Per-expert top-quota selection.
+//
+// Follows "LRMoE урезает обратный проход MoE ...", section "Что делает LRMoE",
+// bullets 2-3: the quota of every expert is fixed for the layer call, and
+// within it the pairs with the highest score stay.  Key: score bit pattern as
+// uint32 descending, then pair index ascending (scores are >= +0, so the bit
+// order is the numeric order; NaN sorts above +Inf).
+//
+// Four kernels, integer work only, deterministic (no order-dependent atomics):
+//   1. chunk_count : per chunk of pairs, an expert histogram (+ pos = -1 for
+//                    empty/invalid slots)
+//   2. chunk_scan  : per expert, exclusive scan over chunks; counts, the
+//                    segment starts, m_e = min(max(q_e,0), c_e), offsets
+//   3. chunk_scatter: stable counting sort of the pairs by expert (ascending p
+//                    inside each expert) into seg_p / seg_key
+//   4. expert_topk : one CTA per expert: 4 x 8-bit radix select of the m_e-th
+//                    largest key, then an ordered compaction that keeps keys
+//                    above the threshold and the first (m_e - #above) equal
+//                    keys in ascending p; writes perm and pos.
+#include "common.cuh"
+#include "launch.h"
+
+namespace lrmoe {
+namespace {
+
+constexpr int kScanThreads = 1024;
+constexpr int kCountThreads = 256;
+constexpr int kScatterWarps = 8;
+constexpr int kTopkThreads = 1024;
+constexpr int kScanSmemInts = 32768;  // E * nchunks kept in shared memory by chunk_scan
+constexpr int kTopkSmemKeys = 40960;  // segments up to this length are selected in smem
+
+__global__ void __launch_bounds__(kCountThreads) chunk_count(const int32_t* __restrict__ idx,
+                                                              int P, int E, int chunk,
+                                                              int nchunks, int32_t* __restrict__ cc,
+                                                              int32_t* __restrict__ pos,
+                                                              uint32_t* __restrict__ status) {
+  extern __shared__ int hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int c = blockIdx.x;
+  const int begin = c * chunk;
+  const int end = min(P, begin + chunk);
+  bool bad = false;
+  for (int p = begin + threadIdx.x; p < end; p += blockDim.x) {
+    const int e = __ldg(idx + p);
+    if (e >= 0 && e < E) {
+      atomicAdd(&hist[e], 1);
+    } else {
+      pos[p] = -1;
+      bad |= (e >= E);
+    }
+  }
+  if (__any_sync(kFull, bad) && (threadIdx.x & 31) == 0) raise_status(status, LRMOE_ST_BAD_EXPERT);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cc[(size_t)e * nchunks + c] = hist[e];
+}
+
+// Exclusive scan of n ints held one per thread (n <= blockDim.x * items); returns
+// per-thread exclusive prefix of the thread's item sum, and the total.
+__device__ int block_excl_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+  const int incl = warp_incl_scan(v);
+  if (lane == 31) warp_sums[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    int s = lane < nw ? warp_sums[lane] : 0;
+    int si = warp_incl_scan(s);
+    if (lane < nw) warp_sums[lane] = si - s;
+    if (lane == 31) warp_sums[32] = si;
+  }
+  __syncthreads();
+  const int r = warp_sums[wid] + incl - v;
+  *total = warp_sums[32];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kScanThreads) chunk_scan(int32_t* __restrict__ cc, int E,
+                                                           int nchunks,
+                                                           const int32_t* __restrict__ quota,
+                                                           int32_t* __restrict__ counts,
+                                                           int32_t* __restrict__ kept,
+                                                           int32_t* __restrict__ offsets,
+                                                           int32_t* __restrict__ seg_start,
+                                                           uint32_t* __restrict__ status) {
+  extern __shared__ int sm[];  // [33] warp sums, then [E] counts, then cc copy if it fits
+  int* warp_sums = sm;
+  int* cnt = sm + 33;
+  int* ccs = cnt + E;
+  const bool in_smem = (size_t)E * nchunks <= (size_t)kScanSmemInts;
+  int* mat = in_smem ? ccs : cc;
+  const int n = E * nchunks;
+  if (in_smem)
+    for (int i = threadIdx.x; i < n; i += blockDim.x) ccs[i] = cc[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int e = wid; e < E; e += nw) {
+    int carry = 0;
+    int* row = mat + (size_t)e * nchunks;
+    for (int c0 = 0; c0 < nchunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < nchunks ? row[c] : 0;
+      const int incl = warp_incl_scan(v);
+      if (c < nchunks) row[c] = carry + incl - v;
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) cnt[e] = carry;
+  }
+  __syncthreads();
+  if (in_smem)
+    for (int i = threadIdx.x; i < n; i += blockDim.x) cc[i] = ccs[i];
+  // segment starts (exclusive scan of counts) and offsets (exclusive scan of kept)
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = threadIdx.x * per;
+  int csum = 0, ksum = 0;
+  bool badq = false;
+  for (int i = 0; i < per; ++i) {
+    const int e = e0 + i;
+    if (e < E) {
+      const int c = cnt[e];
+      const int q = quota[e];
+      badq |= q < 0;
+      csum += c;
+      ksum += min(max(q, 0), c);
+    }
+  }
+  if (__any_sync(kFull, badq) && lane == 0) raise_status(status, LRMOE_ST_BAD_QUOTA);
+  int ctot, ktot;
+  int cex = block_excl_scan(csum, warp_sums, &ctot);
+  int kex = block_excl_scan(ksum, warp_sums, &ktot);
+  for (int i = 0; i < per; ++i) {
+    const int e = e0 + i;
+    if (e < E) {
+      const int c = cnt[e];
+      const int m = min(max(quota[e], 0), c);
+      counts[e] = c;
+      kept[e] = m;
+      seg_start[e] = cex;
+      offsets[e] = kex;
+      cex += c;
+      kex += m;
+    }
+  }
+  if (threadIdx.x == 0) {
+    seg_start[E] = ctot;
+    offsets[E] = ktot;
+  }
+}
+
+__global__ void __launch_bounds__(kScatterWarps * 32) chunk_scatter(
+    const int32_t* __restrict__ idx, const uint32_t* __restrict__ score_bits, int P, int E,
+    int chunk, int nchunks, const int32_t* __restrict__ cc, const int32_t* __restrict__ seg_start,
+    int32_t* __restrict__ seg_p, uint32_t* __restrict__ seg_key) {
+  extern __shared__ int wbase[];  // [kScatterWarps][E]
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int c = blockIdx.x;
+  const int begin = c * chunk;
+  const int end = min(P, begin + chunk);
+  const int sub = (chunk + kScatterWarps - 1) / kScatterWarps;
+  const int wbeg = min(end, begin + wid * sub);
+  const int wend = min(end, wbeg + sub);
+  for (int i = threadIdx.x; i < kScatterWarps * E; i += blockDim.x) wbase[i] = 0;
+  __syncthreads();
+  int* mine = wbase + wid * E;
+  for (int p = wbeg + lane; p < wend; p += 32) {
+    const int e = __ldg(idx + p);
+    if (e >= 0 && e < E) atomicAdd(&mine[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = seg_start[e] + cc[(size_t)e * nchunks + c];
+#pragma unroll
+    for (int w = 0; w < kScatterWarps; ++w) {
+      const int v = wbase[w * E + e];
+      wbase[w * E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int p0 = wbeg; p0 < wend; p0 += 32) {
+    const int p = p0 + lane;
+    const int e = p < wend ? __ldg(idx + p) : -1;
+    const bool valid = e >= 0 && e < E;
+    const int key = valid ? e : -1;
+    const unsigned m = __match_any_sync(kFull, key);
+    int base = 0;
+    if (valid) {
+      base = mine[e];
+      const int dst = base + __popc(m & lt);
+      seg_p[dst] = p;
+      seg_key[dst] = __ldg(score_bits + p);
+    }
+    __syncwarp();
+    if (valid && lane == __ffs(m) - 1) mine[e] = base + __popc(m);
+    __syncwarp();
+  }
+}
+
+// Block-wide exclusive scan for 1024 threads (32 warps); returns the total too.
+__device__ __forceinline__ uint32_t block_excl_scan_u32(uint32_t v, uint32_t* ws,
+                                                        uint32_t* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t n = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) ws[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    uint32_t s = ws[lane];
+    uint32_t si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t n = __shfl_up_sync(kFull, si, o);
+      if (lane >= o) si += n;
+    }
+    ws[lane] = si - s;
+    if (lane == 31) ws[32] = si;
+  }
+  __syncthreads();
+  const uint32_t r = ws[wid] + incl - v;
+  *total = ws[32];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) expert_topk(
+    const int32_t* __restrict__ counts, const int32_t* __restrict__ kept,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ seg_start,
+    const int32_t* __restrict__ seg_p, const uint32_t* __restrict__ seg_key,
+    int32_t* __restrict__ perm, int32_t* __restrict__ pos) {
+  extern __shared__ uint32_t keys_smem[];
+  __shared__ int hist[256];
+  __shared__ uint32_t scan_ws[33];
+  __shared__ int found_bin, found_above;
+  const int e = blockIdx.x;
+  const int c = counts[e];
+  const int m = kept[e];
+  const int s0 = seg_start[e];
+  const int out0 = offsets[e];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int32_t* sp = seg_p + s0;
+  const uint32_t* sk = seg_key + s0;
+
+  if (m == c) {  // everything stays, already in ascending p
+    for (int i = tid; i < c; i += blockDim.x) {
+      const int p = sp[i];
+      perm[out0 + i] = p;
+      pos[p] = out0 + i;
+    }
+    return;
+  }
+  if (m == 0) {
+    for (int i = tid; i < c; i += blockDim.x) pos[sp[i]] = -1;
+    return;
+  }
+
+  const bool in_smem = c <= kTopkSmemKeys;
+  const uint32_t* K = sk;
+  if (in_smem) {
+    for (int i = tid; i < c; i += blockDim.x) keys_smem[i] = sk[i];
+    K = keys_smem;
+  }
+  __syncthreads();
+
+  // radix select of the m-th largest key, most significant byte first
+  uint32_t prefix = 0;
+  int need = m;
+  for (int d = 3; d >= 0; --d) {
+    const int shift = 8 * d;
+    const uint32_t hmask = d == 3 ? 0u : (0xffffffffu << (shift + 8));
+    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i0 = 0; i0 < c; i0 += blockDim.x) {
+      const int i = i0 + tid;
+      int digit = -1;
+      if (i < c) {
+        const uint32_t key = K[i];
+        if ((key & hmask) == prefix) digit = (int)((key >> shift) & 255u);
+      }
+      const unsigned grp = __match_any_sync(kFull, digit);
+      if (digit >= 0 && lane == __ffs(grp) - 1) atomicAdd(&hist[digit], __popc(grp));
+    }
+    __syncthreads();
+    if (wid == 0) {
+      // lane l owns bins 255-8l down to 248-8l (descending key order)
+      int cnt8[8];
+      int lsum = 0;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        cnt8[b] = hist[255 - 8 * lane - b];
+        lsum += cnt8[b];
+      }
+      const int incl = warp_incl_scan(lsum);
+      const int excl = incl - lsum;
+      if (excl < need && need <= incl) {
+        int cum = excl;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          if (cum + cnt8[b] >= need) {
+            found_bin = 255 - 8 * lane - b;
+            found_above = cum;
+            break;
+          }
+          cum += cnt8[b];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= (uint32_t)found_bin << shift;
+    need -= found_above;
+    __syncthreads();
+  }
+  const uint32_t tau = prefix;
+  const uint32_t need_eq = (uint32_t)need;  // equal keys to keep, in ascending p
+
+  // ordered compaction
+  uint32_t carry_gt = 0, carry_eq = 0;
+  for (int i0 = 0; i0 < c; i0 += blockDim.x) {
+    const int i = i0 + tid;
+    uint32_t key = 0;
+    bool gt = false, eq = false;
+    if (i < c) {
+      key = K[i];
+      gt = key > tau;
+      eq = key == tau;
+    }
+    const uint32_t packed = (gt ? 1u : 0u) | (eq ? 0x10000u : 0u);
+    uint32_t tot;
+    const uint32_t ex = block_excl_scan_u32(packed, scan_ws, &tot);
+    if (i < c) {
+      const uint32_t gt_before = carry_gt + (ex & 0xffffu);
+      const uint32_t eq_before = carry_eq + (ex >> 16);
+      const int p = sp[i];
+      const bool keep = gt || (eq && eq_before < need_eq);
+      if (keep) {
+        const int row = out0 + (int)(gt_before + min(eq_before, need_eq));
+        perm[row] = p;
+        pos[p] = row;
+      } else {
+        pos[p] = -1;
+      }
+    }
+    carry_gt += tot & 0xffffu;
+    carry_eq += tot >> 16;
+  }
+}
+
+}  // namespace
+
+static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+SelectWs select_ws_layout(int T, int k, int E) {
+  SelectWs L;
+  const long long P = (long long)T * k;
+  long long chunk = 2048;
+  const long long max_chunks = kScanSmemInts / (E > 0 ? E : 1);
+  if (max_chunks > 0 && (P + chunk - 1) / chunk > max_chunks) {
+    chunk = (P + max_chunks - 1) / max_chunks;
+    chunk = (chunk + 255) / 256 * 256;
+  }
+  L.chunk = (int)chunk;
+  L.nchunks = (int)((P + chunk - 1) / chunk);
+  if (L.nchunks < 1) L.nchunks = 1;
+  size_t off = 0;
+  L.off_cc = off;
+  off += align256((size_t)E * L.nchunks * 4);
+  L.off_seg_start = off;
+  off += align256((size_t)(E + 1) * 4);
+  L.off_seg_p = off;
+  off += align256((size_t)P * 4);
+  L.off_seg_key = off;
+  off += align256((size_t)P * 4);
+  L.total = off;
+  return L;
+}
+
+cudaError_t launch_select(const int32_t* idx, const float* score, int T, int k, int E,
+                          const int32_t* quota, int32_t* counts, int32_t* kept, int32_t* offsets,
+                          int32_t* perm, int32_t* pos, void* ws, uint32_t* status,
+                          cudaStream_t s) {
+  const SelectWs L = select_ws_layout(T, k, E);
+  const int P = T * k;
+  char* base = static_cast<char*>(ws);
+  int32_t* cc = reinterpret_cast<int32_t*>(base + L.off_cc);
+  int32_t* seg_start = reinterpret_cast<int32_t*>(base + L.off_seg_start);
+  int32_t* seg_p = reinterpret_cast<int32_t*>(base + L.off_seg_p);
+  uint32_t* seg_key = reinterpret_cast<uint32_t*>(base + L.off_seg_key);
+
+  static unsigned long long attrs_set = 0;  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !((attrs_set >> dev) & 1ull)) {
+    cudaFuncSetAttribute(chunk_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (33 + 4096 + kScanSmemInts) * 4);
+    cudaFuncSetAttribute(chunk_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kScatterWarps * 4096 * 4);
+    cudaFuncSetAttribute(expert_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kTopkSmemKeys * 4);
+    attrs_set |= 1ull << dev;
+  }
+  chunk_count<<<L.nchunks, kCountThreads, E * 4, s>>>(idx, P, E, L.chunk, L.nchunks, cc, pos,
+                                                      status);
+  const bool fits = (size_t)E * L.nchunks <= (size_t)kScanSmemInts;
+  const size_t scan_smem = (33 + (size_t)E + (fits ? (size_t)E * L.nchunks : 0)) * 4;
+  chunk_scan<<<1, kScanThreads, scan_smem, s>>>(cc, E, L.nchunks, quota, counts, kept, offsets,
+                                                seg_start, status);
+  chunk_scatter<<<L.nchunks, kScatterWarps * 32, kScatterWarps * E * 4, s>>>(
+      idx, reinterpret_cast<const uint32_t*>(score), P, E, L.chunk, L.nchunks, cc, seg_start,
+      seg_p, seg_key);
+  expert_topk<<<E, kTopkThreads, kTopkSmemKeys * 4, s>>>(counts, kept, offsets, seg_start, seg_p,
+                                                         seg_key, perm, pos);
+  return cudaGetLastError();
+}
+
+}  // namespace lrmoe

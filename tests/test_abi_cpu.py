@@ -1,0 +1,107 @@
+"""The C ABI library builds, loads without a GPU, exports every declared symbol,
+and rejects host-detectable bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from pruned_expert_backward_lrmoe_b200 import build as B
+from pruned_expert_backward_lrmoe_b200 import lrmoe as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "lrmoe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lrmoe_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(L.EXPORTS)
+
+
+def test_version_and_strings(lib):
+    assert lib.lrmoe_version() >> 16 == 1
+    assert lib.lrmoe_status_string(0) == b"ok"
+    assert lib.lrmoe_status_string(4) == b"workspace too small"
+
+
+def test_workspace_size_grows_with_pairs(lib):
+    a = L.lrmoe_select_workspace_bytes(256, 2, 8)
+    b = L.lrmoe_select_workspace_bytes(8192, 8, 128)
+    assert 0 < a < b
+    assert b >= 2 * 8192 * 8 * 4
+    assert L.lrmoe_select_workspace_bytes(0, 8, 128) == 0
+
+
+NULL = ctypes.c_void_p(0)
+FAKE = ctypes.c_void_p(0x10000)  # aligned non-null; never dereferenced by the host checks
+
+
+def test_score_rejects_bad_arguments(lib):
+    f = lib.lrmoe_score
+    # null pointer
+    assert f(NULL, FAKE, 4, 2, 3, FAKE, 8, FAKE, 8, 1, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert b"topk_idx" in lib.lrmoe_last_error()
+    # H not a multiple of 8 for bf16
+    assert f(FAKE, FAKE, 4, 2, 3, FAKE, 12, FAKE, 8, 1, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    # misaligned pointer
+    bad = ctypes.c_void_p(0x10004)
+    assert f(FAKE, FAKE, 4, 2, 3, bad, 8, FAKE, 8, 1, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    # non-positive sizes, unknown dtype, k > 32
+    assert f(FAKE, FAKE, 0, 2, 3, FAKE, 8, FAKE, 8, 1, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, 2, 3, FAKE, 8, FAKE, 8, 7, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, 33, 40, FAKE, 8, FAKE, 8, 1, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+
+
+def test_select_rejects_small_workspace(lib):
+    f = lib.lrmoe_select_quota
+    need = L.lrmoe_select_workspace_bytes(64, 2, 4)
+    ws = ctypes.c_void_p(0x100000)
+    r = f(FAKE, FAKE, 64, 2, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, need - 1, NULL, NULL)
+    assert r == L.LRMOE_ERR_WORKSPACE
+    r = f(FAKE, FAKE, 64, 2, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_void_p(0x100010),
+          need, NULL, NULL)
+    assert r == L.LRMOE_ERR_WORKSPACE       # not 256-byte aligned
+    r = f(FAKE, FAKE, 64, 2, 5000, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, 1 << 30, NULL, NULL)
+    assert r == L.LRMOE_ERR_UNSUPPORTED     # E > 4096
+
+
+def test_gemm_rejects_bad_arguments(lib):
+    d = lib.lrmoe_grouped_dgrad
+    # unknown epilogue
+    assert d(FAKE, 16, FAKE, FAKE, 2, 64, 64, 1, 9, NULL, NULL, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    # SwiGLU epilogue needs g and u
+    assert d(FAKE, 16, FAKE, FAKE, 2, 64, 64, 1, 1, NULL, NULL, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    # too many experts for the tile table
+    assert d(FAKE, 16, FAKE, FAKE, 2000, 64, 64, 1, 0, NULL, NULL, FAKE, NULL, NULL) == L.LRMOE_ERR_UNSUPPORTED
+    w = lib.lrmoe_grouped_wgrad
+    assert w(FAKE, FAKE, 16, FAKE, 2, 60, 64, 1, FAKE, 0, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert w(FAKE, FAKE, 16, NULL, 2, 64, 64, 1, FAKE, 0, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+
+
+def test_pack_unpack_reject_bad_arguments(lib):
+    p = lib.lrmoe_pack
+    assert p(FAKE, FAKE, FAKE, 4, 2, 3, FAKE, FAKE, 8, FAKE, FAKE, FAKE, 8, 1, FAKE, FAKE, FAKE,
+             FAKE, NULL, 8, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert p(FAKE, FAKE, FAKE, 4, 2, 3, FAKE, FAKE, 8, FAKE, FAKE, FAKE, 8, 1, FAKE, FAKE, FAKE,
+             FAKE, FAKE, 0, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    u = lib.lrmoe_unpack
+    assert u(FAKE, 8, FAKE, 4, 2, 6, 0, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG  # H % 4
+    assert u(FAKE, 8, NULL, 4, 2, 8, 0, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+
+
+def test_pruned_backward_rejects_null_struct(lib):
+    assert lib.lrmoe_pruned_backward(None, 4, 2, 3, 8, 8, 8, 1, NULL) == L.LRMOE_ERR_INVALID_ARG

@@ -385,3 +385,22 @@ def test_swiglu_derivative_closed_form():
     silu = lambda v: v / (1 + np.exp(-v))
     fd = (silu(g + h) - silu(g - h)) / (2 * h)
     np.testing.assert_allclose(s * (1 + g * (1 - s)), fd, rtol=1e-7, atol=1e-9)
+
+
+def test_row_sampled_backward_matches_whole_expert_backward():
+    """The per-row helpers used on full-size layers agree with the whole-expert path."""
+    L = small_layer("qwen", T=96, E=8, H=64, I=32)
+    s = L.spec
+    r = O.pruned_backward(L)
+    rows = np.arange(0, r["perm"].size, 3)
+    dgu, dxp = O.expert_backward_rows(rows, r["offsets"], r["DYp"], r["Gp"], r["Up"], L.W_gu,
+                                      L.W_down, s.dtype)
+    for row in rows:
+        np.testing.assert_allclose(dgu[int(row)], r["dGUp"][row], rtol=1e-13, atol=1e-300)
+        np.testing.assert_allclose(dxp[int(row)], r["dXp"][row], rtol=1e-13, atol=1e-300)
+    tokens = [0, 5, 17, 95]
+    need = [int(p) for t in tokens for p in r["pos"].reshape(-1, s.k)[t] if p >= 0]
+    _, dxp_all = O.expert_backward_rows(need, r["offsets"], r["DYp"], r["Gp"], r["Up"], L.W_gu,
+                                        L.W_down, s.dtype)
+    got = O.unpack_tokens(tokens, dxp_all, r["pos"], s.k, s.H)
+    np.testing.assert_allclose(got, r["dX"][tokens], rtol=1e-12, atol=1e-300)
