@@ -1,0 +1,502 @@
+"""Benchmark of the pruned MoE expert backward (LRMoE) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config qwen] [--impl reference]
+
+A step is one pass of the whole hot path over one synthetic layer: LRM score,
+per-expert top-quota selection, compaction, the four grouped GEMMs (SwiGLU
+dgrad, dW_down, dW_gate|up, dX_p) and the unpack of dX, issued as the eight
+C-ABI calls of liblrmoe.so on one stream.  The metric is retained pairs per
+second (plus expert-backward TFLOP/s of the grouped GEMMs), measured with CUDA
+events on the launching stream; inputs are resident in HBM and L2 is flushed
+(512 MiB write) between timed steps, outside the events.
+
+N > 1 (torchrun, one process per GPU): every rank runs its own replica of the
+layer (the single-GPU path has no exchange step), the timed region is bracketed
+by barriers, the max time over ranks is taken, and value = all ranks' retained
+pairs / that time ("scaling": "weak").
+
+--impl reference times the CPU oracle (numpy, fp64) on the host cores, one
+bounded sample of the same layer per step, and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "retained pairs/s + expert-bwd TFLOP/s on 1 B200; % of HBM / bf16 roofline"
+UNIT = "retained pairs/s"
+DEFAULT_CONFIG = "qwen"
+KERNELS = ("score", "select", "pack", "dgrad_swiglu", "wgrad_down", "wgrad_gu", "dgrad_x", "unpack")
+KERNEL_LAUNCHES = {"score": 1, "select": 4, "pack": 1, "dgrad_swiglu": 1, "wgrad_down": 1,
+                   "wgrad_gu": 1, "dgrad_x": 1, "unpack": 1}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--config", default=DEFAULT_CONFIG)
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--impl", choices=("lrmoe", "reference"), default="lrmoe")
+    p.add_argument("--no-cpu-baseline", action="store_true",
+                   help="skip timing the CPU oracle (profiling runs)")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes and flops per launch (per kernel), from the layer's sizes
+# ---------------------------------------------------------------------------
+def algorithmic(T, k, E, H, I, M, b):
+    """Bytes each step must move at minimum, and the grouped-GEMM flops."""
+    P = T * k
+    by = {
+        "score": T * H * b + P * I * b + 8 * P + 4 * P,
+        "select": 4 * P + 4 * P + 4 * E + 12 * E + 4 * M + 4 * P,
+        "pack": 2 * M * (2 * H + 3 * I) * b + 8 * M,
+        "dgrad_swiglu": M * H * b + E * H * I * b + 2 * M * I * b + 2 * M * I * b,
+        "wgrad_down": M * H * b + M * I * b + E * H * I * 4,
+        "wgrad_gu": 2 * M * I * b + M * H * b + E * 2 * I * H * 4,
+        "dgrad_x": 2 * M * I * b + E * 2 * I * H * b + M * H * b,
+        "unpack": M * H * b + 4 * P + T * H * b,
+    }
+    fl = {"dgrad_swiglu": 2 * M * H * I, "wgrad_down": 2 * M * H * I, "wgrad_gu": 4 * M * I * H,
+          "dgrad_x": 4 * M * I * H}
+    return by, fl
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def recorded_traffic(kernel: str, config: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, or None.
+
+    profiles/traffic.json maps "<kernel>@<config>" to {"bytes": B, "source_sha1": S};
+    the figure is dropped when the kernel's source changed since the capture.
+    """
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            table = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = table.get(f"{kernel}@{config}")
+    if not ent:
+        return None
+    if ent.get("source_sha1") != kernel_source_sha1():
+        return None
+    return ent.get("bytes")
+
+
+def kernel_source_sha1() -> str:
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "pruned_expert_backward_lrmoe_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, sampled from a thread)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {  # NVML clocks-event reason bits
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: clocks are reported as unknown
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+                self.reasons |= int(get(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        reasons = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}; launch N>1 with torchrun")
+    if world == 1:
+        return 0, 1, 0, None
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    rank, local = int(os.environ["RANK"]), int(os.environ.get("LOCAL_RANK", "0"))
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local, dist
+
+
+def max_over_ranks(value: float, dist) -> float:
+    if dist is None:
+        return value
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, dist) -> float:
+    if dist is None:
+        return value
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timings
+# ---------------------------------------------------------------------------
+def oracle_full_pass(layer):
+    """One pass of the oracle over the whole layer; returns (seconds, retained pairs)."""
+    from oracle import lrmoe_oracle as O
+    t0 = time.perf_counter()
+    r = O.pruned_backward(layer)
+    return time.perf_counter() - t0, int(r["offsets"][-1])
+
+
+def oracle_expert_sample(layer, experts):
+    """The oracle on the pairs of a few experts, as a standalone mini layer per expert.
+
+    Each expert's routed pairs become a layer with k = 1 and one expert; the
+    oracle runs score, selection, compaction, backward and unpack on it.
+    Returns (seconds, retained pairs).
+    """
+    from oracle import lrmoe_oracle as O
+    s = layer.spec
+    flat = layer.topk_idx.reshape(-1)
+    done = 0
+    t0 = time.perf_counter()
+    for e in experts:
+        pairs = np.nonzero(flat == e)[0]
+        if pairs.size == 0:
+            continue
+        tok = pairs // s.k
+        idx = np.zeros((pairs.size, 1), np.int32)
+        w = layer.topk_w.reshape(-1)[pairs].reshape(-1, 1)
+        score, _ = O.lrm_score(idx, w, layer.dY[tok], layer.a[pairs], s.dtype, 1)
+        _, _, off, perm, pos, _ = O.select_quota(idx, score, layer.quota[e:e + 1], 1)
+        Xp, DYp, Ap, Gp, Up = O.pack(perm, w, 1, layer.x[tok], layer.dY[tok], layer.a[pairs],
+                                     layer.g[pairs], layer.u[pairs], s.dtype)
+        _, _, dXp, _ = O.expert_backward(Xp, DYp, Ap, Gp, Up, off, layer.W_gu[e:e + 1],
+                                         layer.W_down[e:e + 1], s.dtype)
+        O.unpack(dXp, pos, pairs.size, 1)
+        done += int(off[-1])
+    return time.perf_counter() - t0, done
+
+
+def host_cores() -> int:
+    try:
+        import torch
+        return int(torch.get_num_threads())
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    """The oracle on the host cores, one bounded expert sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from pruned_expert_backward_lrmoe_b200 import inputs
+    layer = inputs.make_layer(args.config, seed=args.seed)
+    s = layer.spec
+    E = s.E
+    # size the per-step sample so that warmup + steps end within ~3 minutes
+    t_one, _ = oracle_expert_sample(layer, [0])
+    per_step_budget = 150.0 / max(1, args.steps + args.warmup)
+    group = int(max(1, min(E, per_step_budget / max(t_one, 1e-3))))
+    nxt = 0
+    for _ in range(args.warmup):
+        oracle_expert_sample(layer, [(nxt + i) % E for i in range(group)])
+        nxt = (nxt + group) % E
+    tot_s, tot_m = 0.0, 0
+    for _ in range(args.steps):
+        dt_, m = oracle_expert_sample(layer, [(nxt + i) % E for i in range(group)])
+        nxt = (nxt + group) % E
+        tot_s += dt_
+        tot_m += m
+    value = tot_m / tot_s if tot_s > 0 else 0.0
+    cores = host_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_s / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(s, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{group} expert(s) per step as standalone k=1 layers "
+                                   f"(score, selection, compaction, fp64 backward, unpack)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(s, n_gpus):
+    return {"workload": f"{s.name} MoE layer expert backward: T={s.T} E={s.E} top-{s.k} "
+                        f"H={s.H} I={s.I} {s.dtype}, quota rule '{s.quota}'",
+            "T": s.T, "E": s.E, "k": s.k, "H": s.H, "I": s.I, "global_batch": s.T * n_gpus,
+            "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
+            "l2": "flushed (512 MiB write) between timed steps; inputs also exceed L2"}
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args):
+    import torch
+
+    from pruned_expert_backward_lrmoe_b200 import inputs
+    from pruned_expert_backward_lrmoe_b200 import lrmoe as L
+
+    rank, world, local, dist = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    layer = inputs.make_layer(args.config, seed=args.seed)
+    s = layer.spec
+    tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
+    b = 2 if s.dtype == "bf16" else 4
+
+    def storage(arr):
+        if s.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(arr))
+
+    host = {"topk_idx": torch.from_numpy(layer.topk_idx), "topk_w": torch.from_numpy(layer.topk_w),
+            "quota": torch.from_numpy(layer.quota), "x": storage(layer.x), "dY": storage(layer.dY),
+            "g": storage(layer.g), "u": storage(layer.u), "a": storage(layer.a)}
+    weights = {"W_gu": storage(layer.W_gu).to(dev), "W_down": storage(layer.W_down).to(dev)}
+    inp = {k_: v.to(dev) for k_, v in host.items()}
+    inp.update(weights)
+    out = L.alloc_buffers(s.T, s.k, s.E, s.H, s.I, tdt, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    st = out["status"]
+
+    def step(ev=None):
+        calls = (
+            lambda: L.lrmoe_score(inp["topk_idx"], inp["topk_w"], inp["dY"], inp["a"], s.E,
+                                  out["score"], st, stream),
+            lambda: L.lrmoe_select_quota(inp["topk_idx"], out["score"], inp["quota"], out["counts"],
+                                         out["kept"], out["offsets"], out["perm"], out["pos"],
+                                         out["workspace"], st, stream),
+            lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], inp["x"], inp["dY"],
+                                 inp["a"], inp["g"], inp["u"], out["Xp"], out["DYp"], out["Ap"],
+                                 out["Gp"], out["Up"], st, stream),
+            lambda: L.lrmoe_grouped_dgrad(out["DYp"], inp["W_down"], out["offsets"],
+                                          L.LRMOE_EPI_SWIGLU_BWD, out["dGUp"], Gp=out["Gp"],
+                                          Up=out["Up"], status=st, stream=stream),
+            lambda: L.lrmoe_grouped_wgrad(out["DYp"], out["Ap"], out["offsets"], out["dW_down"],
+                                          status=st, stream=stream),
+            lambda: L.lrmoe_grouped_wgrad(out["dGUp"], out["Xp"], out["offsets"], out["dW_gu"],
+                                          status=st, stream=stream),
+            lambda: L.lrmoe_grouped_dgrad(out["dGUp"], inp["W_gu"], out["offsets"],
+                                          L.LRMOE_EPI_STORE, out["dXp"], status=st, stream=stream),
+            lambda: L.lrmoe_unpack(out["dXp"], out["pos"], s.T, s.k, out["dX"], st, stream),
+        )
+        for i, c in enumerate(calls):
+            if ev is not None:
+                ev[i].record(stream)
+            c()
+        if ev is not None:
+            ev[len(calls)].record(stream)
+
+    st.zero_()
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(st.item()) != 0:
+        raise SystemExit(f"device status {int(st.item())} after warm-up")
+    M = int(out["offsets"][-1].item())
+    counts = out["kept"].cpu().numpy()
+
+    # ---------------- device-timed region ----------------
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS) + 1)]
+           for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        barrier(dist)
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+        barrier(dist)
+    per_kernel = {kname: [] for kname in KERNELS}
+    step_ms = []
+    for ev in evs:
+        for j, kname in enumerate(KERNELS):
+            per_kernel[kname].append(ev[j].elapsed_time(ev[j + 1]))
+        step_ms.append(ev[0].elapsed_time(ev[-1]))
+    mean_step = statistics.fmean(step_ms)
+    mean_step_max = max_over_ranks(mean_step, dist)
+    M_all = sum_over_ranks(float(M), dist)
+    value = M_all / (mean_step_max * 1e-3)
+    kern_ms = {kname: statistics.fmean(v) for kname, v in per_kernel.items()}
+
+    by, fl = algorithmic(s.T, s.k, s.E, s.H, s.I, M, b)
+    gemm_ms = sum(kern_ms[n] for n in fl)
+    gemm_flops = sum(fl.values())
+    peaks, peak_src = load_peaks()
+    dominant = max(kern_ms, key=kern_ms.get)
+    dom_bytes = by[dominant]
+    achieved_gbs = dom_bytes / (kern_ms[dominant] * 1e-3) / 1e9
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    traffic = recorded_traffic(dominant, s.name)
+    roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
+                "unit": "GB/s", "frac": achieved_gbs / hbm_peak, "traffic": traffic,
+                "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes": dom_bytes}
+    breakdown = {}
+    for kname in KERNELS:
+        gbs = by[kname] / (kern_ms[kname] * 1e-3) / 1e9
+        e = {"ms": kern_ms[kname], "GB/s": gbs, "hbm_frac": gbs / hbm_peak}
+        if kname in fl:
+            tf = fl[kname] / (kern_ms[kname] * 1e-3) / 1e12
+            e["TFLOP/s"] = tf
+            e["tensor_frac"] = tf / float(peaks.get("bf16_tflops_sustained",
+                                                    FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        breakdown[kname] = e
+
+    # ---------------- end to end through host buffers ----------------
+    pin = {k_: v.pin_memory() for k_, v in host.items()}
+    dX_host = torch.empty(s.T, s.H, dtype=tdt).pin_memory()
+    st_host = torch.empty(1, dtype=torch.int32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = dX_host.numel() * dX_host.element_size() + 4
+    n_e2e = max(3, min(args.steps, 50))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_e2e)]
+    for i in range(n_e2e + 2):
+        timed = i >= 2
+        flush.zero_()
+        if timed:
+            e2e_ev[i - 2][0].record(stream)
+        for k_, v in pin.items():
+            inp[k_].copy_(v, non_blocking=True)
+        L.lrmoe_pruned_backward(inp, out, stream)
+        dX_host.copy_(out["dX"], non_blocking=True)
+        st_host.copy_(out["status"], non_blocking=True)
+        if timed:
+            e2e_ev[i - 2][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = statistics.fmean(a_.elapsed_time(b_) for a_, b_ in e2e_ev)
+    e2e_value = M_all / (max_over_ranks(e2e_ms, dist) * 1e-3)
+
+    # ---------------- CPU baseline (rank 0 at N = 1) ----------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, m_cpu = oracle_full_pass(layer)
+        cpu = {"value": m_cpu / secs, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+               "sample": f"one full oracle pass over the {s.name} layer "
+                         f"({m_cpu} retained of {s.P} pairs), {secs:.1f} s"}
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": mean_step_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
+        "config": config_block(s, world),
+        "retained_pairs": M, "routed_pairs": s.P,
+        "expert_bwd_tflops": gemm_flops / (gemm_ms * 1e-3) / 1e12,
+        "gemm_ms": gemm_ms,
+        "roofline": roofline,
+        "breakdown": breakdown,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * sum(KERNEL_LAUNCHES.values()),
+        "clocks": clk.summary(),
+        "empty_experts": int((counts == 0).sum()),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
