@@ -130,6 +130,36 @@ int lrmoe_select_quota(const int32_t* topk_idx, const float* score, int T, int k
                        uint32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Selection that allocates nothing.  The LRMoE pages have no counterpart of
+ * this entry point; it exists for callers of this library that cannot hand
+ * it device scratch: a host framework or plugin host that owns every byte of
+ * device memory and gives its extensions no allocator, or a latency-critical
+ * caller that must not call cudaMalloc/cudaFree because those calls can
+ * synchronise the device and stall work on other streams.
+ *
+ * Same arguments (minus the workspace), same outputs and the same guarantees
+ * as lrmoe_select_quota.  The scratch is a fixed array of
+ * LRMOE_NOALLOC_SCRATCH_BYTES that the library keeps in device memory: every
+ * GPU that loads the library holds it until the process exits.  The first
+ * call on a device looks up that array's device address (once per device,
+ * with the device current), so make the first call on each device before any
+ * stream capture.  The call itself allocates nothing and calls no allocating
+ * routine.  All calls on one device share the array: two calls whose kernels
+ * overlap on the GPU (different streams, no ordering between them) race and
+ * give undefined results; calls on one stream are safe.  Nothing in the
+ * array has to start at zero and its stale contents never affect a result.
+ * Returns LRMOE_ERR_WORKSPACE, writing nothing, when the problem needs more
+ * scratch than the array holds (lrmoe_select_workspace_bytes(T,k,E) >
+ * LRMOE_NOALLOC_SCRATCH_BYTES, roughly T*k > 500 000 pairs at E = 128).
+ * ------------------------------------------------------------------------- */
+#define LRMOE_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+int lrmoe_select_quota_noalloc(const int32_t* topk_idx, const float* score, int T, int k, int E,
+                               const int32_t* quota, int32_t* counts, int32_t* kept,
+                               int32_t* offsets, int32_t* perm, int32_t* pos, uint32_t* status,
+                               void* stream);
+
+/* ---------------------------------------------------------------------------
  * a3  Physical compaction.  RU-B bullet 5 and the note after it, FR-B bullet
  * 5, DE paragraph 4: the retained gradient and activation rows are gathered
  * into dense blocks per expert; masking rows inside full-size tensors would

@@ -134,6 +134,36 @@ int lrmoe_select_quota(const int32_t* topk_idx, const float* score, int T, int k
   return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_select_quota launch");
 }
 
+// Selection for callers that cannot provide device scratch: the kernels use a
+// fixed array inside the library instead (see select.cu).  Nothing here or
+// below allocates.
+int lrmoe_select_quota_noalloc(const int32_t* topk_idx, const float* score, int T, int k, int E,
+                               const int32_t* quota, int32_t* counts, int32_t* kept,
+                               int32_t* offsets, int32_t* perm, int32_t* pos, uint32_t* status,
+                               void* stream) {
+  g_last_error[0] = 0;
+  if (int r = check_pairs(T, k, E)) return r;
+  if (E > 4096) return fail(LRMOE_ERR_UNSUPPORTED, "E=%d > 4096", E);
+  REQUIRE_PTR(topk_idx);
+  REQUIRE_PTR(score);
+  REQUIRE_PTR(quota);
+  REQUIRE_PTR(counts);
+  REQUIRE_PTR(kept);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(perm);
+  REQUIRE_PTR(pos);
+  const size_t need = select_ws_layout(T, k, E).total;
+  const size_t have = select_noalloc_scratch_bytes();
+  if (need > have)
+    return fail(LRMOE_ERR_WORKSPACE,
+                "T*k=%lld pairs need %zu bytes of scratch, more than the %zu-byte built-in "
+                "array; call lrmoe_select_quota with a workspace instead",
+                (long long)T * k, need, have);
+  cudaError_t e = launch_select_noalloc(topk_idx, score, T, k, E, quota, counts, kept, offsets,
+                                        perm, pos, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_select_quota_noalloc");
+}
+
 int lrmoe_pack(const int32_t* perm, const int32_t* offsets, const float* topk_w, int T, int k, int E,
                const void* x, const void* dY, int H, const void* a, const void* g, const void* u,
                int I, lrmoe_dtype dt, void* Xp, void* DYp, void* Ap, void* Gp, void* Up,

@@ -31,6 +31,13 @@ cudaError_t launch_select(const int32_t* idx, const float* score, int T, int k, 
                           int32_t* perm, int32_t* pos, void* ws, uint32_t* status,
                           cudaStream_t s);
 
+// Selection with the library's built-in scratch array (no caller workspace).
+size_t select_noalloc_scratch_bytes();
+cudaError_t launch_select_noalloc(const int32_t* idx, const float* score, int T, int k, int E,
+                                  const int32_t* quota, int32_t* counts, int32_t* kept,
+                                  int32_t* offsets, int32_t* perm, int32_t* pos, uint32_t* status,
+                                  cudaStream_t s);
+
 cudaError_t launch_pack(const int32_t* perm, const int32_t* offsets, const float* w, int T,
                         int k, int E, const void* x, const void* dY, int H, const void* a,
                         const void* g, const void* u, int I, lrmoe_dtype dt, void* Xp, void* DYp,

@@ -17,6 +17,8 @@
 //                    largest key, then an ordered compaction that keeps keys
 //                    above the threshold and the first (m_e - #above) equal
 //                    keys in ascending p; writes perm and pos.
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -353,6 +355,15 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Scratch for lrmoe_select_quota_noalloc: a fixed device array owned by the
+// library, so callers that may not allocate device memory can still select.
+// Every GPU that loads this module holds these bytes until the process exits.
+// All calls on a device share it; calls that overlap on the GPU race on it.
+// No byte of it needs to start at zero: each kernel writes what it reads.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_select_scratch[LRMOE_NOALLOC_SCRATCH_BYTES];
+
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 SelectWs select_ws_layout(int T, int k, int E) {
@@ -385,6 +396,77 @@ cudaError_t launch_select(const int32_t* idx, const float* score, int T, int k, 
                           int32_t* perm, int32_t* pos, void* ws, uint32_t* status,
                           cudaStream_t s) {
   const SelectWs L = select_ws_layout(T, k, E);
+  const int P = T * k;
+  char* base = static_cast<char*>(ws);
+  int32_t* cc = reinterpret_cast<int32_t*>(base + L.off_cc);
+  int32_t* seg_start = reinterpret_cast<int32_t*>(base + L.off_seg_start);
+  int32_t* seg_p = reinterpret_cast<int32_t*>(base + L.off_seg_p);
+  uint32_t* seg_key = reinterpret_cast<uint32_t*>(base + L.off_seg_key);
+
+  static unsigned long long attrs_set = 0;  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !((attrs_set >> dev) & 1ull)) {
+    cudaFuncSetAttribute(chunk_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (33 + 4096 + kScanSmemInts) * 4);
+    cudaFuncSetAttribute(chunk_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kScatterWarps * 4096 * 4);
+    cudaFuncSetAttribute(expert_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kTopkSmemKeys * 4);
+    attrs_set |= 1ull << dev;
+  }
+  chunk_count<<<L.nchunks, kCountThreads, E * 4, s>>>(idx, P, E, L.chunk, L.nchunks, cc, pos,
+                                                      status);
+  const bool fits = (size_t)E * L.nchunks <= (size_t)kScanSmemInts;
+  const size_t scan_smem = (33 + (size_t)E + (fits ? (size_t)E * L.nchunks : 0)) * 4;
+  chunk_scan<<<1, kScanThreads, scan_smem, s>>>(cc, E, L.nchunks, quota, counts, kept, offsets,
+                                                seg_start, status);
+  chunk_scatter<<<L.nchunks, kScatterWarps * 32, kScatterWarps * E * 4, s>>>(
+      idx, reinterpret_cast<const uint32_t*>(score), P, E, L.chunk, L.nchunks, cc, seg_start,
+      seg_p, seg_key);
+  expert_topk<<<E, kTopkThreads, kTopkSmemKeys * 4, s>>>(counts, kept, offsets, seg_start, seg_p,
+                                                         seg_key, perm, pos);
+  return cudaGetLastError();
+}
+
+namespace {
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {nullptr};  // device address of g_select_scratch, per device ordinal
+}  // namespace
+
+// Device address of the built-in scratch array on the current device.  In
+// host code `g_select_scratch` names only a host-side stand-in, never device
+// memory; the real address comes from the runtime, once per device, with that
+// device current, and is cached here.
+static cudaError_t select_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_select_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+size_t select_noalloc_scratch_bytes() { return sizeof(g_select_scratch); }
+
+// Same kernels and launch sequence as launch_select, with the built-in array
+// as the workspace.  The caller has checked that the layout fits in it.
+cudaError_t launch_select_noalloc(const int32_t* idx, const float* score, int T, int k, int E,
+                                  const int32_t* quota, int32_t* counts, int32_t* kept,
+                                  int32_t* offsets, int32_t* perm, int32_t* pos, uint32_t* status,
+                                  cudaStream_t s) {
+  const SelectWs L = select_ws_layout(T, k, E);
+  if (L.total > sizeof(g_select_scratch)) return cudaErrorInvalidValue;
+  void* ws = nullptr;
+  cudaError_t err = select_scratch_address(&ws);
+  if (err != cudaSuccess) return err;
   const int P = T * k;
   char* base = static_cast<char*>(ws);
   int32_t* cc = reinterpret_cast<int32_t*>(base + L.off_cc);

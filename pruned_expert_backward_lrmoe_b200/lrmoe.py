@@ -24,7 +24,9 @@ ST_BAD_EXPERT, ST_BAD_QUOTA, ST_NONFINITE, ST_TIMEOUT, ST_BAD_INDEX = 1, 2, 4, 8
 # every symbol the header declares
 EXPORTS = ("lrmoe_version", "lrmoe_status_string", "lrmoe_last_error", "lrmoe_score",
            "lrmoe_select_workspace_bytes", "lrmoe_select_quota", "lrmoe_pack",
-           "lrmoe_grouped_dgrad", "lrmoe_grouped_wgrad", "lrmoe_unpack", "lrmoe_pruned_backward")
+           "lrmoe_grouped_dgrad", "lrmoe_grouped_wgrad", "lrmoe_unpack", "lrmoe_pruned_backward",
+           "lrmoe_select_quota_noalloc")
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class LrmoeError(RuntimeError):
@@ -62,6 +64,7 @@ def load() -> ctypes.CDLL:
     lib.lrmoe_select_workspace_bytes.argtypes = [I, I, I]
     lib.lrmoe_select_workspace_bytes.restype = Z
     lib.lrmoe_select_quota.argtypes = [P, P, I, I, I, P, P, P, P, P, P, P, Z, P, P]
+    lib.lrmoe_select_quota_noalloc.argtypes = [P, P, I, I, I, P, P, P, P, P, P, P, P]
     lib.lrmoe_pack.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, I, I, P, P, P, P, P, I, P, P]
     lib.lrmoe_grouped_dgrad.argtypes = [P, I, P, P, I, I, I, I, I, P, P, P, P, P]
     lib.lrmoe_grouped_wgrad.argtypes = [P, P, I, P, I, I, I, I, P, I, P, P]
@@ -127,6 +130,20 @@ def lrmoe_select_quota(topk_idx, score, quota, counts, kept, offsets, perm, pos,
                                      _ptr(counts), _ptr(kept), _ptr(offsets), _ptr(perm),
                                      _ptr(pos), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                      _ptr(status), _stream(stream)))
+
+
+def lrmoe_select_quota_noalloc(topk_idx, score, quota, counts, kept, offsets, perm, pos,
+                               status=None, stream=None) -> None:
+    """Selection without a workspace, for callers that cannot allocate device scratch.
+
+    The library's own fixed scratch array (NOALLOC_SCRATCH_BYTES per GPU) is used
+    instead; calls that overlap on the GPU race on it.
+    """
+    T, k = topk_idx.shape
+    E = quota.numel()
+    _check(load().lrmoe_select_quota_noalloc(_ptr(topk_idx), _ptr(score), T, k, E, _ptr(quota),
+                                             _ptr(counts), _ptr(kept), _ptr(offsets), _ptr(perm),
+                                             _ptr(pos), _ptr(status), _stream(stream)))
 
 
 def lrmoe_pack(perm, offsets, topk_w, x, dY, a, g, u, Xp, DYp, Ap, Gp, Up, status=None,
