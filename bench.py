@@ -8,7 +8,7 @@ dgrad, dW_down, dW_gate|up, dX_p) and the unpack of dX, issued as the eight
 C-ABI calls of liblrmoe.so on one stream.  The metric is retained pairs per
 second (plus expert-backward TFLOP/s of the grouped GEMMs), measured with CUDA
 events on the launching stream; inputs are resident in HBM and L2 is flushed
-(512 MiB write) between timed steps, outside the events.
+between timed steps (a 512 MiB buffer written, then read back), outside the events.
 
 N > 1 (torchrun, one process per GPU): every rank runs its own replica of the
 layer (the single-GPU path has no exchange step), the timed region is bracketed
@@ -55,7 +55,18 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=("lrmoe", "reference"), default="lrmoe")
     p.add_argument("--no-cpu-baseline", action="store_true",
                    help="skip timing the CPU oracle (profiling runs)")
+    p.add_argument("--override", default="",
+                   help="layer fields to replace, e.g. T=4096,E=64 (smaller profiling cases)")
     return p.parse_args(argv)
+
+
+def layer_spec(args):
+    from pruned_expert_backward_lrmoe_b200 import inputs
+    over = {}
+    for item in filter(None, args.override.split(",")):
+        key, val = item.split("=")
+        over[key] = val if key in ("quota", "dtype", "name") else int(val)
+    return inputs.spec(args.config, **over)
 
 
 # ---------------------------------------------------------------------------
@@ -275,7 +286,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     from pruned_expert_backward_lrmoe_b200 import inputs
-    layer = inputs.make_layer(args.config, seed=args.seed)
+    layer = inputs.make_layer(layer_spec(args), seed=args.seed)
     s = layer.spec
     E = s.E
     # size the per-step sample so that warmup + steps end within ~3 minutes
@@ -314,7 +325,7 @@ def config_block(s, n_gpus):
                         f"H={s.H} I={s.I} {s.dtype}, quota rule '{s.quota}'",
             "T": s.T, "E": s.E, "k": s.k, "H": s.H, "I": s.I, "global_batch": s.T * n_gpus,
             "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
-            "l2": "flushed (512 MiB write) between timed steps; inputs also exceed L2"}
+            "l2": "flushed between timed steps (512 MiB written, then read back); inputs also exceed L2"}
 
 
 # ---------------------------------------------------------------------------
@@ -329,7 +340,7 @@ def run_gpu(args):
     rank, world, local, dist = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    layer = inputs.make_layer(args.config, seed=args.seed)
+    layer = inputs.make_layer(layer_spec(args), seed=args.seed)
     s = layer.spec
     tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
     b = 2 if s.dtype == "bf16" else 4
@@ -347,7 +358,13 @@ def run_gpu(args):
     inp.update(weights)
     out = L.alloc_buffers(s.T, s.k, s.E, s.H, s.I, tdt, device=dev)
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.empty(128 << 20, dtype=torch.float32, device=dev)  # 512 MiB > 126 MB L2
+
+    def flush_l2():
+        # write the buffer (evicts everything), then read it back so that the
+        # dirty lines are written out here rather than by the next timed kernel
+        flush.zero_()
+        flush.sum()
     st = out["status"]
 
     def step(ev=None):
@@ -394,7 +411,7 @@ def run_gpu(args):
         barrier(dist)
         torch.cuda.synchronize(dev)
         for i in range(args.steps):
-            flush.zero_()
+            flush_l2()
             step(evs[i])
         torch.cuda.synchronize(dev)
         barrier(dist)
@@ -444,7 +461,7 @@ def run_gpu(args):
               for _ in range(n_e2e)]
     for i in range(n_e2e + 2):
         timed = i >= 2
-        flush.zero_()
+        flush_l2()
         if timed:
             e2e_ev[i - 2][0].record(stream)
         for k_, v in pin.items():

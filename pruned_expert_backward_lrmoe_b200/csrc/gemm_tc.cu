@@ -10,10 +10,10 @@
 //          A = rows, K-major;   B = W[e], N-major;  epilogue STORE or SwiGLU-bwd
 //   wgrad (variable K): D = grad[R_e]^T (N1 x m_e) . in[R_e] (m_e x N2)
 //          A = grad, M-major;   B = in, N-major;    epilogue fp32 store / add
-// Roles (192 threads): warp 0 issues TMA loads into a ring of shared-memory
+// Roles (320 threads): warp 0 issues TMA loads into a ring of shared-memory
 // stages; warp 1 owns tensor memory and one lane issues tcgen05.mma (128 x BN
 // x 16 per instruction, fp32 accumulators in TMEM, two accumulator buffers so
-// that the epilogue of one tile overlaps the main loop of the next); warps 2-5
+// that the epilogue of one tile overlaps the main loop of the next); warps 2-9
 // drain TMEM with tcgen05.ld and store.  Group sizes are read on the device.
 // In wgrad the last K block of an expert may reach into the next expert's
 // rows: those rows are zeroed in shared memory before the MMAs read them.
@@ -30,19 +30,25 @@ namespace {
 constexpr int BM = 128;        // tile rows = TMEM lanes
 constexpr int BK = 64;         // 64 bf16 = one 128-byte swizzle row
 constexpr int UK = 16;         // K of one kind::f16 MMA
-constexpr int kThreads = 192;  // TMA warp, MMA warp, 4 epilogue warps
-constexpr int kEpiThreads = 128;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kEpiThreads = 32 * kEpiWarps;
 
 enum Mode : int { kDgradStore = 0, kDgradSwiglu = 1, kWgrad = 2 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool STAGED_OUT>
 struct Layout {
   static constexpr int kABytes = BM * BK * 2;                 // 16 KB
   static constexpr int kBBytes = BN * BK * 2;                 // 32 KB at BN = 256
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTilesBytes = STAGES * kStageBytes;
-  static constexpr int kTableInts = 2 * (kMaxExperts + 1) + 33;
-  static constexpr int kBarOff = kTilesBytes;                 // 8-byte barriers
+  // fp32 output staging: per epilogue warp two 32 x 32 fp32 sub-tiles (4 KB each)
+  static constexpr int kOutBufBytes = 32 * 32 * 4;
+  static constexpr int kOutOff = kTilesBytes;
+  static constexpr int kOutBytes = STAGED_OUT ? kEpiWarps * 2 * kOutBufBytes : 0;
+  // tile table, expert order / sizes, scan scratch, and a copy of offsets[0..E]
+  static constexpr int kTableInts = 3 * (kMaxExperts + 1) + 33;
+  static constexpr int kBarOff = kOutOff + kOutBytes;         // 8-byte barriers
   static constexpr int kNumBars = 2 * STAGES + 5;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;     // tmem base, abort flag
   static constexpr int kTableOff = kMiscOff + 16;
@@ -87,13 +93,83 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const int32_t* __restrict
 
 __device__ __forceinline__ float sigmoid_fast(float x) { return 1.0f / (1.0f + __expf(-x)); }
 
+// Make later uses of `r` depend on the preceding tcgen05.wait::ld.
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i])::"memory");
+}
+
+// bf16 row segment [nb, nb + 32) of `orow`, columns >= N skipped (N % 8 == 0).
+__device__ __forceinline__ void epi_store_bf16(const uint32_t (&r)[32], uint16_t* orow, int nb,
+                                               int N) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    if (nb + v * 8 < N) {
+      uint4 w;
+      w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+      w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+      w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+      w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+      *reinterpret_cast<uint4*>(orow + nb + v * 8) = w;
+    }
+  }
+}
+
+// saved g, u of one row, columns [nb, nb + 32)
+__device__ __forceinline__ void load_gu(uint4 (&gv)[4], uint4 (&uv)[4],
+                                        const uint16_t* __restrict__ Gp,
+                                        const uint16_t* __restrict__ Up, int row, int nb, int N) {
+  const uint16_t* gp = Gp + (size_t)row * N + nb;
+  const uint16_t* up = Up + (size_t)row * N + nb;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    if (nb + v * 8 < N) {
+      gv[v] = __ldg(reinterpret_cast<const uint4*>(gp + v * 8));
+      uv[v] = __ldg(reinterpret_cast<const uint4*>(up + v * 8));
+    }
+  }
+}
+
+// SwiGLU backward of one row segment: with s = sigmoid(g),
+// dG = dA u s (1 + g (1 - s)), dU = dA g s; stored as bf16.
+__device__ __forceinline__ void epi_swiglu(const uint32_t (&r)[32], const uint4 (&gv)[4],
+                                           const uint4 (&uv)[4], uint16_t* og, uint16_t* ou, int nb,
+                                           int N) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    if (nb + v * 8 < N) {
+      const uint32_t gw[4] = {gv[v].x, gv[v].y, gv[v].z, gv[v].w};
+      const uint32_t uw[4] = {uv[v].x, uv[v].y, uv[v].z, uv[v].w};
+      uint32_t dg[4], du[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float res_g[2], res_u[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float da = __uint_as_float(r[8 * v + 2 * i + h]);
+          const float g = bf16_bits_to_f32(h ? (gw[i] >> 16) : (gw[i] & 0xffffu));
+          const float u = bf16_bits_to_f32(h ? (uw[i] >> 16) : (uw[i] & 0xffffu));
+          const float s = sigmoid_fast(g);
+          res_g[h] = da * u * s * (1.0f + g * (1.0f - s));
+          res_u[h] = da * g * s;
+        }
+        dg[i] = pack_bf16x2(res_g[0], res_g[1]);
+        du[i] = pack_bf16x2(res_u[0], res_u[1]);
+      }
+      *reinterpret_cast<uint4*>(og + nb + v * 8) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+      *reinterpret_cast<uint4*>(ou + nb + v * 8) = make_uint4(du[0], du[1], du[2], du[3]);
+    }
+  }
+}
+
 template <int MODE, int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const __grid_constant__ CUtensorMap tmOut /* wgrad: dW [E][N1][N2] fp32 */,
     const int32_t* __restrict__ offsets, int E, int K, int N /* dgrad N or wgrad N2 */,
     int N1 /* wgrad only */, const uint16_t* __restrict__ Gp, const uint16_t* __restrict__ Up,
     void* __restrict__ out, int accumulate, uint32_t* __restrict__ status) {
-  using L = Layout<BN, STAGES>;
+  using L = Layout<BN, STAGES, MODE == kWgrad>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -108,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   int* tab0 = reinterpret_cast<int*>(smem + L::kTableOff);
   int* tab1 = tab0 + (kMaxExperts + 1);
   int* scratch = tab1 + (kMaxExperts + 1);
+  int* offs_s = scratch + 33;  // offsets[0..E] in shared memory (read once per CTA)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -142,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   } else {
     total = build_dgrad_tiles(offsets, E, BM, n_tiles, tab0, scratch);
   }
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) offs_s[i] = offsets[i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -153,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
       int stage = 0;
       uint32_t phase = 0;
       for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-        const TileInfo ti = decode_tile<MODE, BN>(t, offsets, tab0, E, K, n_tiles, m_tiles);
+        const TileInfo ti = decode_tile<MODE, BN>(t, offs_s, tab0, E, K, n_tiles, m_tiles);
         for (int kb = 0; kb < ti.nk; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status)) break;
           uint8_t* sa = smem + stage * L::kStageBytes;
@@ -186,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     uint32_t phase = 0;
     uint32_t acc_iter = 0;
     for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-      const TileInfo ti = decode_tile<MODE, BN>(t, offsets, tab0, E, K, n_tiles, m_tiles);
+      const TileInfo ti = decode_tile<MODE, BN>(t, offs_s, tab0, E, K, n_tiles, m_tiles);
       if (ti.nk == 0) continue;
       const uint32_t b = acc_iter & 1u, bphase = (acc_iter >> 1) & 1u;
       if (!__all_sync(kFull, mbar_wait_bounded(&tempty[b], bphase ^ 1u, abort_flag, status)))
@@ -202,29 +280,35 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         tc_fence_after();
         uint8_t* sa = smem + stage * L::kStageBytes;
         uint8_t* sb = sa + L::kABytes;
+        int nkk = BK / UK;  // MMAs of this K block
         if constexpr (MODE == kWgrad) {
           const int valid = ti.row_end - (ti.row0 + kb * BK);
           if (valid < BK) {
-            // zero the K rows that belong to the next expert (or lie past the data)
-            const int nchunk = 2 + BN / 64;
-            const int rows_bad = BK - valid;
-            const int n16 = nchunk * rows_bad * 8;  // 16-byte pieces
-            for (int i = lane; i < n16; i += 32) {
-              const int ch = i / (rows_bad * 8);
-              const int rem = i - ch * rows_bad * 8;
-              const int row = valid + rem / 8;
-              const int piece = rem & 7;
-              uint8_t* base = ch < 2 ? sa + ch * 8192 : sb + (ch - 2) * 8192;
-              *reinterpret_cast<uint4*>(base + row * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
+            // Last K block of the expert: only the 16-row groups that hold valid rows
+            // are multiplied, and the rows of the last such group past the expert's
+            // end (another expert's rows, or unwritten memory) are zeroed first.
+            nkk = (valid + UK - 1) / UK;
+            const int rows_bad = nkk * UK - valid;  // 0..15
+            if (rows_bad > 0) {
+              constexpr int nchunk = 2 + BN / 64;  // 64-wide column chunks of A and B
+              const int per_chunk = rows_bad * 8;  // 16-byte pieces per chunk
+              for (int i = lane; i < nchunk * per_chunk; i += 32) {
+                const int ch = i / per_chunk;
+                const int rem = i - ch * per_chunk;
+                uint8_t* base = ch < 2 ? sa + ch * 8192 : sb + (ch - 2) * 8192;
+                *reinterpret_cast<uint4*>(base + (valid + (rem >> 3)) * 128 + (rem & 7) * 16) =
+                    make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
             }
-            fence_proxy_async_smem();
-            __syncwarp();
           }
         }
         if (lane == 0) {
           const uint32_t a_addr = smem_u32(sa), b_addr = smem_u32(sb);
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk) {
+            if (kk >= nkk) break;
             uint64_t adesc, bdesc;
             if constexpr (MODE == kWgrad)
               adesc = smem_desc_sw128(a_addr + kk * 2048, 8192, 1024);
@@ -251,119 +335,109 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     __syncwarp();
     mbar_wait_bounded(mma_done, 0, abort_flag, status);
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // ---------------- epilogue (warps 2..9) ----------------
+    // Two warps per TMEM lane quarter q = warp % 4; warp half h owns the 32-column
+    // chunks [h * kCW, (h + 1) * kCW) of the tile.  The next chunk's tcgen05.ld is
+    // in flight while the current chunk is written out.
+    constexpr int kCW = BN / 64;  // chunks per warp
+    const int ew = warp - 2;
+    const int q = warp & 3;
+    const int cbase = (ew >> 2) * kCW;
     const int row_in_tile = q * 32 + lane;
+    const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
     uint32_t acc_iter = 0;
+    // wgrad output staging: this warp's two 32 x 32 fp32 buffers (128-byte swizzled rows)
+    uint8_t* obuf = smem + L::kOutOff + ew * 2 * L::kOutBufBytes;
+    uint32_t obuf_iter = 0;
+    uint32_t ra[32], rb[32];
     for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-      const TileInfo ti = decode_tile<MODE, BN>(t, offsets, tab0, E, K, n_tiles, m_tiles);
-      if constexpr (MODE == kWgrad) {
-        float* dW = static_cast<float*>(out) + (size_t)ti.e * N1 * N;
-        const int m = ti.m0 + row_in_tile;
-        if (ti.nk == 0) {
-          if (!accumulate && m < N1) {
-            for (int c = 0; c < BN; c += 4) {
-              const int n = ti.n0 + c;
-              if (n < N)
-                *reinterpret_cast<uint4*>(dW + (size_t)m * N + n) = make_uint4(0, 0, 0, 0);
-            }
-          }
-          continue;
-        }
-        const uint32_t b = acc_iter & 1u, bphase = (acc_iter >> 1) & 1u;
+      const TileInfo ti = decode_tile<MODE, BN>(t, offs_s, tab0, E, K, n_tiles, m_tiles);
+      const bool zero_tile = (MODE == kWgrad) && ti.nk == 0;
+      if (zero_tile && accumulate) continue;  // adding zero changes nothing
+      uint32_t b = 0;
+      if (!zero_tile) {
+        b = acc_iter & 1u;
+        const uint32_t bphase = (acc_iter >> 1) & 1u;
         if (!__all_sync(kFull, mbar_wait_bounded(&tfull[b], bphase, abort_flag, status))) break;
         tc_fence_after();
-        for (int ch = 0; ch < BN / 32; ++ch) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + b * BN + ch * 32, r);
-          tmem_wait_ld();
-          if (m < N1) {
-            float* dst = dW + (size_t)m * N + ti.n0 + ch * 32;
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              if (ti.n0 + ch * 32 + v * 4 < N) {
-                float4 o = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                       __uint_as_float(r[4 * v + 2]),
-                                       __uint_as_float(r[4 * v + 3]));
-                if (accumulate) {
-                  const float4 old = *reinterpret_cast<const float4*>(dst + 4 * v);
-                  o.x += old.x;
-                  o.y += old.y;
-                  o.z += old.z;
-                  o.w += old.w;
-                }
-                *reinterpret_cast<float4*>(dst + 4 * v) = o;
-              }
-            }
-          }
+        tmem_ld_32x32b_x32(lane_base + b * BN + cbase * 32, ra);
+        tmem_wait_ld();
+        reg_fence(ra);
+        if (kCW == 1) {
+          tc_fence_before();
+          mbar_arrive(&tempty[b]);
         }
-        tc_fence_before();
-        mbar_arrive(&tempty[b]);
-        ++acc_iter;
       } else {
-        const uint32_t b = acc_iter & 1u, bphase = (acc_iter >> 1) & 1u;
-        if (!__all_sync(kFull, mbar_wait_bounded(&tfull[b], bphase, abort_flag, status))) break;
-        tc_fence_after();
-        const int row = ti.row0 + row_in_tile;
-        const bool row_ok = row < ti.row_end;
-        for (int ch = 0; ch < BN / 32; ++ch) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + b * BN + ch * 32, r);
-          tmem_wait_ld();
-          if (!row_ok) continue;
-          const int nb = ti.n0 + ch * 32;
-          if constexpr (MODE == kDgradStore) {
-            uint16_t* o = static_cast<uint16_t*>(out) + (size_t)row * N + nb;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (nb + v * 8 < N) {
-                uint4 w;
-                w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-                w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-                w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-                w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-                *reinterpret_cast<uint4*>(o + v * 8) = w;
-              }
+        for (int i = 0; i < 32; ++i) ra[i] = rb[i] = 0u;
+      }
+      const int row = ti.row0 + row_in_tile;  // dgrad output row
+      const bool row_ok = row < ti.row_end;
+      uint4 ga[4], ua[4], gb[4], ub[4];        // SwiGLU: saved g, u of the current / next chunk
+      if constexpr (MODE == kDgradSwiglu) {
+        if (row_ok) load_gu(ga, ua, Gp, Up, row, ti.n0 + cbase * 32, N);
+      }
+      auto step = [&](uint32_t (&cur)[32], uint32_t (&nxt)[32], uint4 (&gc)[4], uint4 (&uc)[4],
+                      uint4 (&gn)[4], uint4 (&un)[4], int i) {
+        const int ch = cbase + i;
+        const bool more = i + 1 < kCW;
+        if (more && !zero_tile) tmem_ld_32x32b_x32(lane_base + b * BN + (ch + 1) * 32, nxt);
+        const int nb = ti.n0 + ch * 32;
+        if constexpr (MODE == kWgrad) {
+          const int mrow = ti.m0 + q * 32;
+          if (mrow < N1 && nb < N) {
+            uint8_t* buf = obuf + (obuf_iter & 1u) * L::kOutBufBytes;
+            ++obuf_iter;
+            if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` read it
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int slot = j ^ (lane & 7);
+              *reinterpret_cast<uint4*>(buf + lane * 128 + slot * 16) =
+                  make_uint4(cur[4 * j], cur[4 * j + 1], cur[4 * j + 2], cur[4 * j + 3]);
             }
-          } else {
-            const uint16_t* gp = Gp + (size_t)row * N + nb;
-            const uint16_t* up = Up + (size_t)row * N + nb;
-            uint16_t* og = static_cast<uint16_t*>(out) + (size_t)row * 2 * N + nb;
-            uint16_t* ou = og + N;
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (nb + v * 8 < N) {
-                const uint4 gv = *reinterpret_cast<const uint4*>(gp + v * 8);
-                const uint4 uv = *reinterpret_cast<const uint4*>(up + v * 8);
-                const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-                const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
-                uint32_t dg[4], du[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  float res_g[2], res_u[2];
-#pragma unroll
-                  for (int h = 0; h < 2; ++h) {
-                    const float da = __uint_as_float(r[8 * v + 2 * i + h]);
-                    const float g = bf16_bits_to_f32(h ? (gw[i] >> 16) : (gw[i] & 0xffffu));
-                    const float u = bf16_bits_to_f32(h ? (uw[i] >> 16) : (uw[i] & 0xffffu));
-                    const float s = sigmoid_fast(g);
-                    res_g[h] = da * u * s * (1.0f + g * (1.0f - s));
-                    res_u[h] = da * g * s;
-                  }
-                  dg[i] = pack_bf16x2(res_g[0], res_g[1]);
-                  du[i] = pack_bf16x2(res_u[0], res_u[1]);
-                }
-                *reinterpret_cast<uint4*>(og + v * 8) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
-                *reinterpret_cast<uint4*>(ou + v * 8) = make_uint4(du[0], du[1], du[2], du[3]);
-              }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (accumulate)
+                tma_reduce_add_3d(&tmOut, buf, nb, mrow, ti.e);
+              else
+                tma_store_3d(&tmOut, buf, nb, mrow, ti.e);
+              bulk_commit_group();
             }
           }
+        } else if constexpr (MODE == kDgradStore) {
+          if (row_ok) epi_store_bf16(cur, static_cast<uint16_t*>(out) + (size_t)row * N, nb, N);
+        } else {
+          if (more && row_ok) load_gu(gn, un, Gp, Up, row, nb + 32, N);
+          if (row_ok) {
+            uint16_t* og = static_cast<uint16_t*>(out) + (size_t)row * 2 * N;
+            epi_swiglu(cur, gc, uc, og, og + N, nb, N);
+          }
         }
-        tc_fence_before();
-        mbar_arrive(&tempty[b]);
-        ++acc_iter;
+        if (more && !zero_tile) {
+          tmem_wait_ld();
+          reg_fence(nxt);
+          if (i + 2 == kCW) {  // last chunk is in registers: the accumulator is free
+            tc_fence_before();
+            mbar_arrive(&tempty[b]);
+          }
+        }
+      };
+#pragma unroll
+      for (int i = 0; i < kCW; ++i) {
+        if (i & 1)
+          step(rb, ra, gb, ub, ga, ua, i);
+        else
+          step(ra, rb, ga, ua, gb, ub, i);
       }
+      if (!zero_tile) ++acc_iter;
     }
+  }
+  if constexpr (MODE == kWgrad) {
+    // shared memory must outlive the bulk stores that read it
+    if (warp >= 2 && lane == 0) bulk_wait_group<0>();  // every epilogue warp
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -421,25 +495,44 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D fp32 map over dW [E][N1][N2], box = 32 (N2) x 32 (N1) x 1, 128-B swizzle (store side).
+bool make_map_out_f32(CUtensorMap* m, void* base, uint64_t E, uint64_t N1, uint64_t N2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {N2, N1, E};
+  cuuint64_t strides[2] = {N2 * 4, N1 * N2 * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 constexpr int kBN = 256;
-constexpr int kStages = 4;
+// dgrad K loops are long (K = H or 2I): 4 stages; wgrad K loops are short
+// (K = m_e) and the fp32 output staging needs 32 KB: 3 stages.
+template <int MODE>
+constexpr int stages_for() { return MODE == kWgrad ? 3 : 4; }
 
 template <int MODE>
-cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const int32_t* offsets,
-                        int E, int K, int N, int N1, const void* Gp, const void* Up, void* out,
-                        int accumulate, uint32_t* status, cudaStream_t s, int grid) {
-  using L = Layout<kBN, kStages>;
+cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
+                        const int32_t* offsets, int E, int K, int N, int N1, const void* Gp,
+                        const void* Up, void* out, int accumulate, uint32_t* status,
+                        cudaStream_t s, int grid) {
+  constexpr int S = stages_for<MODE>();
+  using L = Layout<kBN, S, MODE == kWgrad>;
+  static_assert(L::kAlloc <= 232448, "shared memory over the sm_100 per-block limit");
   static unsigned long long attr_done = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tc<MODE, kBN, kStages>,
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tc<MODE, kBN, S>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (err != cudaSuccess) return err;
     attr_done |= 1ull << dev;
   }
-  grouped_gemm_tc<MODE, kBN, kStages><<<grid, kThreads, L::kAlloc, s>>>(
-      ta, tb, offsets, E, K, N, N1, static_cast<const uint16_t*>(Gp),
+  grouped_gemm_tc<MODE, kBN, S><<<grid, kThreads, L::kAlloc, s>>>(
+      ta, tb, tout, offsets, E, K, N, N1, static_cast<const uint16_t*>(Gp),
       static_cast<const uint16_t*>(Up), out, accumulate, status);
   return cudaGetLastError();
 }
@@ -458,17 +551,19 @@ cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
   }
   const int grid = num_sms();
   if (epi == LRMOE_EPI_SWIGLU_BWD)
-    return launch_mode<kDgradSwiglu>(ta, tb, offsets, E, K, N, 0, Gp, Up, out, 0, status, s, grid);
-  return launch_mode<kDgradStore>(ta, tb, offsets, E, K, N, 0, nullptr, nullptr, out, 0, status, s,
-                                  grid);
+    return launch_mode<kDgradSwiglu>(ta, tb, ta, offsets, E, K, N, 0, Gp, Up, out, 0, status, s,
+                                     grid);
+  return launch_mode<kDgradStore>(ta, tb, ta, offsets, E, K, N, 0, nullptr, nullptr, out, 0, status,
+                                  s, grid);
 }
 
 cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows_cap,
                             const int32_t* offsets, int E, int N1, int N2, float* dW,
                             int accumulate, uint32_t* status, cudaStream_t s, const char** why) {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tout;
   if (!make_map_2d(&ta, grad_rows, (uint64_t)rows_cap, (uint64_t)N1, 64, 64) ||
-      !make_map_2d(&tb, in_rows, (uint64_t)rows_cap, (uint64_t)N2, 64, 64)) {
+      !make_map_2d(&tb, in_rows, (uint64_t)rows_cap, (uint64_t)N2, 64, 64) ||
+      !make_map_out_f32(&tout, dW, (uint64_t)E, (uint64_t)N1, (uint64_t)N2)) {
     *why = "cuTensorMapEncodeTiled failed for a wgrad operand";
     return cudaErrorInvalidValue;
   }
@@ -476,7 +571,7 @@ cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows
       (long long)E * ((N1 + BM - 1) / BM) * ((N2 + kBN - 1) / kBN);
   int grid = num_sms();
   if (total < grid) grid = (int)total;
-  return launch_mode<kWgrad>(ta, tb, offsets, E, 0, N2, N1, nullptr, nullptr, dW, accumulate,
+  return launch_mode<kWgrad>(ta, tb, tout, offsets, E, 0, N2, N1, nullptr, nullptr, dW, accumulate,
                              status, s, grid);
 }
 

@@ -14,6 +14,8 @@
 namespace lrmoe {
 namespace {
 
+constexpr int kUnpackMaxRows = 8;  // retained rows of a token loaded together per column
+
 __device__ __forceinline__ void copy_row(uint4* __restrict__ dst, const uint4* __restrict__ src,
                                          int V, int lane) {
   int c = lane;
@@ -111,28 +113,45 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ d
       r = -1;
     }
     const unsigned have = __ballot_sync(kFull, r >= 0);
+    // retained rows in ascending slot order, compacted: rows[i] for i < nrows
+    const int nrows = __popc(have);
+    int comp = 0;  // lane i: packed row of the i-th retained slot (ascending slot order)
+    {
+      unsigned todo = have;
+      for (int i = 0; todo; ++i) {
+        const int rj = __shfl_sync(kFull, r, __ffs(todo) - 1);
+        if (lane == i) comp = rj;
+        todo &= todo - 1;
+      }
+    }
     for (int c = lane; c < VH; c += 32) {
       float acc[PER];
 #pragma unroll
       for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
-      unsigned todo = have;
-      while (todo) {
-        const int j = __ffs(todo) - 1;
-        todo &= todo - 1;
-        const int row = __shfl_sync(kFull, r, j);
-        const uint4 v = __ldg(dXp + (size_t)row * VH + c);
-        if constexpr (DT == LRMOE_BF16) {
-          const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+      for (int base = 0; base < nrows; base += kUnpackMaxRows) {
+        // all loads of this batch in flight before any add
+        uint4 v[kUnpackMaxRows];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            acc[2 * i] = __fadd_rn(acc[2 * i], bf16_bits_to_f32(ww[i] & 0xffffu));
-            acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], bf16_bits_to_f32(ww[i] >> 16));
+        for (int i = 0; i < kUnpackMaxRows; ++i) {
+          const int row = __shfl_sync(kFull, comp, (base + i) & 31);
+          v[i] = base + i < nrows ? __ldg(dXp + (size_t)row * VH + c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < kUnpackMaxRows; ++i) {
+          if (base + i >= nrows) break;
+          if constexpr (DT == LRMOE_BF16) {
+            const uint32_t ww[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              acc[2 * q] = __fadd_rn(acc[2 * q], bf16_bits_to_f32(ww[q] & 0xffffu));
+              acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_bits_to_f32(ww[q] >> 16));
+            }
+          } else {
+            acc[0] = __fadd_rn(acc[0], __uint_as_float(v[i].x));
+            acc[1] = __fadd_rn(acc[1], __uint_as_float(v[i].y));
+            acc[2] = __fadd_rn(acc[2], __uint_as_float(v[i].z));
+            acc[3] = __fadd_rn(acc[3], __uint_as_float(v[i].w));
           }
-        } else {
-          acc[0] = __fadd_rn(acc[0], __uint_as_float(v.x));
-          acc[1] = __fadd_rn(acc[1], __uint_as_float(v.y));
-          acc[2] = __fadd_rn(acc[2], __uint_as_float(v.z));
-          acc[3] = __fadd_rn(acc[3], __uint_as_float(v.w));
         }
       }
       uint4 o;

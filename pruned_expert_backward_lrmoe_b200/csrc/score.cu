@@ -35,26 +35,46 @@ __device__ __forceinline__ float acc_vec(float acc, const uint4& v) {
   return acc;
 }
 
-// Squared norm of one row of V 16-byte vectors in the canonical order.
-template <lrmoe_dtype DT>
-__device__ __forceinline__ float row_sqnorm(const uint4* __restrict__ row, int V, int lane) {
-  float acc = 0.0f;
-  int c = lane;
-  // four vectors in flight per lane, accumulated in ascending order
-  for (; c + 96 < V; c += 128) {
-    const uint4 v0 = __ldg(row + c);
-    const uint4 v1 = __ldg(row + c + 32);
-    const uint4 v2 = __ldg(row + c + 64);
-    const uint4 v3 = __ldg(row + c + 96);
-    acc = acc_vec<DT>(acc, v0);
-    acc = acc_vec<DT>(acc, v1);
-    acc = acc_vec<DT>(acc, v2);
-    acc = acc_vec<DT>(acc, v3);
+// Vectors a lane keeps in registers per row chunk (rows longer than 32 * kMaxV
+// vectors are processed chunk by chunk, which keeps the same order).
+constexpr int kMaxV = 8;
+
+// Load this lane's vectors c = base + lane + 32 i (i < kMaxV) of a row.
+__device__ __forceinline__ void load_chunk(uint4 (&v)[kMaxV], const uint4* __restrict__ row,
+                                           int base, int V, int lane) {
+#pragma unroll
+  for (int i = 0; i < kMaxV; ++i) {
+    const int c = base + lane + 32 * i;
+    v[i] = c < V ? __ldg(row + c) : make_uint4(0, 0, 0, 0);
   }
-  for (; c < V; c += 32) acc = acc_vec<DT>(acc, __ldg(row + c));
+}
+
+// Accumulate a loaded chunk in ascending vector order (padding vectors are zero).
+template <lrmoe_dtype DT>
+__device__ __forceinline__ float acc_chunk(float acc, const uint4 (&v)[kMaxV], int base, int V,
+                                           int lane) {
+#pragma unroll
+  for (int i = 0; i < kMaxV; ++i)
+    if (base + lane + 32 * i < V) acc = acc_vec<DT>(acc, v[i]);
+  return acc;
+}
+
+__device__ __forceinline__ float butterfly(float acc) {
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(kFull, acc, o));
   return acc;
+}
+
+// Squared norm of a row whose first chunk is already in `v`.
+template <lrmoe_dtype DT>
+__device__ __forceinline__ float row_sqnorm_from(uint4 (&v)[kMaxV],
+                                                 const uint4* __restrict__ row, int V, int lane) {
+  float acc = acc_chunk<DT>(0.0f, v, 0, V, lane);
+  for (int base = 32 * kMaxV; base < V; base += 32 * kMaxV) {
+    load_chunk(v, row, base, V, lane);
+    acc = acc_chunk<DT>(acc, v, base, V, lane);
+  }
+  return butterfly(acc);
 }
 
 template <lrmoe_dtype DT>
@@ -68,24 +88,41 @@ __global__ void __launch_bounds__(256) score_kernel(const int32_t* __restrict__ 
   const int warps_per_block = blockDim.x >> 5;
   for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T;
        t += gridDim.x * warps_per_block) {
-    const float ny = row_sqnorm<DT>(dY + (size_t)t * VH, VH, lane);
-    for (int j = 0; j < k; ++j) {
-      const size_t p = (size_t)t * k + j;
-      const int e = __ldg(idx + p);
-      float s = 0.0f;
-      if (e >= 0 && e < E) {
-        const float na = row_sqnorm<DT>(a + p * VD, VD, lane);
-        const float wp = __ldg(w + p);
-        s = __fmul_rn(__fmul_rn(__fmul_rn(wp, wp), ny), na);
-        if (!isfinite(s)) {
-          if (lane == 0) raise_status(status, LRMOE_ST_NONFINITE);
-          if (isnan(s)) s = __uint_as_float(0x7fffffffu);
-        }
-      } else if (e >= E && lane == 0) {
-        raise_status(status, LRMOE_ST_BAD_EXPERT);
+    // routing slots of this token: lane j holds slot j (k <= 32)
+    const size_t p0 = (size_t)t * k;
+    const int e_l = lane < k ? __ldg(idx + p0 + lane) : -1;
+    const float w_l = lane < k ? __ldg(w + p0 + lane) : 0.0f;
+    const unsigned routed = __ballot_sync(kFull, lane < k && e_l >= 0 && e_l < E);
+    if (__any_sync(kFull, lane < k && e_l >= E) && lane == 0)
+      raise_status(status, LRMOE_ST_BAD_EXPERT);
+
+    uint4 vy[kMaxV], va[kMaxV], vn[kMaxV];
+    load_chunk(vy, dY + (size_t)t * VH, 0, VH, lane);
+    int j = routed ? __ffs(routed) - 1 : -1;
+    if (j >= 0) load_chunk(va, a + (p0 + j) * VD, 0, VD, lane);
+    const float ny = row_sqnorm_from<DT>(vy, dY + (size_t)t * VH, VH, lane);
+
+    float s_mine = 0.0f;  // lane j ends up holding slot j's score
+    unsigned todo = routed;
+    while (todo) {
+      j = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int jn = todo ? __ffs(todo) - 1 : -1;
+      if (jn >= 0) load_chunk(vn, a + (p0 + jn) * VD, 0, VD, lane);  // next row in flight
+      const float na = row_sqnorm_from<DT>(va, a + (p0 + j) * VD, VD, lane);
+      const float wp = __shfl_sync(kFull, w_l, j);
+      float s = __fmul_rn(__fmul_rn(__fmul_rn(wp, wp), ny), na);
+      if (!isfinite(s)) {
+        if (lane == 0) raise_status(status, LRMOE_ST_NONFINITE);
+        if (isnan(s)) s = __uint_as_float(0x7fffffffu);
       }
-      if (lane == 0) score[p] = s;
+      if (lane == j) s_mine = s;
+      if (jn >= 0) {
+#pragma unroll
+        for (int i = 0; i < kMaxV; ++i) va[i] = vn[i];
+      }
     }
+    if (lane < k) score[p0 + lane] = s_mine;
   }
 }
 

@@ -30,7 +30,7 @@ constexpr int kCountThreads = 256;
 constexpr int kScatterWarps = 8;
 constexpr int kTopkThreads = 1024;
 constexpr int kScanSmemInts = 32768;  // E * nchunks kept in shared memory by chunk_scan
-constexpr int kTopkSmemKeys = 40960;  // segments up to this length are selected in smem
+constexpr int kTopkSmemKeys = 24576;  // segments up to this length are staged in smem
 
 __global__ void __launch_bounds__(kCountThreads) chunk_count(const int32_t* __restrict__ idx,
                                                               int P, int E, int chunk,
@@ -201,31 +201,33 @@ __global__ void __launch_bounds__(kScatterWarps * 32) chunk_scatter(
   }
 }
 
-// Block-wide exclusive scan for 1024 threads (32 warps); returns the total too.
-__device__ __forceinline__ uint32_t block_excl_scan_u32(uint32_t v, uint32_t* ws,
-                                                        uint32_t* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  uint32_t incl = v;
+// Block-wide exclusive scan of 64-bit values (two 32-bit counters packed in one
+// word, low and high halves); returns the total too.  blockDim.x <= 1024.
+__device__ __forceinline__ unsigned long long block_excl_scan_u64(unsigned long long v,
+                                                                  unsigned long long* ws,
+                                                                  unsigned long long* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  unsigned long long incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint32_t n = __shfl_up_sync(kFull, incl, o);
+    const unsigned long long n = __shfl_up_sync(kFull, incl, o);
     if (lane >= o) incl += n;
   }
   if (lane == 31) ws[wid] = incl;
   __syncthreads();
   if (wid == 0) {
-    uint32_t s = ws[lane];
-    uint32_t si = s;
+    const unsigned long long x = lane < nw ? ws[lane] : 0ull;
+    unsigned long long xi = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      uint32_t n = __shfl_up_sync(kFull, si, o);
-      if (lane >= o) si += n;
+      const unsigned long long n = __shfl_up_sync(kFull, xi, o);
+      if (lane >= o) xi += n;
     }
-    ws[lane] = si - s;
-    if (lane == 31) ws[32] = si;
+    if (lane < nw) ws[lane] = xi - x;
+    if (lane == 31) ws[32] = xi;
   }
   __syncthreads();
-  const uint32_t r = ws[wid] + incl - v;
+  const unsigned long long r = ws[wid] + incl - v;
   *total = ws[32];
   __syncthreads();
   return r;
@@ -236,9 +238,9 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ seg_start,
     const int32_t* __restrict__ seg_p, const uint32_t* __restrict__ seg_key,
     int32_t* __restrict__ perm, int32_t* __restrict__ pos) {
-  extern __shared__ uint32_t keys_smem[];
+  extern __shared__ uint32_t sm_keys[];  // [kTopkSmemKeys] keys, then [kTopkSmemKeys] pairs
   __shared__ int hist[256];
-  __shared__ uint32_t scan_ws[33];
+  __shared__ unsigned long long scan_ws[33];
   __shared__ int found_bin, found_above;
   const int e = blockIdx.x;
   const int c = counts[e];
@@ -246,11 +248,12 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
   const int s0 = seg_start[e];
   const int out0 = offsets[e];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nt = blockDim.x;
   const int32_t* sp = seg_p + s0;
   const uint32_t* sk = seg_key + s0;
 
   if (m == c) {  // everything stays, already in ascending p
-    for (int i = tid; i < c; i += blockDim.x) {
+    for (int i = tid; i < c; i += nt) {
       const int p = sp[i];
       perm[out0 + i] = p;
       pos[p] = out0 + i;
@@ -258,15 +261,39 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
     return;
   }
   if (m == 0) {
-    for (int i = tid; i < c; i += blockDim.x) pos[sp[i]] = -1;
+    for (int i = tid; i < c; i += nt) pos[sp[i]] = -1;
     return;
   }
 
+  // stage the segment in shared memory (four loads in flight per thread)
   const bool in_smem = c <= kTopkSmemKeys;
   const uint32_t* K = sk;
+  const int32_t* PP = sp;
   if (in_smem) {
-    for (int i = tid; i < c; i += blockDim.x) keys_smem[i] = sk[i];
-    K = keys_smem;
+    uint32_t* ks = sm_keys;
+    int32_t* ps = reinterpret_cast<int32_t*>(sm_keys + kTopkSmemKeys);
+    for (int i0 = 0; i0 < c; i0 += 4 * nt) {
+      uint32_t kv[4];
+      int pv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * nt + tid;
+        if (i < c) {
+          kv[u] = sk[i];
+          pv[u] = sp[i];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * nt + tid;
+        if (i < c) {
+          ks[i] = kv[u];
+          ps[i] = pv[u];
+        }
+      }
+    }
+    K = ks;
+    PP = ps;
   }
   __syncthreads();
 
@@ -276,9 +303,9 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
   for (int d = 3; d >= 0; --d) {
     const int shift = 8 * d;
     const uint32_t hmask = d == 3 ? 0u : (0xffffffffu << (shift + 8));
-    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+    for (int i = tid; i < 256; i += nt) hist[i] = 0;
     __syncthreads();
-    for (int i0 = 0; i0 < c; i0 += blockDim.x) {
+    for (int i0 = 0; i0 < c; i0 += nt) {
       const int i = i0 + tid;
       int digit = -1;
       if (i < c) {
@@ -319,37 +346,34 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
     __syncthreads();
   }
   const uint32_t tau = prefix;
-  const uint32_t need_eq = (uint32_t)need;  // equal keys to keep, in ascending p
+  const unsigned long long need_eq = (unsigned long long)need;  // equal keys kept, in ascending p
 
-  // ordered compaction
-  uint32_t carry_gt = 0, carry_eq = 0;
-  for (int i0 = 0; i0 < c; i0 += blockDim.x) {
-    const int i = i0 + tid;
-    uint32_t key = 0;
-    bool gt = false, eq = false;
-    if (i < c) {
-      key = K[i];
-      gt = key > tau;
-      eq = key == tau;
+  // ordered compaction: thread t owns the contiguous run [t*R, t*R + R); one scan
+  // of (above, equal) counts gives every run its starting row.
+  const int R = (c + nt - 1) / nt;
+  const int b0 = min(c, tid * R), b1 = min(c, b0 + R);
+  unsigned long long ngt = 0, neq = 0;
+  for (int i = b0; i < b1; ++i) {
+    const uint32_t key = K[i];
+    ngt += key > tau;
+    neq += key == tau;
+  }
+  unsigned long long tot;
+  const unsigned long long ex = block_excl_scan_u64(ngt | (neq << 32), scan_ws, &tot);
+  unsigned long long gt_before = ex & 0xffffffffull, eq_before = ex >> 32;
+  for (int i = b0; i < b1; ++i) {
+    const uint32_t key = K[i];
+    const int p = PP[i];
+    const bool gt = key > tau, eq = key == tau;
+    if (gt || (eq && eq_before < need_eq)) {
+      const int row = out0 + (int)(gt_before + (eq_before < need_eq ? eq_before : need_eq));
+      perm[row] = p;
+      pos[p] = row;
+    } else {
+      pos[p] = -1;
     }
-    const uint32_t packed = (gt ? 1u : 0u) | (eq ? 0x10000u : 0u);
-    uint32_t tot;
-    const uint32_t ex = block_excl_scan_u32(packed, scan_ws, &tot);
-    if (i < c) {
-      const uint32_t gt_before = carry_gt + (ex & 0xffffu);
-      const uint32_t eq_before = carry_eq + (ex >> 16);
-      const int p = sp[i];
-      const bool keep = gt || (eq && eq_before < need_eq);
-      if (keep) {
-        const int row = out0 + (int)(gt_before + min(eq_before, need_eq));
-        perm[row] = p;
-        pos[p] = row;
-      } else {
-        pos[p] = -1;
-      }
-    }
-    carry_gt += tot & 0xffffu;
-    carry_eq += tot >> 16;
+    gt_before += gt;
+    eq_before += eq;
   }
 }
 
@@ -412,7 +436,7 @@ cudaError_t launch_select(const int32_t* idx, const float* score, int T, int k, 
     cudaFuncSetAttribute(chunk_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kScatterWarps * 4096 * 4);
     cudaFuncSetAttribute(expert_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kTopkSmemKeys * 4);
+                         kTopkSmemKeys * 8);
     attrs_set |= 1ull << dev;
   }
   chunk_count<<<L.nchunks, kCountThreads, E * 4, s>>>(idx, P, E, L.chunk, L.nchunks, cc, pos,
@@ -424,7 +448,7 @@ cudaError_t launch_select(const int32_t* idx, const float* score, int T, int k, 
   chunk_scatter<<<L.nchunks, kScatterWarps * 32, kScatterWarps * E * 4, s>>>(
       idx, reinterpret_cast<const uint32_t*>(score), P, E, L.chunk, L.nchunks, cc, seg_start,
       seg_p, seg_key);
-  expert_topk<<<E, kTopkThreads, kTopkSmemKeys * 4, s>>>(counts, kept, offsets, seg_start, seg_p,
+  expert_topk<<<E, kTopkThreads, kTopkSmemKeys * 8, s>>>(counts, kept, offsets, seg_start, seg_p,
                                                          seg_key, perm, pos);
   return cudaGetLastError();
 }
@@ -483,7 +507,7 @@ cudaError_t launch_select_noalloc(const int32_t* idx, const float* score, int T,
     cudaFuncSetAttribute(chunk_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kScatterWarps * 4096 * 4);
     cudaFuncSetAttribute(expert_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kTopkSmemKeys * 4);
+                         kTopkSmemKeys * 8);
     attrs_set |= 1ull << dev;
   }
   chunk_count<<<L.nchunks, kCountThreads, E * 4, s>>>(idx, P, E, L.chunk, L.nchunks, cc, pos,
@@ -495,7 +519,7 @@ cudaError_t launch_select_noalloc(const int32_t* idx, const float* score, int T,
   chunk_scatter<<<L.nchunks, kScatterWarps * 32, kScatterWarps * E * 4, s>>>(
       idx, reinterpret_cast<const uint32_t*>(score), P, E, L.chunk, L.nchunks, cc, seg_start,
       seg_p, seg_key);
-  expert_topk<<<E, kTopkThreads, kTopkSmemKeys * 4, s>>>(counts, kept, offsets, seg_start, seg_p,
+  expert_topk<<<E, kTopkThreads, kTopkSmemKeys * 8, s>>>(counts, kept, offsets, seg_start, seg_p,
                                                          seg_key, perm, pos);
   return cudaGetLastError();
 }
