@@ -20,6 +20,8 @@
 // Every mbarrier wait is bounded (LRMOE_ST_TIMEOUT, then a clean exit).
 #include <cuda.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "grouped.cuh"
 #include "launch.h"
@@ -36,6 +38,16 @@ constexpr int kEpiThreads = 32 * kEpiWarps;
 
 enum Mode : int { kDgradStore = 0, kDgradSwiglu = 1, kWgrad = 2 };
 
+// Dynamic tile scheduling.  Each CTA's producer takes the next tile index from a
+// global counter and hands it to the MMA and epilogue warps through a ring of
+// kRing shared-memory slots, so faster SMs take more tiles.  The counters live
+// here, one pair (next tile, CTAs done) per slot; launches rotate over
+// kSchedSlots slots, and the last CTA of a launch to finish puts its pair back
+// to zero.  Up to kSchedSlots grouped-GEMM launches may run at once per device.
+constexpr int kRing = 4;
+constexpr int kSchedSlots = 64;
+__device__ unsigned int g_sched[kSchedSlots][2];
+
 template <int BN, int STAGES, bool STAGED_OUT>
 struct Layout {
   static constexpr int kABytes = BM * BK * 2;                 // 16 KB
@@ -49,9 +61,9 @@ struct Layout {
   // tile table, expert order / sizes, scan scratch, and a copy of offsets[0..E]
   static constexpr int kTableInts = 3 * (kMaxExperts + 1) + 33;
   static constexpr int kBarOff = kOutOff + kOutBytes;         // 8-byte barriers
-  static constexpr int kNumBars = 2 * STAGES + 5;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;     // tmem base, abort flag
-  static constexpr int kTableOff = kMiscOff + 16;
+  static constexpr int kNumBars = 2 * STAGES + 5 + 2 * kRing;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;     // tmem base, abort flag, tile ring
+  static constexpr int kTableOff = kMiscOff + 16 + 4 * kRing;
   static constexpr int kBytes = kTableOff + kTableInts * 4;
   static constexpr int kAlloc = kBytes + 1024;                // slack for 1024-B alignment
 };
@@ -168,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     const __grid_constant__ CUtensorMap tmOut /* wgrad: dW [E][N1][N2] fp32 */,
     const int32_t* __restrict__ offsets, int E, int K, int N /* dgrad N or wgrad N2 */,
     int N1 /* wgrad only */, const uint16_t* __restrict__ Gp, const uint16_t* __restrict__ Up,
-    void* __restrict__ out, int accumulate, uint32_t* __restrict__ status) {
+    void* __restrict__ out, int accumulate, uint32_t* __restrict__ status, int sched_slot) {
   using L = Layout<BN, STAGES, MODE == kWgrad>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -179,8 +191,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   uint64_t* tfull = bars + 2 * STAGES;      // [2]
   uint64_t* tempty = bars + 2 * STAGES + 2; // [2]
   uint64_t* mma_done = bars + 2 * STAGES + 4;
+  uint64_t* ring_full = bars + 2 * STAGES + 5;            // [kRing]
+  uint64_t* ring_empty = bars + 2 * STAGES + 5 + kRing;   // [kRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  volatile int* ring = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 16);  // [kRing]
+  unsigned int* sched = g_sched[sched_slot];
   int* tab0 = reinterpret_cast<int*>(smem + L::kTableOff);
   int* tab1 = tab0 + (kMaxExperts + 1);
   int* scratch = tab1 + (kMaxExperts + 1);
@@ -198,6 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
       mbar_init(&tempty[i], kEpiThreads);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&ring_full[i], 1);
+      mbar_init(&ring_empty[i], 1 + kEpiWarps);  // MMA warp + each epilogue warp
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -225,15 +245,40 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Tile of the it-th round for the MMA and epilogue warps (-1: no more tiles).
+  auto next_tile = [&](int it) -> int {
+    const int slot = it % kRing;
+    const bool ok = __all_sync(
+        kFull, mbar_wait_bounded(&ring_full[slot], (uint32_t)(it / kRing) & 1u, abort_flag, status));
+    const int t = ok ? ring[slot] : -1;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ring_empty[slot]);
+    return t;
+  };
+
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (and tile scheduler) ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+      unsigned int next = atomicAdd(&sched[0], 1u);
+      for (int it = 0;; ++it) {
+        const int slot = it % kRing;
+        int t = (int)next;
+        if (!mbar_wait_bounded(&ring_empty[slot], ((uint32_t)(it / kRing) & 1u) ^ 1u, abort_flag,
+                               status) ||
+            t >= total || *abort_flag)
+          t = -1;
+        ring[slot] = t;
+        mbar_arrive(&ring_full[slot]);
+        if (t < 0) break;
         const TileInfo ti = decode_tile<MODE, BN>(t, offs_s, tab0, E, K, n_tiles, m_tiles);
+        if (ti.nk == 0) next = atomicAdd(&sched[0], 1u);
         for (int kb = 0; kb < ti.nk; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status)) break;
+          // claim the following tile only now, a few K blocks before this one ends,
+          // so that no CTA sits on a tile it cannot start soon
+          if (kb == ti.nk - 1) next = atomicAdd(&sched[0], 1u);
           uint8_t* sa = smem + stage * L::kStageBytes;
           uint8_t* sb = sa + L::kABytes;
           mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
@@ -263,7 +308,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     int stage = 0;
     uint32_t phase = 0;
     uint32_t acc_iter = 0;
-    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+    for (int it = 0;; ++it) {
+      const int t = next_tile(it);
+      if (t < 0) break;
       const TileInfo ti = decode_tile<MODE, BN>(t, offs_s, tab0, E, K, n_tiles, m_tiles);
       if (ti.nk == 0) continue;
       const uint32_t b = acc_iter & 1u, bphase = (acc_iter >> 1) & 1u;
@@ -350,7 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     uint8_t* obuf = smem + L::kOutOff + ew * 2 * L::kOutBufBytes;
     uint32_t obuf_iter = 0;
     uint32_t ra[32], rb[32];
-    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+    for (int it = 0;; ++it) {
+      const int t = next_tile(it);
+      if (t < 0) break;
       const TileInfo ti = decode_tile<MODE, BN>(t, offs_s, tab0, E, K, n_tiles, m_tiles);
       const bool zero_tile = (MODE == kWgrad) && ti.nk == 0;
       if (zero_tile && accumulate) continue;  // adding zero changes nothing
@@ -443,6 +492,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, 2 * BN);
+  if (threadIdx.x == 0) {
+    // every tile request of this CTA is done: the last CTA out zeroes the slot
+    __threadfence();
+    if (atomicAdd(&sched[1], 1u) == gridDim.x - 1) {
+      sched[0] = 0;
+      sched[1] = 0;
+      __threadfence();
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -508,6 +566,9 @@ bool make_map_out_f32(CUtensorMap* m, void* base, uint64_t E, uint64_t N1, uint6
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch counter of all grouped-GEMM kernels (picks the scheduling slot).
+std::atomic<unsigned int> g_launches{0};
+
 constexpr int kBN = 256;
 // dgrad K loops are long (K = H or 2I): 4 stages; wgrad K loops are short
 // (K = m_e) and the fp32 output staging needs 32 KB: 3 stages.
@@ -531,9 +592,10 @@ cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
     if (err != cudaSuccess) return err;
     attr_done |= 1ull << dev;
   }
+  const int slot = (int)(g_launches.fetch_add(1u) % kSchedSlots);
   grouped_gemm_tc<MODE, kBN, S><<<grid, kThreads, L::kAlloc, s>>>(
       ta, tb, tout, offsets, E, K, N, N1, static_cast<const uint16_t*>(Gp),
-      static_cast<const uint16_t*>(Up), out, accumulate, status);
+      static_cast<const uint16_t*>(Up), out, accumulate, status, slot);
   return cudaGetLastError();
 }
 
