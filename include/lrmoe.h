@@ -21,8 +21,12 @@
  *   - Every data pointer is a DEVICE pointer, 16-byte aligned, rows contiguous
  *     and row-major.  `stream` is a cudaStream_t passed as void* (NULL = the
  *     legacy default stream).
- *   - The caller owns all memory.  The library allocates nothing and keeps no
- *     state between calls; calls are re-entrant.
+ *   - The caller owns all memory.  The library allocates nothing.  Its only
+ *     device-side state is fixed and internal: 64 pairs of tile counters that
+ *     the grouped GEMMs use for dynamic tile scheduling (each launch takes the
+ *     next pair and leaves it zeroed, so up to 64 grouped-GEMM launches may be
+ *     in flight at once on one device), and the scratch array of
+ *     lrmoe_select_quota_noalloc.  Calls are thread-safe on the host.
  *   - Calls only enqueue work on `stream` and never synchronise the host.
  *     Counts and offsets stay on the device; later kernels read them there.
  *   - Errors a host can see (null pointer, size <= 0, feature size not a
@@ -268,6 +272,16 @@ typedef struct {
 
 int lrmoe_pruned_backward(const lrmoe_buffers* b, int T, int k, int E, int H, int I,
                           int rows_cap, lrmoe_dtype dt, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostic (no counterpart in the pages): run one bounded device-side wait
+ * on a barrier that nothing ever completes, with a limit of `limit_us`
+ * microseconds (1 .. 1 000 000).  The kernel gives up, sets LRMOE_ST_TIMEOUT
+ * in *status (device memory) and returns; the context stays usable.  It
+ * checks the mechanism that every pipeline wait of the grouped GEMMs uses
+ * (their limit is 2 s) without hanging or faulting the GPU.
+ * ------------------------------------------------------------------------- */
+int lrmoe_selftest_bounded_wait(uint32_t limit_us, uint32_t* status, void* stream);
 
 #ifdef __cplusplus
 }

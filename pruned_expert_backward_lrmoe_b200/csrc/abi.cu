@@ -266,6 +266,15 @@ int lrmoe_unpack(const void* dXp, int rows_cap, const int32_t* pos, int T, int k
   return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_unpack launch");
 }
 
+int lrmoe_selftest_bounded_wait(uint32_t limit_us, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u) == 0,
+          "status is null or misaligned");
+  REQUIRE(limit_us >= 1 && limit_us <= 1000000u, "limit_us=%u outside [1, 1000000]", limit_us);
+  cudaError_t e = launch_selftest_wait(limit_us, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_selftest_bounded_wait launch");
+}
+
 int lrmoe_pruned_backward(const lrmoe_buffers* b, int T, int k, int E, int H, int I,
                           int rows_cap, lrmoe_dtype dt, void* stream) {
   g_last_error[0] = 0;

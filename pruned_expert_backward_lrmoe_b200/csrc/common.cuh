@@ -99,18 +99,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar`, giving up after kWaitLimitNs or when
-// another role has raised `*abort`.  Returns false on give-up (and then sets
-// *abort and LRMOE_ST_TIMEOUT).
+// Wait for phase `parity` of `bar`, giving up after `limit_ns` (default
+// kWaitLimitNs) or when another role has raised `*abort`.  Returns false on
+// give-up (and then sets *abort and LRMOE_ST_TIMEOUT).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort, uint32_t* status) {
+                                                  volatile int* abort, uint32_t* status,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         *abort = 1;
         raise_status(status, LRMOE_ST_TIMEOUT);
         return false;
@@ -272,6 +273,22 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------
+// Every kernel of the path calls pdl_wait() before it touches memory that an
+// earlier kernel wrote, then pdl_trigger() so that the next kernel in the
+// stream may be launched (its own prologue overlaps this kernel's tail; it
+// waits in its pdl_wait() until this grid has finished).  Triggering only after
+// the wait keeps the chain ordered: a kernel can start only once every kernel
+// before its predecessor has completed.  Both are no-ops without the launch
+// attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------

@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(NT) dgrad_simt_kernel(
   __shared__ int scratch[33];
   __shared__ float As[BK][BM + 4];
   __shared__ float Bs[BK][BN];
+  pdl_wait();
+  pdl_trigger();
   const int n_tiles = (N + BN - 1) / BN;
   const int total = build_dgrad_tiles(offsets, E, BM, n_tiles, tstart, scratch);
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -99,6 +101,8 @@ __global__ void __launch_bounds__(NT) wgrad_simt_kernel(
     int accumulate) {
   __shared__ float As[BK][BM];
   __shared__ float Bs[BK][BN];
+  pdl_wait();
+  pdl_trigger();
   const int m_tiles = (N1 + BM - 1) / BM, n_tiles = (N2 + BN - 1) / BN;
   const int per_e = m_tiles * n_tiles;
   const int total = per_e * E;
@@ -158,10 +162,10 @@ cudaError_t launch_dgrad_simt(const void* rows, int rows_cap, const void* W,
   (void)rows_cap;
   (void)dt;
   (void)status;
-  dgrad_simt_kernel<<<num_sms() * 4, NT, 0, s>>>(
-      static_cast<const float*>(rows), static_cast<const float*>(W), offsets, E, K, N, (int)epi,
-      static_cast<const float*>(Gp), static_cast<const float*>(Up), static_cast<float*>(out));
-  return cudaGetLastError();
+  return launch_pdl(dgrad_simt_kernel, dim3(num_sms() * 4), dim3(NT), 0, s,
+                    static_cast<const float*>(rows), static_cast<const float*>(W), offsets, E, K,
+                    N, (int)epi, static_cast<const float*>(Gp), static_cast<const float*>(Up),
+                    static_cast<float*>(out));
 }
 
 cudaError_t launch_wgrad_simt(const void* grad_rows, const void* in_rows, int rows_cap,
@@ -170,10 +174,9 @@ cudaError_t launch_wgrad_simt(const void* grad_rows, const void* in_rows, int ro
   (void)rows_cap;
   (void)dt;
   (void)status;
-  wgrad_simt_kernel<<<num_sms() * 4, NT, 0, s>>>(static_cast<const float*>(grad_rows),
-                                                 static_cast<const float*>(in_rows), offsets, E,
-                                                 N1, N2, dW, accumulate);
-  return cudaGetLastError();
+  return launch_pdl(wgrad_simt_kernel, dim3(num_sms() * 4), dim3(NT), 0, s,
+                    static_cast<const float*>(grad_rows), static_cast<const float*>(in_rows),
+                    offsets, E, N1, N2, dW, accumulate);
 }
 
 }  // namespace lrmoe

@@ -229,6 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
+  // everything above touches no global memory; from here on, earlier kernels' outputs
+  pdl_wait();
+  pdl_trigger();
   // tile table
   const int n_tiles = (N + BN - 1) / BN;
   int m_tiles = 0, total;
@@ -593,10 +596,9 @@ cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
     attr_done |= 1ull << dev;
   }
   const int slot = (int)(g_launches.fetch_add(1u) % kSchedSlots);
-  grouped_gemm_tc<MODE, kBN, S><<<grid, kThreads, L::kAlloc, s>>>(
-      ta, tb, tout, offsets, E, K, N, N1, static_cast<const uint16_t*>(Gp),
-      static_cast<const uint16_t*>(Up), out, accumulate, status, slot);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_tc<MODE, kBN, S>, dim3(grid), dim3(kThreads), (size_t)L::kAlloc,
+                    s, ta, tb, tout, offsets, E, K, N, N1, static_cast<const uint16_t*>(Gp),
+                    static_cast<const uint16_t*>(Up), out, accumulate, status, slot);
 }
 
 }  // namespace

@@ -13,6 +13,25 @@ namespace lrmoe {
 // Largest expert count the grouped GEMMs build their tile table for.
 constexpr int kMaxGroupedExperts = 1024;
 
+// Launch `kernel` on `s` with programmatic stream serialization allowed, so
+// that it may start while the previous kernel in the stream drains (the
+// kernels order themselves with griddepcontrol.wait / launch_dependents).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 int num_sms();
 
 cudaError_t launch_score(const int32_t* idx, const float* w, int T, int k, int E, const void* dY,
@@ -55,6 +74,9 @@ cudaError_t launch_dgrad_simt(const void* rows, int rows_cap, const void* W,
 cudaError_t launch_wgrad_simt(const void* grad_rows, const void* in_rows, int rows_cap,
                               const int32_t* offsets, int E, int N1, int N2, lrmoe_dtype dt,
                               float* dW, int accumulate, uint32_t* status, cudaStream_t s);
+
+// diagnostic: a bounded wait that must time out
+cudaError_t launch_selftest_wait(uint32_t limit_us, uint32_t* status, cudaStream_t s);
 
 // tcgen05 grouped GEMMs (bf16 storage)
 cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,

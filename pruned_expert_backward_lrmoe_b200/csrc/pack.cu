@@ -74,6 +74,8 @@ __global__ void __launch_bounds__(256) pack_kernel(
     uint4* __restrict__ Up, int rows_cap, uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
+  pdl_wait();
+  pdl_trigger();
   int M = offsets[E];
   if (M > rows_cap) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
@@ -105,6 +107,8 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ d
   constexpr int PER = DT == LRMOE_BF16 ? 8 : 4;
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
+  pdl_wait();
+  pdl_trigger();
   for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
     // retained rows of this token, in ascending slot order (k <= 32)
     int r = lane < k ? pos[(size_t)t * k + lane] : -1;
@@ -182,17 +186,11 @@ cudaError_t launch_pack(const int32_t* perm, const int32_t* offsets, const float
   auto A = static_cast<const uint4*>(a);
   auto G = static_cast<const uint4*>(g);
   auto U = static_cast<const uint4*>(u);
-  if (dt == LRMOE_BF16)
-    pack_kernel<LRMOE_BF16><<<blocks, 256, 0, s>>>(
-        perm, offsets, E, w, T * k, k, X, D, VH, A, G, U, VI, static_cast<uint4*>(Xp),
-        static_cast<uint4*>(DYp), static_cast<uint4*>(Ap), static_cast<uint4*>(Gp),
-        static_cast<uint4*>(Up), rows_cap, status);
-  else
-    pack_kernel<LRMOE_F32><<<blocks, 256, 0, s>>>(
-        perm, offsets, E, w, T * k, k, X, D, VH, A, G, U, VI, static_cast<uint4*>(Xp),
-        static_cast<uint4*>(DYp), static_cast<uint4*>(Ap), static_cast<uint4*>(Gp),
-        static_cast<uint4*>(Up), rows_cap, status);
-  return cudaGetLastError();
+  auto kern = dt == LRMOE_BF16 ? pack_kernel<LRMOE_BF16> : pack_kernel<LRMOE_F32>;
+  return launch_pdl(kern, dim3(blocks), dim3(256), 0, s, perm, offsets, E, w, T * k, k, X, D, VH,
+                    A, G, U, VI, static_cast<uint4*>(Xp), static_cast<uint4*>(DYp),
+                    static_cast<uint4*>(Ap), static_cast<uint4*>(Gp), static_cast<uint4*>(Up),
+                    rows_cap, status);
 }
 
 cudaError_t launch_unpack(const void* dXp, int rows_cap, const int32_t* pos, int T, int k, int H,
@@ -203,14 +201,9 @@ cudaError_t launch_unpack(const void* dXp, int rows_cap, const int32_t* pos, int
   int blocks = (T + wpb - 1) / wpb;
   const int maxb = num_sms() * 8;
   if (blocks > maxb) blocks = maxb;
-  if (dt == LRMOE_BF16)
-    unpack_kernel<LRMOE_BF16><<<blocks, 256, 0, s>>>(static_cast<const uint4*>(dXp), rows_cap,
-                                                      pos, T, k, VH, static_cast<uint4*>(dX),
-                                                      status);
-  else
-    unpack_kernel<LRMOE_F32><<<blocks, 256, 0, s>>>(static_cast<const uint4*>(dXp), rows_cap, pos,
-                                                     T, k, VH, static_cast<uint4*>(dX), status);
-  return cudaGetLastError();
+  auto kern = dt == LRMOE_BF16 ? unpack_kernel<LRMOE_BF16> : unpack_kernel<LRMOE_F32>;
+  return launch_pdl(kern, dim3(blocks), dim3(256), 0, s, static_cast<const uint4*>(dXp), rows_cap,
+                    pos, T, k, VH, static_cast<uint4*>(dX), status);
 }
 
 }  // namespace lrmoe

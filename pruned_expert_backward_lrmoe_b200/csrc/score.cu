@@ -86,6 +86,8 @@ __global__ void __launch_bounds__(256) score_kernel(const int32_t* __restrict__ 
                                                     uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const int warps_per_block = blockDim.x >> 5;
+  pdl_wait();
+  pdl_trigger();
   for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T;
        t += gridDim.x * warps_per_block) {
     // routing slots of this token: lane j holds slot j (k <= 32)
@@ -137,15 +139,10 @@ cudaError_t launch_score(const int32_t* idx, const float* w, int T, int k, int E
   const int blocks_needed = (T + wpb - 1) / wpb;
   const int max_blocks = num_sms() * (2048 / threads);
   const int blocks = blocks_needed < max_blocks ? blocks_needed : max_blocks;
-  if (dt == LRMOE_BF16)
-    score_kernel<LRMOE_BF16><<<blocks, threads, 0, s>>>(
-        idx, w, T, k, E, static_cast<const uint4*>(dY), VH, static_cast<const uint4*>(a), VD,
-        score, status);
-  else
-    score_kernel<LRMOE_F32><<<blocks, threads, 0, s>>>(
-        idx, w, T, k, E, static_cast<const uint4*>(dY), VH, static_cast<const uint4*>(a), VD,
-        score, status);
-  return cudaGetLastError();
+  auto kern = dt == LRMOE_BF16 ? score_kernel<LRMOE_BF16> : score_kernel<LRMOE_F32>;
+  return launch_pdl(kern, dim3(blocks), dim3(threads), 0, s, idx, w, T, k, E,
+                    static_cast<const uint4*>(dY), VH, static_cast<const uint4*>(a), VD, score,
+                    status);
 }
 
 }  // namespace lrmoe

@@ -40,17 +40,32 @@ __global__ void __launch_bounds__(kCountThreads) chunk_count(const int32_t* __re
   extern __shared__ int hist[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
+  pdl_wait();
+  pdl_trigger();
   const int c = blockIdx.x;
   const int begin = c * chunk;
   const int end = min(P, begin + chunk);
   bool bad = false;
-  for (int p = begin + threadIdx.x; p < end; p += blockDim.x) {
-    const int e = __ldg(idx + p);
-    if (e >= 0 && e < E) {
-      atomicAdd(&hist[e], 1);
+  // four consecutive pairs per thread and pass, one 16-byte load when in range
+  for (int p0 = begin + 4 * threadIdx.x; p0 < end; p0 += 4 * blockDim.x) {
+    int ev[4];
+    if (p0 + 3 < end) {
+      const int4 v = __ldg(reinterpret_cast<const int4*>(idx + p0));
+      ev[0] = v.x, ev[1] = v.y, ev[2] = v.z, ev[3] = v.w;
     } else {
-      pos[p] = -1;
-      bad |= (e >= E);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ev[i] = p0 + i < end ? __ldg(idx + p0 + i) : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = ev[i];
+      if (p0 + i >= end) break;
+      if (e >= 0 && e < E) {
+        atomicAdd(&hist[e], 1);
+      } else {
+        pos[p0 + i] = -1;
+        bad |= (e >= E);
+      }
     }
   }
   if (__any_sync(kFull, bad) && (threadIdx.x & 31) == 0) raise_status(status, LRMOE_ST_BAD_EXPERT);
@@ -94,8 +109,24 @@ __global__ void __launch_bounds__(kScanThreads) chunk_scan(int32_t* __restrict__
   const bool in_smem = (size_t)E * nchunks <= (size_t)kScanSmemInts;
   int* mat = in_smem ? ccs : cc;
   const int n = E * nchunks;
-  if (in_smem)
-    for (int i = threadIdx.x; i < n; i += blockDim.x) ccs[i] = cc[i];
+  pdl_wait();
+  pdl_trigger();
+  if (in_smem) {
+    // eight loads in flight per thread, then the stores
+    for (int i0 = 0; i0 < n; i0 += 8 * blockDim.x) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x + threadIdx.x;
+        v[u] = i < n ? __ldcg(cc + i) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x + threadIdx.x;
+        if (i < n) ccs[i] = v[u];
+      }
+    }
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int e = wid; e < E; e += nw) {
@@ -165,10 +196,20 @@ __global__ void __launch_bounds__(kScatterWarps * 32) chunk_scatter(
   const int wend = min(end, wbeg + sub);
   for (int i = threadIdx.x; i < kScatterWarps * E; i += blockDim.x) wbase[i] = 0;
   __syncthreads();
+  pdl_wait();
+  pdl_trigger();
   int* mine = wbase + wid * E;
-  for (int p = wbeg + lane; p < wend; p += 32) {
-    const int e = __ldg(idx + p);
-    if (e >= 0 && e < E) atomicAdd(&mine[e], 1);
+  constexpr int kSteps = 4;  // 32-pair steps whose loads are in flight together
+  for (int q0 = wbeg; q0 < wend; q0 += 32 * kSteps) {
+    int ev[kSteps];
+#pragma unroll
+    for (int s = 0; s < kSteps; ++s) {
+      const int p = q0 + 32 * s + lane;
+      ev[s] = p < wend ? __ldg(idx + p) : -1;
+    }
+#pragma unroll
+    for (int s = 0; s < kSteps; ++s)
+      if (ev[s] >= 0 && ev[s] < E) atomicAdd(&mine[ev[s]], 1);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -182,22 +223,32 @@ __global__ void __launch_bounds__(kScatterWarps * 32) chunk_scatter(
   }
   __syncthreads();
   const unsigned lt = (1u << lane) - 1u;
-  for (int p0 = wbeg; p0 < wend; p0 += 32) {
-    const int p = p0 + lane;
-    const int e = p < wend ? __ldg(idx + p) : -1;
-    const bool valid = e >= 0 && e < E;
-    const int key = valid ? e : -1;
-    const unsigned m = __match_any_sync(kFull, key);
-    int base = 0;
-    if (valid) {
-      base = mine[e];
-      const int dst = base + __popc(m & lt);
-      seg_p[dst] = p;
-      seg_key[dst] = __ldg(score_bits + p);
+  for (int q0 = wbeg; q0 < wend; q0 += 32 * kSteps) {
+    int ev[kSteps];
+    uint32_t sv[kSteps];
+#pragma unroll
+    for (int s = 0; s < kSteps; ++s) {
+      const int p = q0 + 32 * s + lane;
+      ev[s] = p < wend ? __ldg(idx + p) : -1;
+      sv[s] = p < wend ? __ldg(score_bits + p) : 0u;
     }
-    __syncwarp();
-    if (valid && lane == __ffs(m) - 1) mine[e] = base + __popc(m);
-    __syncwarp();
+#pragma unroll
+    for (int s = 0; s < kSteps; ++s) {  // steps in ascending pair order
+      const int p = q0 + 32 * s + lane;
+      const int e = ev[s];
+      const bool valid = e >= 0 && e < E;
+      const unsigned m = __match_any_sync(kFull, valid ? e : -1);
+      int base = 0;
+      if (valid) {
+        base = mine[e];
+        const int dst = base + __popc(m & lt);
+        seg_p[dst] = p;
+        seg_key[dst] = sv[s];
+      }
+      __syncwarp();
+      if (valid && lane == __ffs(m) - 1) mine[e] = base + __popc(m);
+      __syncwarp();
+    }
   }
 }
 
@@ -242,6 +293,8 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
   __shared__ int hist[256];
   __shared__ unsigned long long scan_ws[33];
   __shared__ int found_bin, found_above;
+  pdl_wait();
+  pdl_trigger();
   const int e = blockIdx.x;
   const int c = counts[e];
   const int m = kept[e];
@@ -312,8 +365,10 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
         const uint32_t key = K[i];
         if ((key & hmask) == prefix) digit = (int)((key >> shift) & 255u);
       }
-      const unsigned grp = __match_any_sync(kFull, digit);
-      if (digit >= 0 && lane == __ffs(grp) - 1) atomicAdd(&hist[digit], __popc(grp));
+      if (__any_sync(kFull, digit >= 0)) {  // later passes: most warps hold no candidate
+        const unsigned grp = __match_any_sync(kFull, digit);
+        if (digit >= 0 && lane == __ffs(grp) - 1) atomicAdd(&hist[digit], __popc(grp));
+      }
     }
     __syncthreads();
     if (wid == 0) {
@@ -390,10 +445,36 @@ static __device__ __align__(256) unsigned char g_select_scratch[LRMOE_NOALLOC_SC
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// The four selection kernels on `s` (workspace pieces already carved out).
+static cudaError_t enqueue_select(const SelectWs& L, const int32_t* idx, const float* score, int P,
+                                  int E, const int32_t* quota, int32_t* counts, int32_t* kept,
+                                  int32_t* offsets, int32_t* perm, int32_t* pos, int32_t* cc,
+                                  int32_t* seg_start, int32_t* seg_p, uint32_t* seg_key,
+                                  uint32_t* status, cudaStream_t s) {
+  cudaError_t e = launch_pdl(chunk_count, dim3(L.nchunks), dim3(kCountThreads), (size_t)E * 4, s,
+                             idx, P, E, L.chunk, L.nchunks, cc, pos, status);
+  if (e != cudaSuccess) return e;
+  const bool fits = (size_t)E * L.nchunks <= (size_t)kScanSmemInts;
+  const size_t scan_smem = (33 + (size_t)E + (fits ? (size_t)E * L.nchunks : 0)) * 4;
+  e = launch_pdl(chunk_scan, dim3(1), dim3(kScanThreads), scan_smem, s, cc, E, L.nchunks, quota,
+                 counts, kept, offsets, seg_start, status);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(chunk_scatter, dim3(L.nchunks), dim3(kScatterWarps * 32),
+                 (size_t)kScatterWarps * E * 4, s, idx, reinterpret_cast<const uint32_t*>(score),
+                 P, E, L.chunk, L.nchunks, static_cast<const int32_t*>(cc),
+                 static_cast<const int32_t*>(seg_start), seg_p, seg_key);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(expert_topk, dim3(E), dim3(kTopkThreads), (size_t)kTopkSmemKeys * 8, s,
+                    static_cast<const int32_t*>(counts), static_cast<const int32_t*>(kept),
+                    static_cast<const int32_t*>(offsets), static_cast<const int32_t*>(seg_start),
+                    static_cast<const int32_t*>(seg_p), static_cast<const uint32_t*>(seg_key),
+                    perm, pos);
+}
+
 SelectWs select_ws_layout(int T, int k, int E) {
   SelectWs L;
   const long long P = (long long)T * k;
-  long long chunk = 2048;
+  long long chunk = 1024;  // one 16-byte load per count thread; 4 steps per scatter warp
   const long long max_chunks = kScanSmemInts / (E > 0 ? E : 1);
   if (max_chunks > 0 && (P + chunk - 1) / chunk > max_chunks) {
     chunk = (P + max_chunks - 1) / max_chunks;
@@ -439,18 +520,8 @@ cudaError_t launch_select(const int32_t* idx, const float* score, int T, int k, 
                          kTopkSmemKeys * 8);
     attrs_set |= 1ull << dev;
   }
-  chunk_count<<<L.nchunks, kCountThreads, E * 4, s>>>(idx, P, E, L.chunk, L.nchunks, cc, pos,
-                                                      status);
-  const bool fits = (size_t)E * L.nchunks <= (size_t)kScanSmemInts;
-  const size_t scan_smem = (33 + (size_t)E + (fits ? (size_t)E * L.nchunks : 0)) * 4;
-  chunk_scan<<<1, kScanThreads, scan_smem, s>>>(cc, E, L.nchunks, quota, counts, kept, offsets,
-                                                seg_start, status);
-  chunk_scatter<<<L.nchunks, kScatterWarps * 32, kScatterWarps * E * 4, s>>>(
-      idx, reinterpret_cast<const uint32_t*>(score), P, E, L.chunk, L.nchunks, cc, seg_start,
-      seg_p, seg_key);
-  expert_topk<<<E, kTopkThreads, kTopkSmemKeys * 8, s>>>(counts, kept, offsets, seg_start, seg_p,
-                                                         seg_key, perm, pos);
-  return cudaGetLastError();
+  return enqueue_select(L, idx, score, P, E, quota, counts, kept, offsets, perm, pos, cc,
+                        seg_start, seg_p, seg_key, status, s);
 }
 
 namespace {
@@ -510,18 +581,8 @@ cudaError_t launch_select_noalloc(const int32_t* idx, const float* score, int T,
                          kTopkSmemKeys * 8);
     attrs_set |= 1ull << dev;
   }
-  chunk_count<<<L.nchunks, kCountThreads, E * 4, s>>>(idx, P, E, L.chunk, L.nchunks, cc, pos,
-                                                      status);
-  const bool fits = (size_t)E * L.nchunks <= (size_t)kScanSmemInts;
-  const size_t scan_smem = (33 + (size_t)E + (fits ? (size_t)E * L.nchunks : 0)) * 4;
-  chunk_scan<<<1, kScanThreads, scan_smem, s>>>(cc, E, L.nchunks, quota, counts, kept, offsets,
-                                                seg_start, status);
-  chunk_scatter<<<L.nchunks, kScatterWarps * 32, kScatterWarps * E * 4, s>>>(
-      idx, reinterpret_cast<const uint32_t*>(score), P, E, L.chunk, L.nchunks, cc, seg_start,
-      seg_p, seg_key);
-  expert_topk<<<E, kTopkThreads, kTopkSmemKeys * 8, s>>>(counts, kept, offsets, seg_start, seg_p,
-                                                         seg_key, perm, pos);
-  return cudaGetLastError();
+  return enqueue_select(L, idx, score, P, E, quota, counts, kept, offsets, perm, pos, cc,
+                        seg_start, seg_p, seg_key, status, s);
 }
 
 }  // namespace lrmoe

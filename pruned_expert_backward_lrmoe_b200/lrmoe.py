@@ -25,7 +25,7 @@ ST_BAD_EXPERT, ST_BAD_QUOTA, ST_NONFINITE, ST_TIMEOUT, ST_BAD_INDEX = 1, 2, 4, 8
 EXPORTS = ("lrmoe_version", "lrmoe_status_string", "lrmoe_last_error", "lrmoe_score",
            "lrmoe_select_workspace_bytes", "lrmoe_select_quota", "lrmoe_pack",
            "lrmoe_grouped_dgrad", "lrmoe_grouped_wgrad", "lrmoe_unpack", "lrmoe_pruned_backward",
-           "lrmoe_select_quota_noalloc")
+           "lrmoe_select_quota_noalloc", "lrmoe_selftest_bounded_wait")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -65,6 +65,7 @@ def load() -> ctypes.CDLL:
     lib.lrmoe_select_workspace_bytes.restype = Z
     lib.lrmoe_select_quota.argtypes = [P, P, I, I, I, P, P, P, P, P, P, P, Z, P, P]
     lib.lrmoe_select_quota_noalloc.argtypes = [P, P, I, I, I, P, P, P, P, P, P, P, P]
+    lib.lrmoe_selftest_bounded_wait.argtypes = [U32, P, P]
     lib.lrmoe_pack.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, I, I, P, P, P, P, P, I, P, P]
     lib.lrmoe_grouped_dgrad.argtypes = [P, I, P, P, I, I, I, I, I, P, P, P, P, P]
     lib.lrmoe_grouped_wgrad.argtypes = [P, P, I, P, I, I, I, I, P, I, P, P]
@@ -175,6 +176,11 @@ def lrmoe_grouped_wgrad(grad_rows, in_rows, offsets, dW, accumulate: bool = Fals
 def lrmoe_unpack(dXp, pos, T: int, k: int, dX, status=None, stream=None) -> None:
     _check(load().lrmoe_unpack(_ptr(dXp), dXp.shape[0], _ptr(pos), T, k, dXp.shape[-1], _dt(dXp),
                                _ptr(dX), _ptr(status), _stream(stream)))
+
+
+def lrmoe_selftest_bounded_wait(limit_us: int, status, stream=None) -> None:
+    """Run one device wait that must give up after `limit_us` and set ST_TIMEOUT."""
+    _check(load().lrmoe_selftest_bounded_wait(int(limit_us), _ptr(status), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------

@@ -105,3 +105,10 @@ def test_pack_unpack_reject_bad_arguments(lib):
 
 def test_pruned_backward_rejects_null_struct(lib):
     assert lib.lrmoe_pruned_backward(None, 4, 2, 3, 8, 8, 8, 1, NULL) == L.LRMOE_ERR_INVALID_ARG
+
+
+def test_selftest_rejects_bad_arguments(lib):
+    f = lib.lrmoe_selftest_bounded_wait
+    assert f(0, FAKE, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert f(2_000_000, FAKE, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert f(100, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
