@@ -48,25 +48,29 @@ constexpr int kRing = 4;
 constexpr int kSchedSlots = 64;
 __device__ unsigned int g_sched[kSchedSlots][2];
 
-template <int BN, int STAGES, bool STAGED_OUT>
+// Shared-memory layout.  OUTBUFS = fp32 staging buffers per epilogue warp (wgrad
+// only).  The tables at the end are sized by the launch's expert count E.
+template <int BN, int STAGES, int OUTBUFS>
 struct Layout {
   static constexpr int kABytes = BM * BK * 2;                 // 16 KB
   static constexpr int kBBytes = BN * BK * 2;                 // 32 KB at BN = 256
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTilesBytes = STAGES * kStageBytes;
-  // fp32 output staging: per epilogue warp two 32 x 32 fp32 sub-tiles (4 KB each)
+  // fp32 output staging: per epilogue warp OUTBUFS 32 x 32 fp32 sub-tiles (4 KB each)
   static constexpr int kOutBufBytes = 32 * 32 * 4;
   static constexpr int kOutOff = kTilesBytes;
-  static constexpr int kOutBytes = STAGED_OUT ? kEpiWarps * 2 * kOutBufBytes : 0;
-  // tile table, expert order / sizes, scan scratch, and a copy of offsets[0..E]
-  static constexpr int kTableInts = 3 * (kMaxExperts + 1) + 33;
+  static constexpr int kOutBytes = kEpiWarps * OUTBUFS * kOutBufBytes;
   static constexpr int kBarOff = kOutOff + kOutBytes;         // 8-byte barriers
   static constexpr int kNumBars = 2 * STAGES + 5 + 2 * kRing;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;     // tmem base, abort flag, tile ring
   static constexpr int kTableOff = kMiscOff + 16 + 4 * kRing;
-  static constexpr int kBytes = kTableOff + kTableInts * 4;
-  static constexpr int kAlloc = kBytes + 1024;                // slack for 1024-B alignment
+  // tile table, expert order / sizes (E + 1 each), scan scratch, offsets[0..E]
+  __host__ __device__ static constexpr int table_ints(int E) { return 3 * (E + 1) + 33; }
+  __host__ __device__ static constexpr int alloc(int E) {
+    return kTableOff + table_ints(E) * 4 + 1024;  // + slack for 1024-B alignment
+  }
 };
+constexpr int kSmemLimit = 232448;  // per-block dynamic shared memory on sm_100
 
 struct TileInfo {
   int e;       // expert
@@ -174,14 +178,14 @@ __device__ __forceinline__ void epi_swiglu(const uint32_t (&r)[32], const uint4 
   }
 }
 
-template <int MODE, int BN, int STAGES>
+template <int MODE, int BN, int STAGES, int OUTBUFS>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const __grid_constant__ CUtensorMap tmOut /* wgrad: dW [E][N1][N2] fp32 */,
     const int32_t* __restrict__ offsets, int E, int K, int N /* dgrad N or wgrad N2 */,
     int N1 /* wgrad only */, const uint16_t* __restrict__ Gp, const uint16_t* __restrict__ Up,
     void* __restrict__ out, int accumulate, uint32_t* __restrict__ status, int sched_slot) {
-  using L = Layout<BN, STAGES, MODE == kWgrad>;
+  using L = Layout<BN, STAGES, OUTBUFS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -198,8 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   volatile int* ring = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 16);  // [kRing]
   unsigned int* sched = g_sched[sched_slot];
   int* tab0 = reinterpret_cast<int*>(smem + L::kTableOff);
-  int* tab1 = tab0 + (kMaxExperts + 1);
-  int* scratch = tab1 + (kMaxExperts + 1);
+  int* tab1 = tab0 + (E + 1);
+  int* scratch = tab1 + (E + 1);
   int* offs_s = scratch + 33;  // offsets[0..E] in shared memory (read once per CTA)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -397,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
     uint32_t acc_iter = 0;
     // wgrad output staging: this warp's two 32 x 32 fp32 buffers (128-byte swizzled rows)
-    uint8_t* obuf = smem + L::kOutOff + ew * 2 * L::kOutBufBytes;
+    uint8_t* obuf = smem + L::kOutOff + ew * OUTBUFS * L::kOutBufBytes;
     uint32_t obuf_iter = 0;
     uint32_t ra[32], rb[32];
     for (int it = 0;; ++it) {
@@ -438,9 +442,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         if constexpr (MODE == kWgrad) {
           const int mrow = ti.m0 + q * 32;
           if (mrow < N1 && nb < N) {
-            uint8_t* buf = obuf + (obuf_iter & 1u) * L::kOutBufBytes;
+            uint8_t* buf = obuf + (obuf_iter % OUTBUFS) * L::kOutBufBytes;
             ++obuf_iter;
-            if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` read it
+            // the store that last used `buf` has read it
+            if (lane == 0) bulk_wait_group_read<OUTBUFS - 1>();
             __syncwarp();
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -573,32 +578,53 @@ bool make_map_out_f32(CUtensorMap* m, void* base, uint64_t E, uint64_t N1, uint6
 std::atomic<unsigned int> g_launches{0};
 
 constexpr int kBN = 256;
-// dgrad K loops are long (K = H or 2I): 4 stages; wgrad K loops are short
-// (K = m_e) and the fp32 output staging needs 32 KB: 3 stages.
-template <int MODE>
-constexpr int stages_for() { return MODE == kWgrad ? 3 : 4; }
 
+// Launch one instantiation; the dynamic shared memory depends on E.
+template <int MODE, int S, int OB>
+cudaError_t launch_variant(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
+                           const int32_t* offsets, int E, int K, int N, int N1, const void* Gp,
+                           const void* Up, void* out, int accumulate, uint32_t* status,
+                           cudaStream_t s, int grid) {
+  using L = Layout<kBN, S, OB>;
+  static_assert(L::alloc(kMaxExperts) <= kSmemLimit || OB == 1,
+                "shared memory over the sm_100 per-block limit");
+  const int smem = L::alloc(E);
+  if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
+  static unsigned long long attr_done = 0;  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tc<MODE, kBN, S, OB>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kSmemLimit);
+    if (err != cudaSuccess) return err;
+    attr_done |= 1ull << dev;
+  }
+  const int slot = (int)(g_launches.fetch_add(1u) % kSchedSlots);
+  return launch_pdl(grouped_gemm_tc<MODE, kBN, S, OB>, dim3(grid), dim3(kThreads), (size_t)smem,
+                    s, ta, tb, tout, offsets, E, K, N, N1, static_cast<const uint16_t*>(Gp),
+                    static_cast<const uint16_t*>(Up), out, accumulate, status, slot);
+}
+
+// dgrad K loops are long (K = H or 2I): 4 stages.  wgrad K loops are short
+// (K = m_e) and its fp32 output goes through shared memory: 4 stages with one
+// staging buffer per epilogue warp when that fits for this E (E <= ~130), else
+// 3 stages with two buffers.
 template <int MODE>
 cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
                         const int32_t* offsets, int E, int K, int N, int N1, const void* Gp,
                         const void* Up, void* out, int accumulate, uint32_t* status,
                         cudaStream_t s, int grid) {
-  constexpr int S = stages_for<MODE>();
-  using L = Layout<kBN, S, MODE == kWgrad>;
-  static_assert(L::kAlloc <= 232448, "shared memory over the sm_100 per-block limit");
-  static unsigned long long attr_done = 0;  // one bit per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tc<MODE, kBN, S>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-    if (err != cudaSuccess) return err;
-    attr_done |= 1ull << dev;
+  if constexpr (MODE == kWgrad) {
+    if (Layout<kBN, 4, 1>::alloc(E) <= kSmemLimit)
+      return launch_variant<MODE, 4, 1>(ta, tb, tout, offsets, E, K, N, N1, Gp, Up, out,
+                                        accumulate, status, s, grid);
+    return launch_variant<MODE, 3, 2>(ta, tb, tout, offsets, E, K, N, N1, Gp, Up, out, accumulate,
+                                      status, s, grid);
+  } else {
+    return launch_variant<MODE, 4, 0>(ta, tb, tout, offsets, E, K, N, N1, Gp, Up, out, accumulate,
+                                      status, s, grid);
   }
-  const int slot = (int)(g_launches.fetch_add(1u) % kSchedSlots);
-  return launch_pdl(grouped_gemm_tc<MODE, kBN, S>, dim3(grid), dim3(kThreads), (size_t)L::kAlloc,
-                    s, ta, tb, tout, offsets, E, K, N, N1, static_cast<const uint16_t*>(Gp),
-                    static_cast<const uint16_t*>(Up), out, accumulate, status, slot);
 }
 
 }  // namespace
