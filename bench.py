@@ -55,6 +55,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=("lrmoe", "reference"), default="lrmoe")
     p.add_argument("--no-cpu-baseline", action="store_true",
                    help="skip timing the CPU oracle (profiling runs)")
+    p.add_argument("--sweep", action="store_true",
+                   help="quota sweep (keep 1, 3/4, 1/2, 1/4) on the GLM-shaped T=16384 layer")
     p.add_argument("--override", default="",
                    help="layer fields to replace, e.g. T=4096,E=64 (smaller profiling cases)")
     return p.parse_args(argv)
@@ -331,19 +333,14 @@ def config_block(s, n_gpus):
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
-def run_gpu(args):
+def make_runner(layer, dev):
+    """Device copies of a layer, output buffers, an L2 flush and the step (eight C-ABI calls)."""
     import torch
 
-    from pruned_expert_backward_lrmoe_b200 import inputs
     from pruned_expert_backward_lrmoe_b200 import lrmoe as L
 
-    rank, world, local, dist = dist_setup(args.gpus)
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    layer = inputs.make_layer(layer_spec(args), seed=args.seed)
     s = layer.spec
     tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
-    b = 2 if s.dtype == "bf16" else 4
 
     def storage(arr):
         if s.dtype == "bf16":
@@ -395,6 +392,24 @@ def run_gpu(args):
         if ev is not None:
             ev[len(calls)].record(stream)
 
+    return host, inp, out, stream, flush_l2, step
+
+
+def run_gpu(args):
+    import torch
+
+    from pruned_expert_backward_lrmoe_b200 import inputs
+    from pruned_expert_backward_lrmoe_b200 import lrmoe as L
+
+    rank, world, local, dist = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    layer = inputs.make_layer(layer_spec(args), seed=args.seed)
+    s = layer.spec
+    tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
+    b = 2 if s.dtype == "bf16" else 4
+    host, inp, out, stream, flush_l2, step = make_runner(layer, dev)
+    st = out["status"]
     st.zero_()
     for _ in range(max(1, args.warmup)):
         step()
@@ -523,10 +538,76 @@ def run_gpu(args):
     return 0
 
 
+def run_sweep(args):
+    """Quota sweep on one GLM-shaped layer (T=16384): keep 4/4, 3/4, 2/4, 1/4 of every
+    expert's pairs.  One JSON line per keep ratio (step time, grouped-GEMM TFLOP/s and
+    their fraction of the bf16 peak), then a least-squares fit of step time against the
+    retained pairs M (time should follow M, not the routed pairs P)."""
+    import torch
+
+    from pruned_expert_backward_lrmoe_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = inputs.spec(args.config if args.config.startswith("sweep") else "sweep100")
+    layer = inputs.make_layer(base, seed=args.seed)
+    s = layer.spec
+    host, inp, out, stream, flush_l2, step = make_runner(layer, dev)
+    peaks, peak_src = load_peaks()
+    tf_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    points = []
+    for n in (4, 3, 2, 1):
+        q = inputs.quota_from_counts(layer.counts, inputs.spec("sweep100", quota=f"keep:{n}/4"))
+        inp["quota"].copy_(torch.from_numpy(q))
+        out["status"].zero_()
+        for _ in range(max(1, args.warmup)):
+            step()
+        torch.cuda.synchronize(dev)
+        if int(out["status"].item()) != 0:
+            raise SystemExit(f"device status {int(out['status'].item())} at keep {n}/4")
+        M = int(out["offsets"][-1].item())
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS) + 1)]
+               for _ in range(args.steps)]
+        with ClockSampler(0) as clk:
+            for i in range(args.steps):
+                flush_l2()
+                step(evs[i])
+            torch.cuda.synchronize(dev)
+        kern = {kn: statistics.fmean(ev[j].elapsed_time(ev[j + 1]) for ev in evs)
+                for j, kn in enumerate(KERNELS)}
+        step_ms = statistics.fmean(ev[0].elapsed_time(ev[-1]) for ev in evs)
+        by, fl = algorithmic(s.T, s.k, s.E, s.H, s.I, M, 2)
+        gemm_ms = sum(kern[kn] for kn in fl)
+        tf = sum(fl.values()) / (gemm_ms * 1e-3) / 1e12
+        gemm_bytes = sum(by[kn] for kn in fl)
+        points.append((M, step_ms))
+        print(json.dumps({
+            "sweep_keep": f"{n}/4", "retained_pairs": M, "routed_pairs": s.P,
+            "ms_per_step": step_ms, "value": M / (step_ms * 1e-3), "unit": UNIT,
+            "gemm_ms": gemm_ms, "gemm_tflops": tf, "gemm_tensor_frac": tf / tf_peak,
+            "gemm_hbm_frac": gemm_bytes / (gemm_ms * 1e-3) / 1e9 / hbm_peak,
+            "gemm_flop_per_byte": sum(fl.values()) / gemm_bytes,
+            "peaks": f"{peak_src}: bf16 {tf_peak} TFLOP/s sustained, HBM {hbm_peak} GB/s",
+            "kernels_ms": kern, "clocks": clk.summary(), "steps": args.steps,
+            "config": config_block(s, 1)}), flush=True)
+    xs = np.array([p[0] for p in points], np.float64)
+    ys = np.array([p[1] for p in points], np.float64)
+    slope, intercept = np.polyfit(xs, ys, 1)
+    resid = ys - (slope * xs + intercept)
+    print(json.dumps({"sweep_fit": "ms_per_step = slope * M + intercept",
+                      "slope_us_per_1k_pairs": slope * 1e6, "intercept_ms": intercept,
+                      "max_abs_residual_ms": float(np.abs(resid).max()),
+                      "routed_pairs": s.P}), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_gpu(args)
 
 
