@@ -159,6 +159,34 @@ def lrm_score_f64(topk_idx, topk_w, dY64, a64):
 
 
 # ----------------------------------------------------------------------------
+# quota controller (before the backward)
+# ----------------------------------------------------------------------------
+def quota_controller(topk_idx, E: int, cap: int, max_pairs: int):
+    """Per-expert quotas from routed counts, a per-expert cap and a pair budget.
+
+    [RU-B] bullet 2: before the backward a controller sees how many tokens came to
+    each expert and, within memory limits, fixes how many pairs of each expert stay
+    for the whole layer call.  Reading (water-filling): q_e = min(c_e, cap, tau) with
+    tau the largest integer level for which sum_e q_e <= max_pairs, so the most
+    loaded experts are cut first.  cap <= 0: no per-expert cap; max_pairs < 0: no
+    budget.  Returns (quota[E] int32, counts[E] int32).
+    """
+    idx = np.asarray(topk_idx).reshape(-1)
+    counts = np.zeros(E, dtype=np.int64)
+    for e in idx:
+        if 0 <= e < E:
+            counts[e] += 1
+    capped = counts.copy() if cap <= 0 else np.minimum(counts, cap)
+    if max_pairs < 0 or capped.sum() <= max_pairs:
+        return capped.astype(np.int32), counts.astype(np.int32)
+    tau = 0
+    for level in range(int(capped.max()) + 1):     # largest level within the budget
+        if np.minimum(capped, level).sum() <= max_pairs:
+            tau = level
+    return np.minimum(capped, tau).astype(np.int32), counts.astype(np.int32)
+
+
+# ----------------------------------------------------------------------------
 # a2: per-expert top-quota selection
 # ----------------------------------------------------------------------------
 def select_quota(topk_idx, score, quota, E: int):

@@ -404,3 +404,49 @@ def test_row_sampled_backward_matches_whole_expert_backward():
                                         L.W_down, s.dtype)
     got = O.unpack_tokens(tokens, dxp_all, r["pos"], s.k, s.H)
     np.testing.assert_allclose(got, r["dX"][tokens], rtol=1e-12, atol=1e-300)
+
+
+# ----------------------------------------------------------------------------
+# quota controller
+# ----------------------------------------------------------------------------
+def test_quota_controller_reduces_to_the_capacity_rule():
+    """No budget and cap = T*k/E gives the configs' capacity quotas (written independently)."""
+    for name, over in (("qwen", dict(T=512, E=16, H=64, I=64)), ("glm", dict(T=384, E=8, H=64, I=64))):
+        L = small_layer(name, **over)
+        s = L.spec
+        q, c = O.quota_controller(L.topk_idx, s.E, (s.T * s.k) // s.E, -1)
+        np.testing.assert_array_equal(c, L.counts)
+        np.testing.assert_array_equal(q, inputs.quota_from_counts(L.counts, s))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_quota_controller_budget_properties(seed):
+    """Within budget, never above count or cap, and maximal: one more level would not fit."""
+    rng = np.random.default_rng(seed)
+    E = int(rng.integers(1, 20))
+    idx = rng.integers(-1, E + 2, size=(int(rng.integers(1, 300)), 3)).astype(np.int32)
+    c = np.bincount(idx[(idx >= 0) & (idx < E)], minlength=E)
+    cap = int(rng.integers(-1, 60))
+    budget = int(rng.integers(-1, int(c.sum()) + 5))
+    q, counts = O.quota_controller(idx, E, cap, budget)
+    np.testing.assert_array_equal(counts, c)
+    capped = c if cap <= 0 else np.minimum(c, cap)
+    assert (q <= capped).all() and (q >= 0).all()
+    if budget < 0 or capped.sum() <= budget:
+        np.testing.assert_array_equal(q, capped)
+        return
+    assert q.sum() <= budget
+    tau = q.max()
+    assert (q == np.minimum(capped, tau)).all()
+    assert np.minimum(capped, tau + 1).sum() > budget      # the next level would not fit
+
+
+def test_quota_controller_worked_example():
+    """counts (9, 5, 2, 0), budget 10 -> level 4 -> quotas (4, 4, 2, 0); with cap 3 -> (3, 3, 2, 0)."""
+    idx = np.array([0] * 9 + [1] * 5 + [2] * 2, np.int32).reshape(-1, 1)
+    q, c = O.quota_controller(idx, 4, 0, 10)
+    assert c.tolist() == [9, 5, 2, 0] and q.tolist() == [4, 4, 2, 0]
+    q, _ = O.quota_controller(idx, 4, 3, 10)
+    assert q.tolist() == [3, 3, 2, 0]
+    q, _ = O.quota_controller(idx, 4, 0, 0)
+    assert q.tolist() == [0, 0, 0, 0]
