@@ -478,6 +478,22 @@ def run_gpu(args):
                                                     FALLBACK_PEAKS["bf16_tflops_sustained"]))
         breakdown[kname] = e
 
+    # ---------------- quota controller (runs before the backward; not in the step) ----------------
+    q_dev = torch.empty(s.E, dtype=torch.int32, device=dev)
+    c_dev = torch.empty(s.E, dtype=torch.int32, device=dev)
+    cap = (s.T * s.k) // s.E
+    ctl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(20)]
+    for i in range(23):
+        if i >= 3:
+            ctl_ev[i - 3][0].record(stream)
+        L.lrmoe_quota_controller(inp["topk_idx"], s.E, cap, -1, q_dev, c_dev, st, stream)
+        if i >= 3:
+            ctl_ev[i - 3][1].record(stream)
+    torch.cuda.synchronize(dev)
+    controller_us = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in ctl_ev)
+    controller_matches = bool(torch.equal(q_dev, inp["quota"])) if s.quota == "capacity" else None
+
     # ---------------- end to end through host buffers ----------------
     pin = {k_: v.pin_memory() for k_, v in host.items()}
     dX_host = torch.empty(s.T, s.H, dtype=tdt).pin_memory()
@@ -525,6 +541,8 @@ def run_gpu(args):
         "gemm_ms": gemm_ms,
         "roofline": roofline,
         "breakdown": breakdown,
+        "quota_controller_us": controller_us,
+        "quota_controller_equals_capacity_rule": controller_matches,
         "breakdown_steps": n_bd,
         "breakdown_step_ms": sum(kern_ms.values()),
         "cpu_baseline": cpu,

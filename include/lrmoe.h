@@ -134,6 +134,26 @@ int lrmoe_select_quota(const int32_t* topk_idx, const float* score, int T, int k
                        uint32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Quota controller.  RU-B bullet 2, FR-B bullet 2, DE paragraph 3: before the
+ * backward a controller sees how many tokens came to each expert and, within
+ * the memory limit, fixes how many pairs of each expert stay for the layer
+ * call.  Reading implemented (water-filling):
+ *
+ *   c_e = #{p : topk_idx[p] == e},  q_e = min(c_e, cap, tau),
+ *   tau = the largest integer level with sum_e q_e <= max_pairs,
+ *
+ * so the most loaded experts are cut first.  cap <= 0 disables the per-expert
+ * cap; max_pairs < 0 disables the budget (then q_e = min(c_e, cap); with
+ * cap = T*k/E this is the "capacity" quota of the configs).  Outputs quota[E]
+ * and counts[E] (int32, device); nothing goes back to the host, so the result
+ * can feed lrmoe_select_quota on the same stream.  ids >= E are skipped and set
+ * LRMOE_ST_BAD_EXPERT.  E <= 4096.
+ * ------------------------------------------------------------------------- */
+int lrmoe_quota_controller(const int32_t* topk_idx, int T, int k, int E, int32_t cap,
+                           int64_t max_pairs, int32_t* quota, int32_t* counts, uint32_t* status,
+                           void* stream);
+
+/* ---------------------------------------------------------------------------
  * Selection that allocates nothing.  The LRMoE pages have no counterpart of
  * this entry point; it exists for callers of this library that cannot hand
  * it device scratch: a host framework or plugin host that owns every byte of

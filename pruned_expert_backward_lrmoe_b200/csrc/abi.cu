@@ -134,6 +134,20 @@ int lrmoe_select_quota(const int32_t* topk_idx, const float* score, int T, int k
   return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_select_quota launch");
 }
 
+int lrmoe_quota_controller(const int32_t* topk_idx, int T, int k, int E, int32_t cap,
+                           int64_t max_pairs, int32_t* quota, int32_t* counts, uint32_t* status,
+                           void* stream) {
+  g_last_error[0] = 0;
+  if (int r = check_pairs(T, k, E)) return r;
+  if (E > 4096) return fail(LRMOE_ERR_UNSUPPORTED, "E=%d > 4096", E);
+  REQUIRE_PTR(topk_idx);
+  REQUIRE_PTR(quota);
+  REQUIRE_PTR(counts);
+  cudaError_t e = launch_quota(topk_idx, T * k, E, cap, (long long)max_pairs, quota, counts,
+                               status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_quota_controller launch");
+}
+
 // Selection for callers that cannot provide device scratch: the kernels use a
 // fixed array inside the library instead (see select.cu).  Nothing here or
 // below allocates.

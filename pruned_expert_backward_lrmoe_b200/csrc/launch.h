@@ -75,6 +75,10 @@ cudaError_t launch_wgrad_simt(const void* grad_rows, const void* in_rows, int ro
                               const int32_t* offsets, int E, int N1, int N2, lrmoe_dtype dt,
                               float* dW, int accumulate, uint32_t* status, cudaStream_t s);
 
+// quota controller: water-filling of per-expert quotas under a cap and a pair budget
+cudaError_t launch_quota(const int32_t* idx, int P, int E, int cap, long long budget,
+                         int32_t* quota, int32_t* counts, uint32_t* status, cudaStream_t s);
+
 // diagnostic: a bounded wait that must time out
 cudaError_t launch_selftest_wait(uint32_t limit_us, uint32_t* status, cudaStream_t s);
 

@@ -25,7 +25,7 @@ ST_BAD_EXPERT, ST_BAD_QUOTA, ST_NONFINITE, ST_TIMEOUT, ST_BAD_INDEX = 1, 2, 4, 8
 EXPORTS = ("lrmoe_version", "lrmoe_status_string", "lrmoe_last_error", "lrmoe_score",
            "lrmoe_select_workspace_bytes", "lrmoe_select_quota", "lrmoe_pack",
            "lrmoe_grouped_dgrad", "lrmoe_grouped_wgrad", "lrmoe_unpack", "lrmoe_pruned_backward",
-           "lrmoe_select_quota_noalloc", "lrmoe_selftest_bounded_wait")
+           "lrmoe_select_quota_noalloc", "lrmoe_selftest_bounded_wait", "lrmoe_quota_controller")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -66,6 +66,7 @@ def load() -> ctypes.CDLL:
     lib.lrmoe_select_quota.argtypes = [P, P, I, I, I, P, P, P, P, P, P, P, Z, P, P]
     lib.lrmoe_select_quota_noalloc.argtypes = [P, P, I, I, I, P, P, P, P, P, P, P, P]
     lib.lrmoe_selftest_bounded_wait.argtypes = [U32, P, P]
+    lib.lrmoe_quota_controller.argtypes = [P, I, I, I, ctypes.c_int32, ctypes.c_int64, P, P, P, P]
     lib.lrmoe_pack.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, I, I, P, P, P, P, P, I, P, P]
     lib.lrmoe_grouped_dgrad.argtypes = [P, I, P, P, I, I, I, I, I, P, P, P, P, P]
     lib.lrmoe_grouped_wgrad.argtypes = [P, P, I, P, I, I, I, I, P, I, P, P]
@@ -131,6 +132,15 @@ def lrmoe_select_quota(topk_idx, score, quota, counts, kept, offsets, perm, pos,
                                      _ptr(counts), _ptr(kept), _ptr(offsets), _ptr(perm),
                                      _ptr(pos), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                      _ptr(status), _stream(stream)))
+
+
+def lrmoe_quota_controller(topk_idx, E: int, cap: int, max_pairs: int, quota, counts, status=None,
+                           stream=None) -> None:
+    """Per-expert quotas on the device: min(count, cap, tau) with tau the largest level
+    whose total fits max_pairs (cap <= 0 / max_pairs < 0 disable the limits)."""
+    T, k = topk_idx.shape
+    _check(load().lrmoe_quota_controller(_ptr(topk_idx), T, k, E, int(cap), int(max_pairs),
+                                         _ptr(quota), _ptr(counts), _ptr(status), _stream(stream)))
 
 
 def lrmoe_select_quota_noalloc(topk_idx, score, quota, counts, kept, offsets, perm, pos,

@@ -112,3 +112,10 @@ def test_selftest_rejects_bad_arguments(lib):
     assert f(0, FAKE, NULL) == L.LRMOE_ERR_INVALID_ARG
     assert f(2_000_000, FAKE, NULL) == L.LRMOE_ERR_INVALID_ARG
     assert f(100, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+
+
+def test_quota_controller_rejects_bad_arguments(lib):
+    f = lib.lrmoe_quota_controller
+    assert f(NULL, 4, 2, 3, 0, -1, FAKE, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert f(FAKE, 4, 2, 5000, 0, -1, FAKE, FAKE, NULL, NULL) == L.LRMOE_ERR_UNSUPPORTED
+    assert f(FAKE, 0, 2, 3, 0, -1, FAKE, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
