@@ -35,6 +35,11 @@ dense_backward   the ordinary unpruned SwiGLU MoE expert backward (textbook
                  calculus); used only to pin the pruned functions.
 forward          the ordinary SwiGLU MoE forward in fp64, used only by the
                  finite-difference pin ([RU-B] bullet 1: the forward stays full).
+lrm_score_from_norms  the score with ||a_p||^2 given (saved by the forward);
+                 the same three factors, multiplied in the same order.
+router_grad      the gradient of the routing weights, dL/dw_p = <dY_t, y_p>
+                 with y_p = W_down[e] a_p the pair's expert output (the layer
+                 output is sum_j w_tj y_tj); the pages do not treat it (R8).
 
 Readings where the pages are silent:
   R1  "saved projection input" = a = silu(g)*u, the input of the down
@@ -48,6 +53,10 @@ Readings where the pages are silent:
   R6  the packed gradient row is RNE_storage(fp32(w) * fp32(dY_t)); all
       gradient arithmetic afterwards is fp64 here.
   R7  topk_idx < 0 = not routed; idx >= E = invalid (skipped, status bit).
+  R8  the routing-weight gradient is not part of the pruned path; when asked
+      for, it is <dY_t, y_p> with y_p saved by the forward, for every routed
+      pair, or for the retained pairs only when pos is given (dropped pairs
+      then get 0), in the canonical order below with x*x replaced by dY*y.
 
 Canonical score order (R3), for one row v of D = V * VEC elements
 (VEC = 8 for bf16 storage, 4 for fp32):
@@ -120,12 +129,40 @@ def row_sq_norm(rows32: np.ndarray, vec: int) -> np.ndarray:
     return acc[:, 0].copy()
 
 
+def row_dot(rows_a32: np.ndarray, rows_b32: np.ndarray, vec: int) -> np.ndarray:
+    """Row-wise dot products in the canonical order: 32 lane partials over
+    vectors, fl(acc + fl(x*y)) element by element, then the butterfly."""
+    A = np.ascontiguousarray(rows_a32, dtype=np.float32)
+    B = np.ascontiguousarray(rows_b32, dtype=np.float32)
+    n, D = A.shape
+    assert B.shape == (n, D) and D % vec == 0
+    V = D // vec
+    va, vb = A.reshape(n, V, vec), B.reshape(n, V, vec)
+    acc = np.zeros((n, 32), dtype=np.float32)
+    with np.errstate(invalid="ignore", over="ignore"):
+        for r in range(0, V, 32):
+            nl = min(32, V - r)
+            for j in range(vec):
+                acc[:, :nl] = acc[:, :nl] + va[:, r:r + nl, j] * vb[:, r:r + nl, j]
+        lane = np.arange(32)
+        for o in (16, 8, 4, 2, 1):
+            acc = acc + acc[:, lane ^ o]
+    return acc[:, 0].copy()
+
+
 def lrm_score(topk_idx, topk_w, dY, a, dtype: str, E: int):
     """score[p] = w_p^2 * ||dY_t||^2 * ||a_p||^2 for every routed pair p = t*k + j.
 
     Non-routed (idx < 0) and invalid (idx >= E) slots get +0 and are never
     selected; invalid ones set ST_BAD_EXPERT.  NaN scores set ST_NONFINITE.
     """
+    n_a = row_sq_norm(decode(a, dtype), VEC[dtype])            # [P]
+    return lrm_score_from_norms(topk_idx, topk_w, dY, n_a, dtype, E)
+
+
+def lrm_score_from_norms(topk_idx, topk_w, dY, a_sqnorm, dtype: str, E: int):
+    """The same score with ||a_p||^2 given (saved by the forward): the three
+    factors of the factorisation, multiplied in the canonical order."""
     T, k = topk_idx.shape
     idx = topk_idx.reshape(-1)
     w = topk_w.reshape(-1).astype(np.float32)
@@ -133,11 +170,11 @@ def lrm_score(topk_idx, topk_w, dY, a, dtype: str, E: int):
     if np.any(idx >= E):
         status |= ST_BAD_EXPERT
     routed = (idx >= 0) & (idx < E)
-    vec = VEC[dtype]
-    n_dy = row_sq_norm(decode(dY, dtype), vec)                 # [T]
-    n_a = row_sq_norm(decode(a, dtype), vec)                   # [P]
+    n_dy = row_sq_norm(decode(dY, dtype), VEC[dtype])          # [T]
+    n_a = np.asarray(a_sqnorm, dtype=np.float32).reshape(-1)
     n_dy_p = np.repeat(n_dy, k)
-    s = ((w * w) * n_dy_p) * n_a
+    with np.errstate(invalid="ignore", over="ignore"):
+        s = ((w * w) * n_dy_p) * n_a
     s = np.where(routed, s, np.float32(0.0)).astype(np.float32)
     bits = s.view(np.uint32).copy()
     nan = np.isnan(s)
@@ -161,6 +198,21 @@ def lrm_score_f64(topk_idx, topk_w, dY64, a64):
 # ----------------------------------------------------------------------------
 # quota controller (before the backward)
 # ----------------------------------------------------------------------------
+def router_grad(topk_idx, dY, y, dtype: str, E: int, pos=None):
+    """dw[p] = <dY_t, y_p> for routed pairs (R8); +0 for empty and invalid slots
+    and, when pos is given, for pairs with pos[p] < 0.  Invalid ids set
+    ST_BAD_EXPERT.  y [T*k, H] is the pair's saved expert output."""
+    T, k = topk_idx.shape
+    idx = topk_idx.reshape(-1)
+    status = ST_BAD_EXPERT if np.any(idx >= E) else 0
+    keep = (idx >= 0) & (idx < E)
+    if pos is not None:
+        keep &= np.asarray(pos).reshape(-1) >= 0
+    dy_p = np.repeat(decode(dY, dtype), k, axis=0)
+    d = row_dot(dy_p, decode(y, dtype), VEC[dtype])
+    return np.where(keep, d, np.float32(0.0)).astype(np.float32), status
+
+
 def quota_controller(topk_idx, E: int, cap: int, max_pairs: int):
     """Per-expert quotas from routed counts, a per-expert cap and a pair budget.
 

@@ -187,6 +187,25 @@ def _saved_forward(x32, Wgu32, idx, s: LayerSpec, dtype: str):
     return g_s, u_s, a_s
 
 
+def saved_expert_outputs(layer: "Layer") -> np.ndarray:
+    """y_p = W_down[e] a_p for every routed pair (the forward's expert output, which
+    it combines as sum_j w_tj y_tj), fp32 accumulation, rounded to storage; zero
+    rows for empty and invalid slots.  Computed on demand: [T*k, H] is large."""
+    import torch
+    s = layer.spec
+    k, H = s.k, s.H
+    y = np.zeros((s.P, H), dtype=np.float32)
+    flat = layer.topk_idx.reshape(-1)
+    a32 = torch.from_numpy(to_float32(layer.a, s.dtype))
+    for e in range(s.E):
+        pairs = np.nonzero(flat == e)[0]
+        if pairs.size == 0:
+            continue
+        Wd = torch.from_numpy(to_float32(layer.W_down[e], s.dtype))   # [H, I]
+        y[pairs] = (a32[torch.from_numpy(pairs)] @ Wd.T).numpy()
+    return _round_storage(y, s.dtype)
+
+
 def make_layer(s: LayerSpec | str, seed: int = 0, topk_idx: Optional[np.ndarray] = None,
                quota: Optional[np.ndarray] = None) -> Layer:
     """Draw one synthetic layer.  `topk_idx` / `quota` override routing / quotas (edge cases)."""

@@ -124,6 +124,34 @@ def test_row_norm_every_element_counted(dtype, D):
     np.testing.assert_array_equal(n.astype(np.float64), x * x)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_row_norm_lane_partials_then_butterfly(dtype):
+    """Hand-worked order check.  Row: 4096 in vector 0 (lane 0) and 1 in vectors 1 and
+    3 (lanes 1 and 3).  Lanes 1 and 3 meet at the o=2 step (1 + 1 = 2), which then
+    joins 2^24 at o=1: 2^24 + 2 is exact.  A plain left-to-right sum would lose both
+    ones (2^24 + 1 rounds to even), giving 2^24."""
+    vec = O.VEC[dtype]
+    x = np.zeros((1, 32 * vec), np.float32)
+    x[0, 0], x[0, vec], x[0, 3 * vec] = 4096.0, 1.0, 1.0
+    n = O.row_sq_norm(O.decode(O.encode_rne(x, dtype), dtype), vec)
+    assert float(n[0]) == 16777218.0
+    seq = np.float32(0.0)
+    for v in (4096.0, 1.0, 1.0):                 # the order this pin rules out
+        seq = np.float32(seq + np.float32(v * v))
+    assert float(seq) == 16777216.0
+
+
+def test_score_from_saved_norms_equals_score():
+    """Splitting the factorisation at ||a_p||^2 changes no bit."""
+    layer = small_layer("qwen", seed=3, T=64, E=8, H=64, I=96)
+    s = layer.spec
+    n_a = O.row_sq_norm(O.decode(layer.a, s.dtype), O.VEC[s.dtype])
+    s1, st1 = O.lrm_score(layer.topk_idx, layer.topk_w, layer.dY, layer.a, s.dtype, s.E)
+    s2, st2 = O.lrm_score_from_norms(layer.topk_idx, layer.topk_w, layer.dY, n_a, s.dtype, s.E)
+    np.testing.assert_array_equal(s1.view(np.uint32), s2.view(np.uint32))
+    assert st1 == st2
+
+
 def test_score_nonrouted_invalid_and_nonfinite():
     T, k, E, H, I = 4, 2, 3, 8, 8
     idx = np.array([[0, -1], [5, 1], [2, 2], [1, 0]], np.int32)
@@ -450,3 +478,68 @@ def test_quota_controller_worked_example():
     assert q.tolist() == [3, 3, 2, 0]
     q, _ = O.quota_controller(idx, 4, 0, 0)
     assert q.tolist() == [0, 0, 0, 0]
+
+
+# ----------------------------------------------------------------------------
+# routing-weight gradient (reading R8)
+# ----------------------------------------------------------------------------
+def test_router_grad_equals_finite_differences_of_the_forward():
+    """L(w) = sum_t <dY_t, Y_t(w)> with the fp64 forward; central differences in
+    each routing weight give dL/dw_p, which must equal <dY_t, y_p>."""
+    layer = small_layer("tiny", seed=4, T=6, E=3, H=16, I=8)
+    s = layer.spec
+    x = O.decode(layer.x, s.dtype).astype(np.float64)
+    Wgu = O.decode(layer.W_gu, s.dtype).astype(np.float64)
+    Wd = O.decode(layer.W_down, s.dtype).astype(np.float64)
+    dY = O.decode(layer.dY, s.dtype).astype(np.float64)
+    w = layer.topk_w.astype(np.float64)
+    _, _, _, a = O.forward(layer.topk_idx, w, x, Wgu, Wd)
+    y = np.zeros((s.P, s.H))
+    for p in range(s.P):
+        y[p] = Wd[layer.topk_idx.reshape(-1)[p]] @ a[p]
+    dw, st = O.router_grad(layer.topk_idx, layer.dY, y.astype(np.float32), s.dtype, s.E)
+    assert st == 0
+    h = 1e-4
+    for p in range(s.P):
+        wp, wm = w.copy(), w.copy()
+        wp.reshape(-1)[p] += h
+        wm.reshape(-1)[p] -= h
+        Lp = float((dY * O.forward(layer.topk_idx, wp, x, Wgu, Wd)[0]).sum())
+        Lm = float((dY * O.forward(layer.topk_idx, wm, x, Wgu, Wd)[0]).sum())
+        fd = (Lp - Lm) / (2 * h)
+        assert abs(float(dw[p]) - fd) <= 1e-5 * max(1e-3, abs(fd)), (p, dw[p], fd)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_router_grad_dyadic_exact_and_masks(dtype):
+    """Small multiples of 1/8 make every step exact: the canonical dot equals the
+    fp64 dot bit for bit.  Empty, invalid and (with pos) dropped slots give +0."""
+    rng = np.random.default_rng(7)
+    T, k, E, H = 5, 3, 4, 64
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    idx[0, 1] = -1
+    idx[2, 2] = E + 1
+    dY = (rng.integers(-8, 9, size=(T, H)) / 8).astype(np.float32)
+    y = (rng.integers(-8, 9, size=(T * k, H)) / 8).astype(np.float32)
+    dw, st = O.router_grad(idx, O.encode_rne(dY, dtype), O.encode_rne(y, dtype), dtype, E)
+    exact = (np.repeat(dY.astype(np.float64), k, axis=0) * y.astype(np.float64)).sum(axis=1)
+    flat = idx.reshape(-1)
+    for p in range(T * k):
+        want = exact[p] if 0 <= flat[p] < E else 0.0
+        assert float(dw[p]) == want and not (want == 0 and np.signbit(dw[p]))
+    assert st == O.ST_BAD_EXPERT
+    pos = np.arange(T * k, dtype=np.int32)
+    pos[[3, 4, 9]] = -1
+    dw2, _ = O.router_grad(idx, O.encode_rne(dY, dtype), O.encode_rne(y, dtype), dtype, E, pos=pos)
+    assert float(dw2[3]) == 0.0 and float(dw2[4]) == 0.0 and float(dw2[9]) == 0.0
+    keep = (pos >= 0)
+    np.testing.assert_array_equal(dw2[keep].view(np.uint32), dw[keep].view(np.uint32))
+
+
+def test_row_dot_of_a_row_with_itself_is_its_norm():
+    """Two separately written loops agree bit for bit on x.x = ||x||^2 (so the
+    hand-worked order pin of the norm also holds for the dot)."""
+    x = np.random.default_rng(8).standard_normal((9, 8 * 40)).astype(np.float32)
+    for vec in (4, 8):
+        np.testing.assert_array_equal(O.row_dot(x, x, vec).view(np.uint32),
+                                      O.row_sq_norm(x, vec).view(np.uint32))
