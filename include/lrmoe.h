@@ -109,6 +109,51 @@ int lrmoe_score(const int32_t* topk_idx, const float* topk_w, int T, int k, int 
                 float* score, uint32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * a1 split at the factorisation (same passage as lrmoe_score): ||a_p||^2 does
+ * not depend on the backward, so the forward, which writes a, can save it, and
+ * the backward's score then reads dY and the saved norms instead of all of a
+ * (T*H + 4*T*k bytes instead of T*H + T*k*I elements).  The pages describe no
+ * such split; it changes no value: the two calls below give, bit for bit,
+ * what lrmoe_score gives (which is itself these two kernels back to back).
+ *
+ * lrmoe_row_sqnorm: out[r] = ||rows[r]||^2 for r < n_rows, rows [n_rows][D] in
+ *   dtype dt, out [n_rows] fp32, in the canonical order of lrmoe_score.
+ *   No status word: a non-finite row gives a non-finite norm (a NaN of
+ *   unspecified payload for NaN input), which the score call then flags.
+ * lrmoe_score_from_norms: score[p] = fl(fl(fl(w_p*w_p) * ||dY_t||^2) *
+ *   a_sqnorm[p]) for routed slots, +0 otherwise; status bits, NaN handling and
+ *   layouts as lrmoe_score.  a_sqnorm [T*k] fp32 may be the score buffer
+ *   itself (each slot is read before it is overwritten).
+ * ------------------------------------------------------------------------- */
+int lrmoe_row_sqnorm(const void* rows, int n_rows, int D, lrmoe_dtype dt, float* out,
+                     void* stream);
+
+int lrmoe_score_from_norms(const int32_t* topk_idx, const float* topk_w, int T, int k, int E,
+                           const void* dY, int H, const float* a_sqnorm, lrmoe_dtype dt,
+                           float* score, uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Routing-weight gradient.  The pages (RU-B, FR-B, DE) prune the expert
+ * weight-gradient contributions and do not treat the router; this call gives
+ * what the layer output sum_j w_tj y_tj implies:
+ *
+ *   dw[p] = <dY_t, y_p>            (p = t*k + j, e = topk_idx[p] in [0,E))
+ *
+ * y_saved [T*k][H] in dtype dt is the pair's expert output y_p = W_down[e] a_p,
+ * saved by the forward (rows of empty or invalid slots are not read).  With
+ * pos == NULL every routed pair is computed; with pos (the [T*k] int32 output
+ * of lrmoe_select_quota) only retained pairs (pos[p] >= 0) are, and dropped
+ * pairs get +0 -- the pages are silent on which reading LRMoE uses.  Empty and
+ * invalid slots get +0; invalid ids set LRMOE_ST_BAD_EXPERT.
+ * Arithmetic: the canonical order of lrmoe_score with x*x replaced by dY*y:
+ * 32 lane partials, fl(acc + fl(dY*y)) element by element, butterfly.
+ * Output dw [T*k] fp32.
+ * ------------------------------------------------------------------------- */
+int lrmoe_router_grad(const int32_t* topk_idx, int T, int k, int E, const void* dY, int H,
+                      const void* y_saved, lrmoe_dtype dt, const int32_t* pos, float* dw,
+                      uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * a2  Per-expert top-quota selection.  RU-B bullets 2-3, FR-B bullets 2-3,
  * DE paragraph 3: a quota per expert is fixed for the layer call before the
  * backward, and within it the pairs with the highest score stay.

@@ -104,6 +104,52 @@ int lrmoe_score(const int32_t* topk_idx, const float* topk_w, int T, int k, int 
   return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_score launch");
 }
 
+int lrmoe_row_sqnorm(const void* rows, int n_rows, int D, lrmoe_dtype dt, float* out,
+                     void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  REQUIRE(n_rows > 0, "n_rows=%d must be positive", n_rows);
+  if (int r = check_feature(D, dt, "D")) return r;
+  REQUIRE_PTR(rows);
+  REQUIRE_PTR(out);
+  cudaError_t e = launch_row_sqnorm(rows, n_rows, D, dt, out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_row_sqnorm launch");
+}
+
+int lrmoe_score_from_norms(const int32_t* topk_idx, const float* topk_w, int T, int k, int E,
+                           const void* dY, int H, const float* a_sqnorm, lrmoe_dtype dt,
+                           float* score, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  if (int r = check_pairs(T, k, E)) return r;
+  if (int r = check_feature(H, dt, "H")) return r;
+  REQUIRE_PTR(topk_idx);
+  REQUIRE_PTR(topk_w);
+  REQUIRE_PTR(dY);
+  REQUIRE_PTR(a_sqnorm);
+  REQUIRE_PTR(score);
+  cudaError_t e = launch_score_from_norms(topk_idx, topk_w, T, k, E, dY, H, a_sqnorm, dt, score,
+                                          status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_score_from_norms launch");
+}
+
+int lrmoe_router_grad(const int32_t* topk_idx, int T, int k, int E, const void* dY, int H,
+                      const void* y_saved, lrmoe_dtype dt, const int32_t* pos, float* dw,
+                      uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  if (int r = check_pairs(T, k, E)) return r;
+  if (int r = check_feature(H, dt, "H")) return r;
+  REQUIRE_PTR(topk_idx);
+  REQUIRE_PTR(dY);
+  REQUIRE_PTR(y_saved);
+  REQUIRE_PTR(dw);
+  REQUIRE(pos == nullptr || aligned16(pos), "pos is not 16-byte aligned");
+  cudaError_t e = launch_router_grad(topk_idx, T, k, E, dY, H, y_saved, dt, pos, dw, status,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_router_grad launch");
+}
+
 size_t lrmoe_select_workspace_bytes(int T, int k, int E) {
   if (T <= 0 || k <= 0 || E <= 0) return 0;
   return select_ws_layout(T, k, E).total;

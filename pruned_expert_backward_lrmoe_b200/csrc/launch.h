@@ -37,6 +37,14 @@ int num_sms();
 cudaError_t launch_score(const int32_t* idx, const float* w, int T, int k, int E, const void* dY,
                          int H, const void* a, int D, lrmoe_dtype dt, float* score,
                          uint32_t* status, cudaStream_t s);
+cudaError_t launch_router_grad(const int32_t* idx, int T, int k, int E, const void* dY, int H,
+                               const void* y, lrmoe_dtype dt, const int32_t* pos, float* dw,
+                               uint32_t* status, cudaStream_t s);
+cudaError_t launch_row_sqnorm(const void* rows, int n, int D, lrmoe_dtype dt, float* out,
+                              cudaStream_t s);
+cudaError_t launch_score_from_norms(const int32_t* idx, const float* w, int T, int k, int E,
+                                    const void* dY, int H, const float* a_sqnorm, lrmoe_dtype dt,
+                                    float* score, uint32_t* status, cudaStream_t s);
 
 struct SelectWs {
   int chunk;        // pairs per chunk

@@ -4,145 +4,143 @@
 // bullet 3: the squared norm of a pair's outer-product contribution factorises,
 // so each pair needs two row norms and three multiplies, never the H x I matrix.
 //
-// One warp per token: it reads dY_t once and the k saved rows a_p, 16 bytes
-// per lane per load (HBM-bound: T*H + T*k*I elements + 8 bytes per pair).
-// The reduction order is fixed so that the result is bit-reproducible:
+// Two HBM-bound kernels:
+//   row_sqnorm        ||row||^2 of every row of a matrix (the saved a, T*k rows);
+//   score_from_norms  ||dY_t||^2 per token, then w^2 * ||dY_t||^2 * ||a_p||^2 per slot.
+// lrmoe_score runs both, parking ||a_p||^2 in the score buffer, which the second
+// kernel then overwrites slot by slot.  When the forward has saved ||a_p||^2
+// (it owns a when a is produced), only the second kernel runs and a is not read.
+//
+// A warp reduces RPW rows at once with every 16-byte load of a row chunk in
+// flight together.  The order is fixed so that results are bit-reproducible:
 // lane l sums vectors l, l+32, ... element by element as fl(acc + fl(x*x)),
 // then a butterfly fl(acc[l] + acc[l^o]) for o = 16, 8, 4, 2, 1.
 #include "common.cuh"
 #include "launch.h"
+#include "rowreduce.cuh"
 
 namespace lrmoe {
 namespace {
 
-template <lrmoe_dtype DT>
-__device__ __forceinline__ float acc_vec(float acc, const uint4& v) {
-  if constexpr (DT == LRMOE_BF16) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float lo = bf16_bits_to_f32(w[i] & 0xffffu);
-      const float hi = bf16_bits_to_f32(w[i] >> 16);
-      acc = __fadd_rn(acc, __fmul_rn(lo, lo));
-      acc = __fadd_rn(acc, __fmul_rn(hi, hi));
-    }
-  } else {
-    const float f[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
-                        __uint_as_float(v.w)};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
-  }
-  return acc;
-}
+using namespace rowred;
 
-// Vectors a lane keeps in registers per row chunk (rows longer than 32 * kMaxV
-// vectors are processed chunk by chunk, which keeps the same order).
-constexpr int kMaxV = 8;
-
-// Load this lane's vectors c = base + lane + 32 i (i < kMaxV) of a row.
-__device__ __forceinline__ void load_chunk(uint4 (&v)[kMaxV], const uint4* __restrict__ row,
-                                           int base, int V, int lane) {
-#pragma unroll
-  for (int i = 0; i < kMaxV; ++i) {
-    const int c = base + lane + 32 * i;
-    v[i] = c < V ? __ldg(row + c) : make_uint4(0, 0, 0, 0);
-  }
-}
-
-// Accumulate a loaded chunk in ascending vector order (padding vectors are zero).
-template <lrmoe_dtype DT>
-__device__ __forceinline__ float acc_chunk(float acc, const uint4 (&v)[kMaxV], int base, int V,
-                                           int lane) {
-#pragma unroll
-  for (int i = 0; i < kMaxV; ++i)
-    if (base + lane + 32 * i < V) acc = acc_vec<DT>(acc, v[i]);
-  return acc;
-}
-
-__device__ __forceinline__ float butterfly(float acc) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(kFull, acc, o));
-  return acc;
-}
-
-// Squared norm of a row whose first chunk is already in `v`.
-template <lrmoe_dtype DT>
-__device__ __forceinline__ float row_sqnorm_from(uint4 (&v)[kMaxV],
-                                                 const uint4* __restrict__ row, int V, int lane) {
-  float acc = acc_chunk<DT>(0.0f, v, 0, V, lane);
-  for (int base = 32 * kMaxV; base < V; base += 32 * kMaxV) {
-    load_chunk(v, row, base, V, lane);
-    acc = acc_chunk<DT>(acc, v, base, V, lane);
-  }
-  return butterfly(acc);
-}
-
-template <lrmoe_dtype DT>
-__global__ void __launch_bounds__(256) score_kernel(const int32_t* __restrict__ idx,
-                                                    const float* __restrict__ w, int T, int k,
-                                                    int E, const uint4* __restrict__ dY, int VH,
-                                                    const uint4* __restrict__ a, int VD,
-                                                    float* __restrict__ score,
-                                                    uint32_t* __restrict__ status) {
+template <lrmoe_dtype DT, int VL, int RPW>
+__global__ void __launch_bounds__(256) row_sqnorm_kernel(const uint4* __restrict__ rows, int n,
+                                                         int V, float* __restrict__ out) {
   const int lane = threadIdx.x & 31;
-  const int warps_per_block = blockDim.x >> 5;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nw = gridDim.x * (blockDim.x >> 5);
   pdl_wait();
   pdl_trigger();
-  for (int t = blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T;
-       t += gridDim.x * warps_per_block) {
-    // routing slots of this token: lane j holds slot j (k <= 32)
-    const size_t p0 = (size_t)t * k;
-    const int e_l = lane < k ? __ldg(idx + p0 + lane) : -1;
-    const float w_l = lane < k ? __ldg(w + p0 + lane) : 0.0f;
-    const unsigned routed = __ballot_sync(kFull, lane < k && e_l >= 0 && e_l < E);
-    if (__any_sync(kFull, lane < k && e_l >= E) && lane == 0)
-      raise_status(status, LRMOE_ST_BAD_EXPERT);
-
-    uint4 vy[kMaxV], va[kMaxV], vn[kMaxV];
-    load_chunk(vy, dY + (size_t)t * VH, 0, VH, lane);
-    int j = routed ? __ffs(routed) - 1 : -1;
-    if (j >= 0) load_chunk(va, a + (p0 + j) * VD, 0, VD, lane);
-    const float ny = row_sqnorm_from<DT>(vy, dY + (size_t)t * VH, VH, lane);
-
-    float s_mine = 0.0f;  // lane j ends up holding slot j's score
-    unsigned todo = routed;
-    while (todo) {
-      j = __ffs(todo) - 1;
-      todo &= todo - 1;
-      const int jn = todo ? __ffs(todo) - 1 : -1;
-      if (jn >= 0) load_chunk(vn, a + (p0 + jn) * VD, 0, VD, lane);  // next row in flight
-      const float na = row_sqnorm_from<DT>(va, a + (p0 + j) * VD, VD, lane);
-      const float wp = __shfl_sync(kFull, w_l, j);
-      float s = __fmul_rn(__fmul_rn(__fmul_rn(wp, wp), ny), na);
-      if (!isfinite(s)) {
-        if (lane == 0) raise_status(status, LRMOE_ST_NONFINITE);
-        if (isnan(s)) s = __uint_as_float(0x7fffffffu);
-      }
-      if (lane == j) s_mine = s;
-      if (jn >= 0) {
+  for (long long r0 = (long long)gw * RPW; r0 < n; r0 += (long long)nw * RPW) {
+    const int here = (int)(n - r0 < RPW ? n - r0 : RPW);
+    float nrm[RPW];
+    warp_row_norms<DT, VL, RPW>(rows + r0 * V, V, here, lane, nrm);
+    float mine = 0.0f;
 #pragma unroll
-        for (int i = 0; i < kMaxV; ++i) va[i] = vn[i];
-      }
-    }
-    if (lane < k) score[p0 + lane] = s_mine;
+    for (int i = 0; i < RPW; ++i)
+      if (lane == i) mine = nrm[i];
+    if (lane < here) out[r0 + lane] = mine;
   }
 }
 
+// score[p] = fl(fl(fl(w*w) * ||dY_t||^2) * na[p]) for routed slots, +0 otherwise.
+// `na` may be the score buffer itself: each slot is read before it is written,
+// by the same thread.
+template <lrmoe_dtype DT, int VL, int RPW>
+__global__ void __launch_bounds__(256) score_norms_kernel(const int32_t* __restrict__ idx,
+                                                          const float* __restrict__ w, int T,
+                                                          int k, int E,
+                                                          const uint4* __restrict__ dY, int VH,
+                                                          const float* na, float* score,
+                                                          uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  pdl_wait();
+  pdl_trigger();
+  for (long long t0 = (long long)gw * RPW; t0 < T; t0 += (long long)nw * RPW) {
+    const int here = (int)(T - t0 < RPW ? T - t0 : RPW);
+    // routing slots of the RPW tokens (lane j holds slot j, k <= 32), in flight
+    // together with the dY rows
+    int e_l[RPW];
+    float w_l[RPW], a_l[RPW];
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+      const bool ok = i < here && lane < k;
+      const size_t p = (size_t)(t0 + i) * k + lane;
+      e_l[i] = ok ? __ldg(idx + p) : -1;
+      w_l[i] = ok ? __ldg(w + p) : 0.0f;
+      a_l[i] = ok ? na[p] : 0.0f;
+    }
+    float ny[RPW];
+    warp_row_norms<DT, VL, RPW>(dY + t0 * VH, VH, here, lane, ny);
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+      if (i >= here) break;
+      if (__any_sync(kFull, lane < k && e_l[i] >= E) && lane == 0)
+        raise_status(status, LRMOE_ST_BAD_EXPERT);
+      const bool routed = lane < k && e_l[i] >= 0 && e_l[i] < E;
+      float s = 0.0f;
+      if (routed) {
+        s = __fmul_rn(__fmul_rn(__fmul_rn(w_l[i], w_l[i]), ny[i]), a_l[i]);
+        if (!isfinite(s)) {
+          raise_status(status, LRMOE_ST_NONFINITE);
+          if (isnan(s)) s = __uint_as_float(0x7fffffffu);
+        }
+      }
+      if (lane < k) score[(size_t)(t0 + i) * k + lane] = s;
+    }
+  }
+}
+
+template <lrmoe_dtype DT, int VL>
+struct NormsF {
+  static cudaError_t run(const void* rows, int n, int V, float* out, cudaStream_t s) {
+    constexpr int RPW = rpw_of<VL>();
+    auto kern = row_sqnorm_kernel<DT, VL, RPW>;
+    const int grid = grid_for(kern, ((long long)n + RPW - 1) / RPW);
+    return launch_pdl(kern, dim3(grid), dim3(256), 0, s, static_cast<const uint4*>(rows), n, V,
+                      out);
+  }
+};
+
+template <lrmoe_dtype DT, int VL>
+struct ScoreF {
+  static cudaError_t run(const int32_t* idx, const float* w, int T, int k, int E, const void* dY,
+                         int VH, const float* na, float* score, uint32_t* status, cudaStream_t s) {
+    constexpr int RPW = rpw_of<VL>();
+    auto kern = score_norms_kernel<DT, VL, RPW>;
+    const int grid = grid_for(kern, ((long long)T + RPW - 1) / RPW);
+    return launch_pdl(kern, dim3(grid), dim3(256), 0, s, idx, w, T, k, E,
+                      static_cast<const uint4*>(dY), VH, na, score, status);
+  }
+};
+
 }  // namespace
+
+cudaError_t launch_row_sqnorm(const void* rows, int n, int D, lrmoe_dtype dt, float* out,
+                              cudaStream_t s) {
+  const int V = D / (dt == LRMOE_BF16 ? 8 : 4);
+  if (dt == LRMOE_BF16) return by_vl<LRMOE_BF16, NormsF>(V, rows, n, V, out, s);
+  return by_vl<LRMOE_F32, NormsF>(V, rows, n, V, out, s);
+}
+
+cudaError_t launch_score_from_norms(const int32_t* idx, const float* w, int T, int k, int E,
+                                    const void* dY, int H, const float* a_sqnorm, lrmoe_dtype dt,
+                                    float* score, uint32_t* status, cudaStream_t s) {
+  const int VH = H / (dt == LRMOE_BF16 ? 8 : 4);
+  if (dt == LRMOE_BF16)
+    return by_vl<LRMOE_BF16, ScoreF>(VH, idx, w, T, k, E, dY, VH, a_sqnorm, score, status, s);
+  return by_vl<LRMOE_F32, ScoreF>(VH, idx, w, T, k, E, dY, VH, a_sqnorm, score, status, s);
+}
 
 cudaError_t launch_score(const int32_t* idx, const float* w, int T, int k, int E, const void* dY,
                          int H, const void* a, int D, lrmoe_dtype dt, float* score,
                          uint32_t* status, cudaStream_t s) {
-  const int per_vec = dt == LRMOE_BF16 ? 8 : 4;
-  const int VH = H / per_vec, VD = D / per_vec;
-  const int threads = 256, wpb = threads / 32;
-  const int blocks_needed = (T + wpb - 1) / wpb;
-  const int max_blocks = num_sms() * (2048 / threads);
-  const int blocks = blocks_needed < max_blocks ? blocks_needed : max_blocks;
-  auto kern = dt == LRMOE_BF16 ? score_kernel<LRMOE_BF16> : score_kernel<LRMOE_F32>;
-  return launch_pdl(kern, dim3(blocks), dim3(threads), 0, s, idx, w, T, k, E,
-                    static_cast<const uint4*>(dY), VH, static_cast<const uint4*>(a), VD, score,
-                    status);
+  cudaError_t e = launch_row_sqnorm(a, T * k, D, dt, score, s);
+  if (e != cudaSuccess) return e;
+  return launch_score_from_norms(idx, w, T, k, E, dY, H, score, dt, score, status, s);
 }
 
 }  // namespace lrmoe

@@ -25,7 +25,8 @@ ST_BAD_EXPERT, ST_BAD_QUOTA, ST_NONFINITE, ST_TIMEOUT, ST_BAD_INDEX = 1, 2, 4, 8
 EXPORTS = ("lrmoe_version", "lrmoe_status_string", "lrmoe_last_error", "lrmoe_score",
            "lrmoe_select_workspace_bytes", "lrmoe_select_quota", "lrmoe_pack",
            "lrmoe_grouped_dgrad", "lrmoe_grouped_wgrad", "lrmoe_unpack", "lrmoe_pruned_backward",
-           "lrmoe_select_quota_noalloc", "lrmoe_selftest_bounded_wait", "lrmoe_quota_controller")
+           "lrmoe_select_quota_noalloc", "lrmoe_selftest_bounded_wait", "lrmoe_quota_controller",
+           "lrmoe_row_sqnorm", "lrmoe_score_from_norms", "lrmoe_router_grad")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -61,6 +62,9 @@ def load() -> ctypes.CDLL:
     lib.lrmoe_status_string.argtypes = [I]
     lib.lrmoe_last_error.restype = ctypes.c_char_p
     lib.lrmoe_score.argtypes = [P, P, I, I, I, P, I, P, I, I, P, P, P]
+    lib.lrmoe_row_sqnorm.argtypes = [P, I, I, I, P, P]
+    lib.lrmoe_router_grad.argtypes = [P, I, I, I, P, I, P, I, P, P, P, P]
+    lib.lrmoe_score_from_norms.argtypes = [P, P, I, I, I, P, I, P, I, P, P, P]
     lib.lrmoe_select_workspace_bytes.argtypes = [I, I, I]
     lib.lrmoe_select_workspace_bytes.restype = Z
     lib.lrmoe_select_quota.argtypes = [P, P, I, I, I, P, P, P, P, P, P, P, Z, P, P]
@@ -122,6 +126,29 @@ def lrmoe_score(topk_idx, topk_w, dY, a_saved, E: int, score, status=None, strea
     _check(load().lrmoe_score(_ptr(topk_idx), _ptr(topk_w), T, k, E, _ptr(dY), dY.shape[-1],
                               _ptr(a_saved), a_saved.shape[-1], _dt(dY), _ptr(score), _ptr(status),
                               _stream(stream)))
+
+
+def lrmoe_row_sqnorm(rows, out, stream=None) -> None:
+    """out[r] = ||rows[r]||^2 (canonical order) for every row of a 2-D tensor."""
+    _check(load().lrmoe_row_sqnorm(_ptr(rows), rows.shape[0], rows.shape[-1], _dt(rows), _ptr(out),
+                                   _stream(stream)))
+
+
+def lrmoe_score_from_norms(topk_idx, topk_w, dY, a_sqnorm, E: int, score, status=None,
+                           stream=None) -> None:
+    T, k = topk_idx.shape
+    _check(load().lrmoe_score_from_norms(_ptr(topk_idx), _ptr(topk_w), T, k, E, _ptr(dY),
+                                         dY.shape[-1], _ptr(a_sqnorm), _dt(dY), _ptr(score),
+                                         _ptr(status), _stream(stream)))
+
+
+def lrmoe_router_grad(topk_idx, dY, y_saved, E: int, dw, pos=None, status=None,
+                      stream=None) -> None:
+    """dw[p] = <dY_t, y_p> for routed pairs (retained pairs only when pos is given)."""
+    T, k = topk_idx.shape
+    _check(load().lrmoe_router_grad(_ptr(topk_idx), T, k, E, _ptr(dY), dY.shape[-1],
+                                    _ptr(y_saved), _dt(dY), _ptr(pos), _ptr(dw), _ptr(status),
+                                    _stream(stream)))
 
 
 def lrmoe_select_quota(topk_idx, score, quota, counts, kept, offsets, perm, pos, workspace,

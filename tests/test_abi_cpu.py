@@ -66,6 +66,32 @@ def test_score_rejects_bad_arguments(lib):
     assert f(FAKE, FAKE, 4, 33, 40, FAKE, 8, FAKE, 8, 1, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
 
 
+def test_row_norm_and_score_from_norms_reject_bad_arguments(lib):
+    f = lib.lrmoe_row_sqnorm
+    assert f(NULL, 4, 8, 1, FAKE, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert b"rows" in lib.lrmoe_last_error()
+    assert f(FAKE, 0, 8, 1, FAKE, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert f(FAKE, 4, 12, 1, FAKE, NULL) == L.LRMOE_ERR_INVALID_ARG   # D % 8 for bf16
+    assert f(FAKE, 4, 8, 5, FAKE, NULL) == L.LRMOE_ERR_INVALID_ARG    # dtype
+    assert f(FAKE, 4, 8, 1, ctypes.c_void_p(0x10004), NULL) == L.LRMOE_ERR_INVALID_ARG
+    g = lib.lrmoe_score_from_norms
+    assert g(FAKE, FAKE, 4, 2, 3, FAKE, 8, NULL, 1, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert b"a_sqnorm" in lib.lrmoe_last_error()
+    assert g(FAKE, FAKE, 4, 2, 3, FAKE, 6, FAKE, 0, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert g(FAKE, FAKE, 4, 33, 40, FAKE, 8, FAKE, 1, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert g(FAKE, FAKE, 4, 2, 0, FAKE, 8, FAKE, 1, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+
+
+def test_router_grad_rejects_bad_arguments(lib):
+    f = lib.lrmoe_router_grad
+    assert f(FAKE, 4, 2, 3, FAKE, 8, NULL, 1, NULL, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert b"y_saved" in lib.lrmoe_last_error()
+    assert f(FAKE, 4, 2, 3, FAKE, 8, FAKE, 1, ctypes.c_void_p(0x10004), FAKE, NULL, NULL) \
+        == L.LRMOE_ERR_INVALID_ARG
+    assert f(FAKE, 4, 2, 3, FAKE, 10, FAKE, 1, NULL, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert f(FAKE, 4, 0, 3, FAKE, 8, FAKE, 1, NULL, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+
+
 def test_select_rejects_small_workspace(lib):
     f = lib.lrmoe_select_quota
     need = L.lrmoe_select_workspace_bytes(64, 2, 4)
