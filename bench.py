@@ -40,7 +40,7 @@ METRIC = "retained pairs/s + expert-bwd TFLOP/s on 1 B200; % of HBM / bf16 roofl
 UNIT = "retained pairs/s"
 DEFAULT_CONFIG = "qwen"
 KERNELS = ("score", "select", "pack", "dgrad_swiglu", "wgrad_down", "wgrad_gu", "dgrad_x", "unpack")
-KERNEL_LAUNCHES = {"score": 1, "select": 4, "pack": 1, "dgrad_swiglu": 1, "wgrad_down": 1,
+KERNEL_LAUNCHES = {"score": 2, "select": 4, "pack": 1, "dgrad_swiglu": 1, "wgrad_down": 1,
                    "wgrad_gu": 1, "dgrad_x": 1, "unpack": 1}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -364,10 +364,16 @@ def make_runner(layer, dev):
         flush.sum()
     st = out["status"]
 
-    def step(ev=None):
+    def step(ev=None, a_sqnorm=None):
+        """One pass of the path; with a_sqnorm (||a_p||^2 saved by the forward) the
+        score reads dY and the saved norms instead of a."""
+        score_call = (
+            (lambda: L.lrmoe_score(inp["topk_idx"], inp["topk_w"], inp["dY"], inp["a"], s.E,
+                                   out["score"], st, stream)) if a_sqnorm is None else
+            (lambda: L.lrmoe_score_from_norms(inp["topk_idx"], inp["topk_w"], inp["dY"], a_sqnorm,
+                                              s.E, out["score"], st, stream)))
         calls = (
-            lambda: L.lrmoe_score(inp["topk_idx"], inp["topk_w"], inp["dY"], inp["a"], s.E,
-                                  out["score"], st, stream),
+            score_call,
             lambda: L.lrmoe_select_quota(inp["topk_idx"], out["score"], inp["quota"], out["counts"],
                                          out["kept"], out["offsets"], out["perm"], out["pos"],
                                          out["workspace"], st, stream),
@@ -494,6 +500,90 @@ def run_gpu(args):
     controller_us = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in ctl_ev)
     controller_matches = bool(torch.equal(q_dev, inp["quota"])) if s.quota == "capacity" else None
 
+    # ---------------- score from forward-saved ||a_p||^2 ----------------
+    # The forward can save ||a_p||^2 when it writes a; the backward's score then
+    # reads dY and 4 bytes per pair.  Timed per call after an L2 flush, and as
+    # whole steps with that score in place of the full one.
+    a2d = inp["a"].view(s.P, s.I)
+    na = torch.empty(s.P, dtype=torch.float32, device=dev)
+    L.lrmoe_row_sqnorm(a2d, na, stream)
+    sn_calls = {
+        "row_sqnorm": lambda: L.lrmoe_row_sqnorm(a2d, na, stream),
+        "score_from_norms": lambda: L.lrmoe_score_from_norms(
+            inp["topk_idx"], inp["topk_w"], inp["dY"], na, s.E, out["score"], st, stream),
+        "score": lambda: L.lrmoe_score(inp["topk_idx"], inp["topk_w"], inp["dY"], inp["a"], s.E,
+                                       out["score"], st, stream),
+    }
+    sn_us = {}
+    for name_, fn in sn_calls.items():
+        evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(20)]
+        for i in range(23):
+            flush_l2()
+            if i >= 3:
+                evp[i - 3][0].record(stream)
+            fn()
+            if i >= 3:
+                evp[i - 3][1].record(stream)
+        torch.cuda.synchronize(dev)
+        sn_us[name_] = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp)
+    sn_steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(n_bd)]
+    for i in range(n_bd):
+        flush_l2()
+        sn_steps[i][0].record(stream)
+        step(a_sqnorm=na)
+        sn_steps[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    sn_step_ms = max_over_ranks(statistics.fmean(a_.elapsed_time(b_) for a_, b_ in sn_steps), dist)
+    sn_bytes = s.T * s.H * b + 16 * s.P          # dY, idx, w, saved norm, score
+    saved_norms = {
+        "row_sqnorm_us": sn_us["row_sqnorm"], "score_from_norms_us": sn_us["score_from_norms"],
+        "score_us": sn_us["score"],
+        "score_from_norms_GB/s": sn_bytes / (sn_us["score_from_norms"] * 1e-6) / 1e9,
+        "score_from_norms_hbm_frac": sn_bytes / (sn_us["score_from_norms"] * 1e-6) / 1e9
+        / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+        "step_ms": sn_step_ms, "value": M_all / (sn_step_ms * 1e-3), "unit": UNIT,
+        "steps": n_bd,
+    }
+    if int(st.item()) != 0:
+        raise SystemExit(f"device status {int(st.item())} after the saved-norm steps")
+
+    # ---------------- routing-weight gradient from saved expert outputs ----------------
+    # y_p = W_down[e] a_p is what the forward saves; it is generated here with torch
+    # (input generation, not part of the path), then dw = <dY_t, y_p> is timed for
+    # the retained pairs (pos from the selection) and for every routed pair.
+    y_dev = torch.empty(s.P, s.H, dtype=tdt, device=dev)
+    flat_idx = inp["topk_idx"].view(-1)
+    for e in range(s.E):
+        sel = (flat_idx == e).nonzero().squeeze(1)
+        if sel.numel():
+            y_dev[sel] = a2d[sel] @ inp["W_down"][e].T
+    dw = torch.empty(s.P, dtype=torch.float32, device=dev)
+    router = {}
+    for mode, pos_arg, nbytes in (
+            ("retained", out["pos"], M * s.H * b + s.T * s.H * b + 12 * s.P),
+            ("all", None, s.P * s.H * b + s.T * s.H * b + 8 * s.P)):
+        evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(20)]
+        for i in range(23):
+            flush_l2()
+            if i >= 3:
+                evp[i - 3][0].record(stream)
+            L.lrmoe_router_grad(inp["topk_idx"], inp["dY"], y_dev, s.E, dw, pos=pos_arg,
+                                status=st, stream=stream)
+            if i >= 3:
+                evp[i - 3][1].record(stream)
+        torch.cuda.synchronize(dev)
+        us = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        router[mode] = {"us": us, "GB/s": gbs,
+                        "hbm_frac": gbs / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+                        "algorithmic_bytes": nbytes}
+    del y_dev
+    if int(st.item()) != 0:
+        raise SystemExit(f"device status {int(st.item())} after the router gradient")
+
     # ---------------- end to end through host buffers ----------------
     pin = {k_: v.pin_memory() for k_, v in host.items()}
     dX_host = torch.empty(s.T, s.H, dtype=tdt).pin_memory()
@@ -543,6 +633,8 @@ def run_gpu(args):
         "breakdown": breakdown,
         "quota_controller_us": controller_us,
         "quota_controller_equals_capacity_rule": controller_matches,
+        "saved_norms": saved_norms,
+        "router_grad": router,
         "breakdown_steps": n_bd,
         "breakdown_step_ms": sum(kern_ms.values()),
         "cpu_baseline": cpu,
