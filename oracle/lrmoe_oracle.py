@@ -37,6 +37,12 @@ forward          the ordinary SwiGLU MoE forward in fp64, used only by the
                  finite-difference pin ([RU-B] bullet 1: the forward stays full).
 lrm_score_from_norms  the score with ||a_p||^2 given (saved by the forward);
                  the same three factors, multiplied in the same order.
+redistribute     [RU-B] bullet 4 / [FR-B] bullet 4: the remaining pairs of each
+                 expert are spread over the admissible copies of that expert
+                 by an integer algorithm that minimises the peak load of one
+                 GPU; no new copies appear (R11).
+split_by_destination  [RU-B] bullet 5: retained rows are grouped by receiver
+                 and expert, so the all-to-all moves compact blocks.
 router_grad      the gradient of the routing weights, dL/dw_p = <dY_t, y_p>
                  with y_p = W_down[e] a_p the pair's expert output (the layer
                  output is sum_j w_tj y_tj); the pages do not treat it (R8).
@@ -53,6 +59,10 @@ Readings where the pages are silent:
   R6  the packed gradient row is RNE_storage(fp32(w) * fp32(dY_t)); all
       gradient arithmetic afterwards is fp64 here.
   R7  topk_idx < 0 = not routed; idx >= E = invalid (skipped, status bit).
+  R11 the load of a GPU is the number of retained pairs it serves (every pair of
+      a layer costs the same); an expert's pairs, in the global order (source
+      rank, then packed row), are cut into consecutive runs, one per copy in
+      ascending GPU order, with the run lengths of the optimal plan.
   R8  the routing-weight gradient is not part of the pruned path; when asked
       for, it is <dY_t, y_p> with y_p saved by the forward, for every routed
       pair, or for the retained pairs only when pos is given (dropped pairs
@@ -211,6 +221,111 @@ def router_grad(topk_idx, dY, y, dtype: str, E: int, pos=None):
     dy_p = np.repeat(decode(dY, dtype), k, axis=0)
     d = row_dot(dy_p, decode(y, dtype), VEC[dtype])
     return np.where(keep, d, np.float32(0.0)).astype(np.float32), status
+
+
+def redistribute_peak(m, admissible):
+    """Smallest achievable peak load, from Hall's condition for the transportation
+    problem: the plan with peak L exists iff for every set S of GPUs the experts
+    whose copies all lie in S fit, sum_{e: A_e within S} m_e <= L |S|.  So
+    L* = max over nonempty S of ceil(D(S) / |S|).  Exponential in G (small G only)."""
+    m = np.asarray(m, np.int64)
+    A = np.asarray(admissible, bool)
+    E, G = A.shape
+    best = 0
+    for mask in range(1, 1 << G):
+        inside = np.array([(mask >> g) & 1 for g in range(G)], bool)
+        confined = ~np.any(A & ~inside[None, :], axis=1) & np.any(A, axis=1)
+        D = int(m[confined].sum())
+        size = int(inside.sum())
+        best = max(best, -(-D // size))
+    return best
+
+
+def redistribute(m, admissible):
+    """Integer plan x[e][g] >= 0: sum_g x[e][g] = m_e, x[e][g] = 0 where expert e
+    has no copy on GPU g, and max_g sum_e x[e][g] equal to redistribute_peak.
+    The plan comes from augmenting paths (breadth-first, Edmonds-Karp) on the
+    network source -> expert (cap m_e) -> its copies -> sink (cap L*)."""
+    m = np.asarray(m, np.int64)
+    A = np.asarray(admissible, bool)
+    E, G = A.shape
+    if np.any((m > 0) & ~np.any(A, axis=1)):
+        raise ValueError("an expert with retained pairs has no copy")
+    L = redistribute_peak(m, A)
+    n = E + G + 2
+    src, snk = E + G, E + G + 1
+    cap = np.zeros((n, n), np.int64)
+    for e in range(E):
+        cap[src, e] = m[e]
+        for g in range(G):
+            if A[e, g]:
+                cap[e, E + g] = m[e]
+    for g in range(G):
+        cap[E + g, snk] = L
+    flow = np.zeros((n, n), np.int64)
+    while True:
+        prev = [-1] * n
+        prev[src] = src
+        queue = [src]
+        for u in queue:
+            for v in range(n):
+                if prev[v] < 0 and cap[u, v] - flow[u, v] > 0:
+                    prev[v] = u
+                    queue.append(v)
+        if prev[snk] < 0:
+            break
+        push, v = None, snk
+        while v != src:
+            u = prev[v]
+            r = cap[u, v] - flow[u, v]
+            push = r if push is None else min(push, r)
+            v = u
+        v = snk
+        while v != src:
+            u = prev[v]
+            flow[u, v] += push
+            flow[v, u] -= push
+            v = u
+    x = np.zeros((E, G), np.int64)
+    for e in range(E):
+        for g in range(G):
+            x[e, g] = max(0, flow[e, E + g])
+    assert np.array_equal(x.sum(axis=1), m), "no plan at the Hall peak"
+    return x, L
+
+
+def split_by_destination(perm, offsets, plan, global_start=None):
+    """Regroup this rank's packed rows by destination GPU, then expert (R11).
+
+    Expert e's local rows r in [offsets[e], offsets[e+1]) have global indices
+    global_start[e] + (r - offsets[e]); copy g serves the global run
+    [C[e][g], C[e][g+1]) with C the prefix sum of plan[e] over g.  Returns
+    perm_dest (pair ids in destination-major order), dest_offsets [G+1] and
+    dest_expert_offsets [G][E+1] (offsets inside each destination's block)."""
+    plan = np.asarray(plan, np.int64)
+    E, G = plan.shape
+    offsets = np.asarray(offsets, np.int64)
+    start = np.zeros(E, np.int64) if global_start is None else np.asarray(global_start, np.int64)
+    C = np.concatenate([np.zeros((E, 1), np.int64), np.cumsum(plan, axis=1)], axis=1)
+    blocks = [[[] for _ in range(E)] for _ in range(G)]
+    for e in range(E):
+        for r in range(offsets[e], offsets[e + 1]):
+            gi = start[e] + (r - offsets[e])
+            for g in range(G):
+                if C[e, g] <= gi < C[e, g + 1]:
+                    blocks[g][e].append(int(perm[r]))
+                    break
+            else:
+                raise ValueError("plan does not cover every retained row")
+    perm_dest, dest_offsets = [], [0]
+    dest_expert_offsets = np.zeros((G, E + 1), np.int32)
+    for g in range(G):
+        for e in range(E):
+            dest_expert_offsets[g, e + 1] = dest_expert_offsets[g, e] + len(blocks[g][e])
+            perm_dest.extend(blocks[g][e])
+        dest_offsets.append(len(perm_dest))
+    return (np.asarray(perm_dest, np.int32), np.asarray(dest_offsets, np.int32),
+            dest_expert_offsets)
 
 
 def quota_controller(topk_idx, E: int, cap: int, max_pairs: int):

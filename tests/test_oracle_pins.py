@@ -543,3 +543,81 @@ def test_row_dot_of_a_row_with_itself_is_its_norm():
     for vec in (4, 8):
         np.testing.assert_array_equal(O.row_dot(x, x, vec).view(np.uint32),
                                       O.row_sq_norm(x, vec).view(np.uint32))
+
+
+# ----------------------------------------------------------------------------
+# integer redistribution over expert copies (reading R11)
+# ----------------------------------------------------------------------------
+def _brute_force_peak(m, A):
+    """Minimum over every integer plan of the peak load (tiny instances)."""
+    import itertools
+    E, G = A.shape
+    per_expert = []
+    for e in range(E):
+        gs = [g for g in range(G) if A[e, g]]
+        opts = []
+        for split in itertools.product(range(m[e] + 1), repeat=len(gs)):
+            if sum(split) == m[e]:
+                row = [0] * G
+                for g, c in zip(gs, split):
+                    row[g] = c
+                opts.append(row)
+        per_expert.append(opts)
+    best = None
+    for plan in itertools.product(*per_expert):
+        peak = max(sum(plan[e][g] for e in range(E)) for g in range(G))
+        best = peak if best is None else min(best, peak)
+    return best
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_redistribute_equals_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    E, G = int(rng.integers(1, 4)), int(rng.integers(1, 4))
+    m = rng.integers(0, 5, size=E)
+    A = rng.random((E, G)) < 0.6
+    A[np.arange(E), rng.integers(0, G, size=E)] = True      # every expert has a copy
+    x, L = O.redistribute(m, A)
+    assert L == _brute_force_peak(m, A)
+    assert np.array_equal(x.sum(axis=1), m) and np.all(x[~A] == 0) and np.all(x >= 0)
+    assert x.sum(axis=0).max() == L if m.sum() else L == 0
+
+
+def test_redistribute_closed_forms():
+    # one copy per expert: the peak is the most loaded GPU's own experts
+    A = np.eye(4, dtype=bool)[[0, 1, 1, 3, 2]]
+    m = np.array([7, 2, 9, 4, 1])
+    assert O.redistribute(m, A)[1] == 11
+    # every expert everywhere: ceil(M / G)
+    A = np.ones((5, 3), bool)
+    assert O.redistribute(m, A)[1] == -(-23 // 3)
+    # a hot expert with two copies next to cold single-copy experts
+    A = np.zeros((3, 3), bool)
+    A[0, [0, 1]] = True
+    A[1, 1] = A[2, 2] = True
+    assert O.redistribute([10, 4, 1], A)[1] == 7
+    with pytest.raises(ValueError):
+        O.redistribute([1, 0], np.array([[False, False], [True, True]]))
+
+
+def test_split_by_destination_covers_each_global_run_once():
+    """Two ranks' rows of the same experts, cut by one plan: every (copy, expert)
+    run is filled exactly once, in global order, and each block keeps pair order."""
+    plan = np.array([[3, 4, 0], [0, 2, 2], [5, 0, 0]])
+    m0 = np.array([4, 1, 2])
+    m1 = plan.sum(axis=1) - m0
+    got = {}
+    for rank, (mine, start) in enumerate([(m0, np.zeros(3)), (m1, m0)]):
+        offsets = np.concatenate([[0], np.cumsum(mine)])
+        perm = np.arange(offsets[-1]) * 10 + rank            # ascending within each expert
+        pd, do, deo = O.split_by_destination(perm, offsets, plan, start)
+        assert sorted(pd.tolist()) == sorted(perm.tolist())
+        for g in range(3):
+            for e in range(3):
+                blk = pd[do[g] + deo[g, e]: do[g] + deo[g, e + 1]]
+                assert list(blk) == sorted(blk)
+                got.setdefault((g, e), 0)
+                got[(g, e)] += len(blk)
+    for g in range(3):
+        for e in range(3):
+            assert got[(g, e)] == plan[e, g]
