@@ -179,6 +179,49 @@ int lrmoe_select_quota(const int32_t* topk_idx, const float* score, int T, int k
                        uint32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Redistribution over expert copies.  RU-B bullet 4, FR-B bullet 4: the
+ * remaining pairs are spread over the admissible copies of their expert by an
+ * integer algorithm that minimises the peak load of one GPU; no new copies
+ * appear in the backward.
+ *
+ * lrmoe_redistribute (HOST pointers, no CUDA call): m [E] int64 retained pairs
+ * per expert (all ranks together), admissible [E][G] uint8 (nonzero: GPU g
+ * holds a copy of expert e).  Writes plan [E][G] int64 with sum_g plan[e][g] =
+ * m_e, plan[e][g] = 0 where there is no copy, and the smallest possible peak
+ * max_g sum_e plan[e][g] into *peak (binary search on the peak, each probe a
+ * max-flow; the load of a GPU is its number of pairs).  The plan is one of
+ * possibly several optimal ones.  Errors: sizes <= 0, m_e < 0, or m_e > 0 for
+ * an expert with no copy -> LRMOE_ERR_INVALID_ARG.
+ * ------------------------------------------------------------------------- */
+int lrmoe_redistribute(const int64_t* m, const uint8_t* admissible, int E, int G, int64_t* plan,
+                       int64_t* peak);
+
+/* ---------------------------------------------------------------------------
+ * Split by destination.  RU-B bullet 5, FR-B bullet 5: the remaining rows are
+ * grouped by receiver and expert, so the all-to-all moves compact blocks.
+ *
+ * This rank's packed rows (perm, offsets [E+1] from lrmoe_select_quota) are
+ * cut by plan [E][G] int32 (device; the redistribute plan): expert e's local
+ * rows have global indices global_start[e] + (r - offsets[e]) (global_start
+ * [E] int32 device = the rows of e on lower ranks; NULL = 0, one rank), and
+ * GPU g serves the global run [C[e][g], C[e][g+1]), C = prefix sum of
+ * plan[e] over g.  Outputs (device, int32):
+ *   perm_dest [rows_cap]         the pair ids regrouped destination-major, then
+ *                                expert, then in packed order
+ *   dest_offsets [G+1]           start of each destination's block (last = M)
+ *   dest_expert_offsets [G][E+1] expert offsets inside each block (the
+ *                                receiver's grouped-GEMM offsets for this source)
+ * lrmoe_pack(perm_dest, dest_offsets, ..., E = G, ...) then gathers the send
+ * buffer (pack reads only offsets[E], the row count).  Rows that the plan
+ * does not cover, and negative plan entries, set LRMOE_ST_BAD_INDEX; such rows
+ * are left out.
+ * ------------------------------------------------------------------------- */
+int lrmoe_split_by_destination(const int32_t* perm, const int32_t* offsets, const int32_t* plan,
+                               const int32_t* global_start, int E, int G, int rows_cap,
+                               int32_t* perm_dest, int32_t* dest_offsets,
+                               int32_t* dest_expert_offsets, uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Quota controller.  RU-B bullet 2, FR-B bullet 2, DE paragraph 3: before the
  * backward a controller sees how many tokens came to each expert and, within
  * the memory limit, fixes how many pairs of each expert stay for the layer

@@ -150,6 +150,46 @@ int lrmoe_router_grad(const int32_t* topk_idx, int T, int k, int E, const void* 
   return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_router_grad launch");
 }
 
+int lrmoe_redistribute(const int64_t* m, const uint8_t* admissible, int E, int G, int64_t* plan,
+                       int64_t* peak) {
+  g_last_error[0] = 0;
+  REQUIRE(E > 0 && G > 0, "E=%d and G=%d must be positive", E, G);
+  REQUIRE(E <= 65536 && G <= 4096, "E=%d or G=%d too large for the planner", E, G);
+  REQUIRE(m != nullptr && admissible != nullptr && plan != nullptr && peak != nullptr,
+          "m, admissible, plan and peak must be non-null host pointers");
+  for (int e = 0; e < E; ++e) {
+    REQUIRE(m[e] >= 0, "m[%d]=%lld is negative", e, (long long)m[e]);
+    bool any = false;
+    for (int g = 0; g < G; ++g) any = any || admissible[(size_t)e * G + g] != 0;
+    REQUIRE(any || m[e] == 0, "expert %d has %lld retained pairs but no copy", e,
+            (long long)m[e]);
+  }
+  if (redistribute_plan(m, admissible, E, G, plan, peak) != 0)
+    return fail(LRMOE_ERR_INVALID_ARG, "no plan exists (an expert without a copy)");
+  return LRMOE_OK;
+}
+
+int lrmoe_split_by_destination(const int32_t* perm, const int32_t* offsets, const int32_t* plan,
+                               const int32_t* global_start, int E, int G, int rows_cap,
+                               int32_t* perm_dest, int32_t* dest_offsets,
+                               int32_t* dest_expert_offsets, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(E > 0 && E <= kMaxGroupedExperts, "E=%d must be in [1, %d]", E, kMaxGroupedExperts);
+  REQUIRE(G > 0 && (size_t)E * G * sizeof(int) <= 200 * 1024, "G=%d out of range for E=%d", G, E);
+  REQUIRE(rows_cap > 0, "rows_cap=%d must be positive", rows_cap);
+  REQUIRE_PTR(perm);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(plan);
+  REQUIRE_PTR(perm_dest);
+  REQUIRE_PTR(dest_offsets);
+  REQUIRE_PTR(dest_expert_offsets);
+  REQUIRE(global_start == nullptr || aligned16(global_start), "global_start is not 16-byte aligned");
+  cudaError_t e = launch_split_by_destination(perm, offsets, plan, global_start, E, G, rows_cap,
+                                              perm_dest, dest_offsets, dest_expert_offsets, status,
+                                              static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_split_by_destination launch");
+}
+
 size_t lrmoe_select_workspace_bytes(int T, int k, int E) {
   if (T <= 0 || k <= 0 || E <= 0) return 0;
   return select_ws_layout(T, k, E).total;

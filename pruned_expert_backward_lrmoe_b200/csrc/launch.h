@@ -40,6 +40,13 @@ cudaError_t launch_score(const int32_t* idx, const float* w, int T, int k, int E
 cudaError_t launch_router_grad(const int32_t* idx, int T, int k, int E, const void* dY, int H,
                                const void* y, lrmoe_dtype dt, const int32_t* pos, float* dw,
                                uint32_t* status, cudaStream_t s);
+int redistribute_plan(const int64_t* m, const uint8_t* adm, int E, int G, int64_t* x,
+                      int64_t* peak);
+cudaError_t launch_split_by_destination(const int32_t* perm, const int32_t* offsets,
+                                        const int32_t* plan, const int32_t* start, int E, int G,
+                                        int rows_cap, int32_t* perm_dest, int32_t* dest_offsets,
+                                        int32_t* dest_expert_offsets, uint32_t* status,
+                                        cudaStream_t s);
 cudaError_t launch_row_sqnorm(const void* rows, int n, int D, lrmoe_dtype dt, float* out,
                               cudaStream_t s);
 cudaError_t launch_score_from_norms(const int32_t* idx, const float* w, int T, int k, int E,

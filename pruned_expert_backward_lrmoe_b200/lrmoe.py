@@ -26,7 +26,8 @@ EXPORTS = ("lrmoe_version", "lrmoe_status_string", "lrmoe_last_error", "lrmoe_sc
            "lrmoe_select_workspace_bytes", "lrmoe_select_quota", "lrmoe_pack",
            "lrmoe_grouped_dgrad", "lrmoe_grouped_wgrad", "lrmoe_unpack", "lrmoe_pruned_backward",
            "lrmoe_select_quota_noalloc", "lrmoe_selftest_bounded_wait", "lrmoe_quota_controller",
-           "lrmoe_row_sqnorm", "lrmoe_score_from_norms", "lrmoe_router_grad")
+           "lrmoe_row_sqnorm", "lrmoe_score_from_norms", "lrmoe_router_grad",
+           "lrmoe_redistribute", "lrmoe_split_by_destination")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -64,6 +65,8 @@ def load() -> ctypes.CDLL:
     lib.lrmoe_score.argtypes = [P, P, I, I, I, P, I, P, I, I, P, P, P]
     lib.lrmoe_row_sqnorm.argtypes = [P, I, I, I, P, P]
     lib.lrmoe_router_grad.argtypes = [P, I, I, I, P, I, P, I, P, P, P, P]
+    lib.lrmoe_redistribute.argtypes = [P, P, I, I, P, P]
+    lib.lrmoe_split_by_destination.argtypes = [P, P, P, P, I, I, I, P, P, P, P, P]
     lib.lrmoe_score_from_norms.argtypes = [P, P, I, I, I, P, I, P, I, P, P, P]
     lib.lrmoe_select_workspace_bytes.argtypes = [I, I, I]
     lib.lrmoe_select_workspace_bytes.restype = Z
@@ -149,6 +152,30 @@ def lrmoe_router_grad(topk_idx, dY, y_saved, E: int, dw, pos=None, status=None,
     _check(load().lrmoe_router_grad(_ptr(topk_idx), T, k, E, _ptr(dY), dY.shape[-1],
                                     _ptr(y_saved), _dt(dY), _ptr(pos), _ptr(dw), _ptr(status),
                                     _stream(stream)))
+
+
+def lrmoe_redistribute(m, admissible):
+    """Host planner: (plan [E][G] int64, peak) for retained counts m [E] and the
+    copy map admissible [E][G] (numpy or CPU tensors)."""
+    import numpy as np
+    m = np.ascontiguousarray(np.asarray(m), dtype=np.int64)
+    adm = np.ascontiguousarray(np.asarray(admissible) != 0, dtype=np.uint8)
+    E, G = adm.shape
+    plan = np.zeros((E, G), dtype=np.int64)
+    peak = np.zeros(1, dtype=np.int64)
+    _check(load().lrmoe_redistribute(m.ctypes.data, adm.ctypes.data, E, G, plan.ctypes.data,
+                                     peak.ctypes.data))
+    return plan, int(peak[0])
+
+
+def lrmoe_split_by_destination(perm, offsets, plan, perm_dest, dest_offsets, dest_expert_offsets,
+                               global_start=None, status=None, stream=None) -> None:
+    E, G = plan.shape
+    _check(load().lrmoe_split_by_destination(_ptr(perm), _ptr(offsets), _ptr(plan),
+                                             _ptr(global_start), E, G, perm.shape[0],
+                                             _ptr(perm_dest), _ptr(dest_offsets),
+                                             _ptr(dest_expert_offsets), _ptr(status),
+                                             _stream(stream)))
 
 
 def lrmoe_select_quota(topk_idx, score, quota, counts, kept, offsets, perm, pos, workspace,

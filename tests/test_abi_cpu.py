@@ -92,6 +92,19 @@ def test_router_grad_rejects_bad_arguments(lib):
     assert f(FAKE, 4, 0, 3, FAKE, 8, FAKE, 1, NULL, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
 
 
+def test_split_by_destination_rejects_bad_arguments(lib):
+    f = lib.lrmoe_split_by_destination
+    args = [FAKE, FAKE, FAKE, NULL, 4, 2, 100, FAKE, FAKE, FAKE, NULL, NULL]
+    bad = list(args); bad[2] = NULL                       # plan
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG and b"plan" in lib.lrmoe_last_error()
+    bad = list(args); bad[4] = 0                          # E
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
+    bad = list(args); bad[5] = 100000                     # G too large for shared memory
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
+    bad = list(args); bad[3] = ctypes.c_void_p(0x10004)   # misaligned global_start
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
+
+
 def test_select_rejects_small_workspace(lib):
     f = lib.lrmoe_select_quota
     need = L.lrmoe_select_workspace_bytes(64, 2, 4)
