@@ -106,7 +106,8 @@ def recorded_traffic(kernel: str, config: str):
     """DRAM bytes per launch of `kernel` from a committed ncu summary, or None.
 
     profiles/traffic.json maps "<kernel>@<config>" to {"bytes": B, "source_sha1": S};
-    the figure is dropped when the kernel's source changed since the capture.
+    the figure is dropped when the kernel's sources (GEMM_SOURCES) changed since the
+    capture.
     """
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
@@ -121,10 +122,14 @@ def recorded_traffic(kernel: str, config: str):
     return ent.get("bytes")
 
 
+# the sources that define the grouped-GEMM kernels whose traffic is recorded
+GEMM_SOURCES = ("gemm_tc.cu", "common.cuh", "grouped.cuh", "launch.h")
+
+
 def kernel_source_sha1() -> str:
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "pruned_expert_backward_lrmoe_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in GEMM_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -584,6 +589,44 @@ def run_gpu(args):
     if int(st.item()) != 0:
         raise SystemExit(f"device status {int(st.item())} after the router gradient")
 
+    # ---------------- redistribution over expert copies (one rank's view) ----------------
+    # An 8-GPU copy map: expert e at home on GPU e % 8, the 16 most loaded experts with
+    # a second copy three GPUs on.  The host planner's time and peak against an even
+    # split and against home-only placement; then this rank's rows cut by the plan.
+    G_plan = 8
+    m_np = out["kept"].cpu().numpy().astype(np.int64)
+    adm = np.zeros((s.E, G_plan), bool)
+    adm[np.arange(s.E), np.arange(s.E) % G_plan] = True
+    hot = np.argsort(-m_np, kind="stable")[:16]
+    adm[hot, (hot + 3) % G_plan] = True
+    t0 = time.perf_counter()
+    plan, peak = L.lrmoe_redistribute(m_np, adm)
+    planner_us = (time.perf_counter() - t0) * 1e6
+    home = np.bincount(np.arange(s.E) % G_plan, weights=m_np, minlength=G_plan)
+    plan_dev = torch.from_numpy(plan.astype(np.int32)).to(dev)
+    pd = torch.empty(s.P, dtype=torch.int32, device=dev)
+    do = torch.empty(G_plan + 1, dtype=torch.int32, device=dev)
+    deo = torch.empty(G_plan, s.E + 1, dtype=torch.int32, device=dev)
+    evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(20)]
+    for i in range(23):
+        flush_l2()
+        if i >= 3:
+            evp[i - 3][0].record(stream)
+        L.lrmoe_split_by_destination(out["perm"], out["offsets"], plan_dev, pd, do, deo,
+                                     status=st, stream=stream)
+        if i >= 3:
+            evp[i - 3][1].record(stream)
+    torch.cuda.synchronize(dev)
+    redistribution = {
+        "gpus_in_plan": G_plan, "copies": int(adm.sum()), "planner_us": planner_us,
+        "peak": int(peak), "even_split": int(-(-int(m_np.sum()) // G_plan)),
+        "home_only_peak": int(home.max()),
+        "split_us": 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp),
+    }
+    if int(st.item()) != 0:
+        raise SystemExit(f"device status {int(st.item())} after the destination split")
+
     # ---------------- end to end through host buffers ----------------
     pin = {k_: v.pin_memory() for k_, v in host.items()}
     dX_host = torch.empty(s.T, s.H, dtype=tdt).pin_memory()
@@ -635,6 +678,7 @@ def run_gpu(args):
         "quota_controller_equals_capacity_rule": controller_matches,
         "saved_norms": saved_norms,
         "router_grad": router,
+        "redistribution": redistribution,
         "breakdown_steps": n_bd,
         "breakdown_step_ms": sum(kern_ms.values()),
         "cpu_baseline": cpu,
