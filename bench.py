@@ -57,6 +57,9 @@ def parse_args(argv=None):
                    help="skip timing the CPU oracle (profiling runs)")
     p.add_argument("--sweep", action="store_true",
                    help="quota sweep (keep 1, 3/4, 1/2, 1/4) on the GLM-shaped T=16384 layer")
+    p.add_argument("--no-extras", action="store_true",
+                   help="time only the step (profiling runs): no controller, fused-GEMM, "
+                        "saved-norm, routing-gradient, redistribution or end-to-end blocks")
     p.add_argument("--override", default="",
                    help="layer fields to replace, e.g. T=4096,E=64 (smaller profiling cases)")
     return p.parse_args(argv)
@@ -89,7 +92,17 @@ def algorithmic(T, k, E, H, I, M, b):
     }
     fl = {"dgrad_swiglu": 2 * M * H * I, "wgrad_down": 2 * M * H * I, "wgrad_gu": 4 * M * I * H,
           "dgrad_x": 4 * M * I * H}
+    # fused launches: the shared gradient rows (DY_p, dGU_p) count once
+    by["dgrad_swiglu+wgrad_down"] = by["dgrad_swiglu"] + by["wgrad_down"] - M * H * b
+    by["dgrad_x+wgrad_gu"] = by["dgrad_x"] + by["wgrad_gu"] - 2 * M * I * b
+    fl["dgrad_swiglu+wgrad_down"] = fl["dgrad_swiglu"] + fl["wgrad_down"]
+    fl["dgrad_x+wgrad_gu"] = fl["dgrad_x"] + fl["wgrad_gu"]
     return by, fl
+
+
+def step_gemms(fl):
+    """The grouped-GEMM entries of KERNELS (the step's launches)."""
+    return [n for n in KERNELS if n in fl]
 
 
 def load_peaks():
@@ -369,7 +382,7 @@ def make_runner(layer, dev):
         flush.sum()
     st = out["status"]
 
-    def step(ev=None, a_sqnorm=None):
+    def step(ev=None, a_sqnorm=None, fused=False):
         """One pass of the path; with a_sqnorm (||a_p||^2 saved by the forward) the
         score reads dY and the saved norms instead of a."""
         score_call = (
@@ -377,7 +390,7 @@ def make_runner(layer, dev):
                                    out["score"], st, stream)) if a_sqnorm is None else
             (lambda: L.lrmoe_score_from_norms(inp["topk_idx"], inp["topk_w"], inp["dY"], a_sqnorm,
                                               s.E, out["score"], st, stream)))
-        calls = (
+        head = (
             score_call,
             lambda: L.lrmoe_select_quota(inp["topk_idx"], out["score"], inp["quota"], out["counts"],
                                          out["kept"], out["offsets"], out["perm"], out["pos"],
@@ -385,17 +398,32 @@ def make_runner(layer, dev):
             lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], inp["x"], inp["dY"],
                                  inp["a"], inp["g"], inp["u"], out["Xp"], out["DYp"], out["Ap"],
                                  out["Gp"], out["Up"], st, stream),
-            lambda: L.lrmoe_grouped_dgrad(out["DYp"], inp["W_down"], out["offsets"],
-                                          L.LRMOE_EPI_SWIGLU_BWD, out["dGUp"], Gp=out["Gp"],
-                                          Up=out["Up"], status=st, stream=stream),
-            lambda: L.lrmoe_grouped_wgrad(out["DYp"], out["Ap"], out["offsets"], out["dW_down"],
-                                          status=st, stream=stream),
-            lambda: L.lrmoe_grouped_wgrad(out["dGUp"], out["Xp"], out["offsets"], out["dW_gu"],
-                                          status=st, stream=stream),
-            lambda: L.lrmoe_grouped_dgrad(out["dGUp"], inp["W_gu"], out["offsets"],
-                                          L.LRMOE_EPI_STORE, out["dXp"], status=st, stream=stream),
-            lambda: L.lrmoe_unpack(out["dXp"], out["pos"], s.T, s.k, out["dX"], st, stream),
         )
+        if not fused:  # the four grouped GEMMs as separate launches
+            gemms = (
+                lambda: L.lrmoe_grouped_dgrad(out["DYp"], inp["W_down"], out["offsets"],
+                                              L.LRMOE_EPI_SWIGLU_BWD, out["dGUp"], Gp=out["Gp"],
+                                              Up=out["Up"], status=st, stream=stream),
+                lambda: L.lrmoe_grouped_wgrad(out["DYp"], out["Ap"], out["offsets"],
+                                              out["dW_down"], status=st, stream=stream),
+                lambda: L.lrmoe_grouped_wgrad(out["dGUp"], out["Xp"], out["offsets"],
+                                              out["dW_gu"], status=st, stream=stream),
+                lambda: L.lrmoe_grouped_dgrad(out["dGUp"], inp["W_gu"], out["offsets"],
+                                              L.LRMOE_EPI_STORE, out["dXp"], status=st,
+                                              stream=stream),
+            )
+        else:  # each dgrad with the wgrad over the same gradient rows in one launch
+            gemms = (
+                lambda: L.lrmoe_grouped_dgrad_wgrad(
+                    out["DYp"], inp["W_down"], out["offsets"], L.LRMOE_EPI_SWIGLU_BWD,
+                    out["dGUp"], out["Ap"], out["dW_down"], Gp=out["Gp"], Up=out["Up"],
+                    status=st, stream=stream),
+                lambda: L.lrmoe_grouped_dgrad_wgrad(
+                    out["dGUp"], inp["W_gu"], out["offsets"], L.LRMOE_EPI_STORE, out["dXp"],
+                    out["Xp"], out["dW_gu"], status=st, stream=stream),
+            )
+        calls = head + gemms + (
+            lambda: L.lrmoe_unpack(out["dXp"], out["pos"], s.T, s.k, out["dX"], st, stream),)
         for i, c in enumerate(calls):
             if ev is not None:
                 ev[i].record(stream)
@@ -467,8 +495,8 @@ def run_gpu(args):
     kern_ms = {kname: statistics.fmean(v) for kname, v in per_kernel.items()}
 
     by, fl = algorithmic(s.T, s.k, s.E, s.H, s.I, M, b)
-    gemm_ms = sum(kern_ms[n] for n in fl)
-    gemm_flops = sum(fl.values())
+    gemm_ms = sum(kern_ms[n] for n in step_gemms(fl))
+    gemm_flops = sum(fl[n] for n in step_gemms(fl))
     peaks, peak_src = load_peaks()
     dominant = max(kern_ms, key=kern_ms.get)
     dom_bytes = by[dominant]
@@ -489,168 +517,184 @@ def run_gpu(args):
                                                     FALLBACK_PEAKS["bf16_tflops_sustained"]))
         breakdown[kname] = e
 
-    # ---------------- quota controller (runs before the backward; not in the step) ----------------
-    q_dev = torch.empty(s.E, dtype=torch.int32, device=dev)
-    c_dev = torch.empty(s.E, dtype=torch.int32, device=dev)
-    cap = (s.T * s.k) // s.E
-    ctl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(20)]
-    for i in range(23):
-        if i >= 3:
-            ctl_ev[i - 3][0].record(stream)
-        L.lrmoe_quota_controller(inp["topk_idx"], s.E, cap, -1, q_dev, c_dev, st, stream)
-        if i >= 3:
-            ctl_ev[i - 3][1].record(stream)
-    torch.cuda.synchronize(dev)
-    controller_us = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in ctl_ev)
-    controller_matches = bool(torch.equal(q_dev, inp["quota"])) if s.quota == "capacity" else None
+    controller_us = controller_matches = fused_step_ms = None
+    saved_norms = router = redistribution = None
+    e2e_value = e2e_ms = None
+    h2d = d2h = 0
+    if not args.no_extras:
+        # ---------------- quota controller (runs before the backward; not in the step) ----------------
+        q_dev = torch.empty(s.E, dtype=torch.int32, device=dev)
+        c_dev = torch.empty(s.E, dtype=torch.int32, device=dev)
+        cap = (s.T * s.k) // s.E
+        ctl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(20)]
+        for i in range(23):
+            if i >= 3:
+                ctl_ev[i - 3][0].record(stream)
+            L.lrmoe_quota_controller(inp["topk_idx"], s.E, cap, -1, q_dev, c_dev, st, stream)
+            if i >= 3:
+                ctl_ev[i - 3][1].record(stream)
+        torch.cuda.synchronize(dev)
+        controller_us = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in ctl_ev)
+        controller_matches = bool(torch.equal(q_dev, inp["quota"])) if s.quota == "capacity" else None
 
-    # ---------------- score from forward-saved ||a_p||^2 ----------------
-    # The forward can save ||a_p||^2 when it writes a; the backward's score then
-    # reads dY and 4 bytes per pair.  Timed per call after an L2 flush, and as
-    # whole steps with that score in place of the full one.
-    a2d = inp["a"].view(s.P, s.I)
-    na = torch.empty(s.P, dtype=torch.float32, device=dev)
-    L.lrmoe_row_sqnorm(a2d, na, stream)
-    sn_calls = {
-        "row_sqnorm": lambda: L.lrmoe_row_sqnorm(a2d, na, stream),
-        "score_from_norms": lambda: L.lrmoe_score_from_norms(
-            inp["topk_idx"], inp["topk_w"], inp["dY"], na, s.E, out["score"], st, stream),
-        "score": lambda: L.lrmoe_score(inp["topk_idx"], inp["topk_w"], inp["dY"], inp["a"], s.E,
-                                       out["score"], st, stream),
-    }
-    sn_us = {}
-    for name_, fn in sn_calls.items():
+        # ---------------- score from forward-saved ||a_p||^2 ----------------
+        # The forward can save ||a_p||^2 when it writes a; the backward's score then
+        # reads dY and 4 bytes per pair.  Timed per call after an L2 flush, and as
+        # whole steps with that score in place of the full one.
+        a2d = inp["a"].view(s.P, s.I)
+        na = torch.empty(s.P, dtype=torch.float32, device=dev)
+        L.lrmoe_row_sqnorm(a2d, na, stream)
+        sn_calls = {
+            "row_sqnorm": lambda: L.lrmoe_row_sqnorm(a2d, na, stream),
+            "score_from_norms": lambda: L.lrmoe_score_from_norms(
+                inp["topk_idx"], inp["topk_w"], inp["dY"], na, s.E, out["score"], st, stream),
+            "score": lambda: L.lrmoe_score(inp["topk_idx"], inp["topk_w"], inp["dY"], inp["a"], s.E,
+                                           out["score"], st, stream),
+        }
+        sn_us = {}
+        for name_, fn in sn_calls.items():
+            evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(20)]
+            for i in range(23):
+                flush_l2()
+                if i >= 3:
+                    evp[i - 3][0].record(stream)
+                fn()
+                if i >= 3:
+                    evp[i - 3][1].record(stream)
+            torch.cuda.synchronize(dev)
+            sn_us[name_] = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp)
+        sn_steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(n_bd)]
+        for i in range(n_bd):
+            flush_l2()
+            sn_steps[i][0].record(stream)
+            step(a_sqnorm=na)
+            sn_steps[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        sn_step_ms = max_over_ranks(statistics.fmean(a_.elapsed_time(b_) for a_, b_ in sn_steps), dist)
+        sn_bytes = s.T * s.H * b + 16 * s.P          # dY, idx, w, saved norm, score
+        # the same steps with each dgrad and its wgrad fused into one launch
+        fu_steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(n_bd)]
+        for i in range(n_bd):
+            flush_l2()
+            fu_steps[i][0].record(stream)
+            step(fused=True)
+            fu_steps[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        fused_step_ms = max_over_ranks(
+            statistics.fmean(a_.elapsed_time(b_) for a_, b_ in fu_steps), dist)
+        saved_norms = {
+            "row_sqnorm_us": sn_us["row_sqnorm"], "score_from_norms_us": sn_us["score_from_norms"],
+            "score_us": sn_us["score"],
+            "score_from_norms_GB/s": sn_bytes / (sn_us["score_from_norms"] * 1e-6) / 1e9,
+            "score_from_norms_hbm_frac": sn_bytes / (sn_us["score_from_norms"] * 1e-6) / 1e9
+            / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+            "step_ms": sn_step_ms, "value": M_all / (sn_step_ms * 1e-3), "unit": UNIT,
+            "steps": n_bd,
+        }
+        if int(st.item()) != 0:
+            raise SystemExit(f"device status {int(st.item())} after the saved-norm steps")
+
+        # ---------------- routing-weight gradient from saved expert outputs ----------------
+        # y_p = W_down[e] a_p is what the forward saves; it is generated here with torch
+        # (input generation, not part of the path), then dw = <dY_t, y_p> is timed for
+        # the retained pairs (pos from the selection) and for every routed pair.
+        y_dev = torch.empty(s.P, s.H, dtype=tdt, device=dev)
+        flat_idx = inp["topk_idx"].view(-1)
+        for e in range(s.E):
+            sel = (flat_idx == e).nonzero().squeeze(1)
+            if sel.numel():
+                y_dev[sel] = a2d[sel] @ inp["W_down"][e].T
+        dw = torch.empty(s.P, dtype=torch.float32, device=dev)
+        router = {}
+        for mode, pos_arg, nbytes in (
+                ("retained", out["pos"], M * s.H * b + s.T * s.H * b + 12 * s.P),
+                ("all", None, s.P * s.H * b + s.T * s.H * b + 8 * s.P)):
+            evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(20)]
+            for i in range(23):
+                flush_l2()
+                if i >= 3:
+                    evp[i - 3][0].record(stream)
+                L.lrmoe_router_grad(inp["topk_idx"], inp["dY"], y_dev, s.E, dw, pos=pos_arg,
+                                    status=st, stream=stream)
+                if i >= 3:
+                    evp[i - 3][1].record(stream)
+            torch.cuda.synchronize(dev)
+            us = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp)
+            gbs = nbytes / (us * 1e-6) / 1e9
+            router[mode] = {"us": us, "GB/s": gbs,
+                            "hbm_frac": gbs / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+                            "algorithmic_bytes": nbytes}
+        del y_dev
+        if int(st.item()) != 0:
+            raise SystemExit(f"device status {int(st.item())} after the router gradient")
+
+        # ---------------- redistribution over expert copies (one rank's view) ----------------
+        # An 8-GPU copy map: expert e at home on GPU e % 8, the 16 most loaded experts with
+        # a second copy three GPUs on.  The host planner's time and peak against an even
+        # split and against home-only placement; then this rank's rows cut by the plan.
+        G_plan = 8
+        m_np = out["kept"].cpu().numpy().astype(np.int64)
+        adm = np.zeros((s.E, G_plan), bool)
+        adm[np.arange(s.E), np.arange(s.E) % G_plan] = True
+        hot = np.argsort(-m_np, kind="stable")[:16]
+        adm[hot, (hot + 3) % G_plan] = True
+        t0 = time.perf_counter()
+        plan, peak = L.lrmoe_redistribute(m_np, adm)
+        planner_us = (time.perf_counter() - t0) * 1e6
+        home = np.bincount(np.arange(s.E) % G_plan, weights=m_np, minlength=G_plan)
+        plan_dev = torch.from_numpy(plan.astype(np.int32)).to(dev)
+        pd = torch.empty(s.P, dtype=torch.int32, device=dev)
+        do = torch.empty(G_plan + 1, dtype=torch.int32, device=dev)
+        deo = torch.empty(G_plan, s.E + 1, dtype=torch.int32, device=dev)
         evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(20)]
         for i in range(23):
             flush_l2()
             if i >= 3:
                 evp[i - 3][0].record(stream)
-            fn()
+            L.lrmoe_split_by_destination(out["perm"], out["offsets"], plan_dev, pd, do, deo,
+                                         status=st, stream=stream)
             if i >= 3:
                 evp[i - 3][1].record(stream)
         torch.cuda.synchronize(dev)
-        sn_us[name_] = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp)
-    sn_steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(n_bd)]
-    for i in range(n_bd):
-        flush_l2()
-        sn_steps[i][0].record(stream)
-        step(a_sqnorm=na)
-        sn_steps[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    sn_step_ms = max_over_ranks(statistics.fmean(a_.elapsed_time(b_) for a_, b_ in sn_steps), dist)
-    sn_bytes = s.T * s.H * b + 16 * s.P          # dY, idx, w, saved norm, score
-    saved_norms = {
-        "row_sqnorm_us": sn_us["row_sqnorm"], "score_from_norms_us": sn_us["score_from_norms"],
-        "score_us": sn_us["score"],
-        "score_from_norms_GB/s": sn_bytes / (sn_us["score_from_norms"] * 1e-6) / 1e9,
-        "score_from_norms_hbm_frac": sn_bytes / (sn_us["score_from_norms"] * 1e-6) / 1e9
-        / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
-        "step_ms": sn_step_ms, "value": M_all / (sn_step_ms * 1e-3), "unit": UNIT,
-        "steps": n_bd,
-    }
-    if int(st.item()) != 0:
-        raise SystemExit(f"device status {int(st.item())} after the saved-norm steps")
+        redistribution = {
+            "gpus_in_plan": G_plan, "copies": int(adm.sum()), "planner_us": planner_us,
+            "peak": int(peak), "even_split": int(-(-int(m_np.sum()) // G_plan)),
+            "home_only_peak": int(home.max()),
+            "split_us": 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp),
+        }
+        if int(st.item()) != 0:
+            raise SystemExit(f"device status {int(st.item())} after the destination split")
 
-    # ---------------- routing-weight gradient from saved expert outputs ----------------
-    # y_p = W_down[e] a_p is what the forward saves; it is generated here with torch
-    # (input generation, not part of the path), then dw = <dY_t, y_p> is timed for
-    # the retained pairs (pos from the selection) and for every routed pair.
-    y_dev = torch.empty(s.P, s.H, dtype=tdt, device=dev)
-    flat_idx = inp["topk_idx"].view(-1)
-    for e in range(s.E):
-        sel = (flat_idx == e).nonzero().squeeze(1)
-        if sel.numel():
-            y_dev[sel] = a2d[sel] @ inp["W_down"][e].T
-    dw = torch.empty(s.P, dtype=torch.float32, device=dev)
-    router = {}
-    for mode, pos_arg, nbytes in (
-            ("retained", out["pos"], M * s.H * b + s.T * s.H * b + 12 * s.P),
-            ("all", None, s.P * s.H * b + s.T * s.H * b + 8 * s.P)):
-        evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(20)]
-        for i in range(23):
+        # ---------------- end to end through host buffers ----------------
+        pin = {k_: v.pin_memory() for k_, v in host.items()}
+        dX_host = torch.empty(s.T, s.H, dtype=tdt).pin_memory()
+        st_host = torch.empty(1, dtype=torch.int32).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in pin.values())
+        d2h = dX_host.numel() * dX_host.element_size() + 4
+        n_e2e = max(3, min(args.steps, 50))
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(n_e2e)]
+        for i in range(n_e2e + 2):
+            timed = i >= 2
             flush_l2()
-            if i >= 3:
-                evp[i - 3][0].record(stream)
-            L.lrmoe_router_grad(inp["topk_idx"], inp["dY"], y_dev, s.E, dw, pos=pos_arg,
-                                status=st, stream=stream)
-            if i >= 3:
-                evp[i - 3][1].record(stream)
+            if timed:
+                e2e_ev[i - 2][0].record(stream)
+            for k_, v in pin.items():
+                inp[k_].copy_(v, non_blocking=True)
+            L.lrmoe_pruned_backward(inp, out, stream)
+            dX_host.copy_(out["dX"], non_blocking=True)
+            st_host.copy_(out["status"], non_blocking=True)
+            if timed:
+                e2e_ev[i - 2][1].record(stream)
         torch.cuda.synchronize(dev)
-        us = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp)
-        gbs = nbytes / (us * 1e-6) / 1e9
-        router[mode] = {"us": us, "GB/s": gbs,
-                        "hbm_frac": gbs / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
-                        "algorithmic_bytes": nbytes}
-    del y_dev
-    if int(st.item()) != 0:
-        raise SystemExit(f"device status {int(st.item())} after the router gradient")
-
-    # ---------------- redistribution over expert copies (one rank's view) ----------------
-    # An 8-GPU copy map: expert e at home on GPU e % 8, the 16 most loaded experts with
-    # a second copy three GPUs on.  The host planner's time and peak against an even
-    # split and against home-only placement; then this rank's rows cut by the plan.
-    G_plan = 8
-    m_np = out["kept"].cpu().numpy().astype(np.int64)
-    adm = np.zeros((s.E, G_plan), bool)
-    adm[np.arange(s.E), np.arange(s.E) % G_plan] = True
-    hot = np.argsort(-m_np, kind="stable")[:16]
-    adm[hot, (hot + 3) % G_plan] = True
-    t0 = time.perf_counter()
-    plan, peak = L.lrmoe_redistribute(m_np, adm)
-    planner_us = (time.perf_counter() - t0) * 1e6
-    home = np.bincount(np.arange(s.E) % G_plan, weights=m_np, minlength=G_plan)
-    plan_dev = torch.from_numpy(plan.astype(np.int32)).to(dev)
-    pd = torch.empty(s.P, dtype=torch.int32, device=dev)
-    do = torch.empty(G_plan + 1, dtype=torch.int32, device=dev)
-    deo = torch.empty(G_plan, s.E + 1, dtype=torch.int32, device=dev)
-    evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(20)]
-    for i in range(23):
-        flush_l2()
-        if i >= 3:
-            evp[i - 3][0].record(stream)
-        L.lrmoe_split_by_destination(out["perm"], out["offsets"], plan_dev, pd, do, deo,
-                                     status=st, stream=stream)
-        if i >= 3:
-            evp[i - 3][1].record(stream)
-    torch.cuda.synchronize(dev)
-    redistribution = {
-        "gpus_in_plan": G_plan, "copies": int(adm.sum()), "planner_us": planner_us,
-        "peak": int(peak), "even_split": int(-(-int(m_np.sum()) // G_plan)),
-        "home_only_peak": int(home.max()),
-        "split_us": 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp),
-    }
-    if int(st.item()) != 0:
-        raise SystemExit(f"device status {int(st.item())} after the destination split")
-
-    # ---------------- end to end through host buffers ----------------
-    pin = {k_: v.pin_memory() for k_, v in host.items()}
-    dX_host = torch.empty(s.T, s.H, dtype=tdt).pin_memory()
-    st_host = torch.empty(1, dtype=torch.int32).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in pin.values())
-    d2h = dX_host.numel() * dX_host.element_size() + 4
-    n_e2e = max(3, min(args.steps, 50))
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(n_e2e)]
-    for i in range(n_e2e + 2):
-        timed = i >= 2
-        flush_l2()
-        if timed:
-            e2e_ev[i - 2][0].record(stream)
-        for k_, v in pin.items():
-            inp[k_].copy_(v, non_blocking=True)
-        L.lrmoe_pruned_backward(inp, out, stream)
-        dX_host.copy_(out["dX"], non_blocking=True)
-        st_host.copy_(out["status"], non_blocking=True)
-        if timed:
-            e2e_ev[i - 2][1].record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = statistics.fmean(a_.elapsed_time(b_) for a_, b_ in e2e_ev)
-    e2e_value = M_all / (max_over_ranks(e2e_ms, dist) * 1e-3)
+        e2e_ms = statistics.fmean(a_.elapsed_time(b_) for a_, b_ in e2e_ev)
+        e2e_value = M_all / (max_over_ranks(e2e_ms, dist) * 1e-3)
 
     # ---------------- CPU baseline (rank 0 at N = 1) ----------------
     cpu = None
@@ -676,6 +720,7 @@ def run_gpu(args):
         "breakdown": breakdown,
         "quota_controller_us": controller_us,
         "quota_controller_equals_capacity_rule": controller_matches,
+        "fused_gemm_step_ms": fused_step_ms,
         "saved_norms": saved_norms,
         "router_grad": router,
         "redistribution": redistribution,
@@ -732,16 +777,17 @@ def run_sweep(args):
                 for j, kn in enumerate(KERNELS)}
         step_ms = statistics.fmean(ev[0].elapsed_time(ev[-1]) for ev in evs)
         by, fl = algorithmic(s.T, s.k, s.E, s.H, s.I, M, 2)
-        gemm_ms = sum(kern[kn] for kn in fl)
-        tf = sum(fl.values()) / (gemm_ms * 1e-3) / 1e12
-        gemm_bytes = sum(by[kn] for kn in fl)
+        gemm_ms = sum(kern[kn] for kn in step_gemms(fl))
+        gemm_fl = sum(fl[kn] for kn in step_gemms(fl))
+        tf = gemm_fl / (gemm_ms * 1e-3) / 1e12
+        gemm_bytes = sum(by[kn] for kn in step_gemms(fl))
         points.append((M, step_ms))
         print(json.dumps({
             "sweep_keep": f"{n}/4", "retained_pairs": M, "routed_pairs": s.P,
             "ms_per_step": step_ms, "value": M / (step_ms * 1e-3), "unit": UNIT,
             "gemm_ms": gemm_ms, "gemm_tflops": tf, "gemm_tensor_frac": tf / tf_peak,
             "gemm_hbm_frac": gemm_bytes / (gemm_ms * 1e-3) / 1e9 / hbm_peak,
-            "gemm_flop_per_byte": sum(fl.values()) / gemm_bytes,
+            "gemm_flop_per_byte": gemm_fl / gemm_bytes,
             "peaks": f"{peak_src}: bf16 {tf_peak} TFLOP/s sustained, HBM {hbm_peak} GB/s",
             "kernels_ms": kern, "clocks": clk.summary(), "steps": args.steps,
             "config": config_block(s, 1)}), flush=True)

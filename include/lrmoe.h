@@ -324,6 +324,25 @@ int lrmoe_grouped_wgrad(const void* grad_rows, const void* in_rows, int rows_cap
                         float* dW, int accumulate, uint32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * a4, two GEMMs that share their gradient rows in one launch (same passages).
+ * Exactly lrmoe_grouped_dgrad(grad_rows, rows_cap, W, offsets, E, K, N, dt,
+ * epi, Gp, Up, out) plus lrmoe_grouped_wgrad(grad_rows, in_rows, rows_cap,
+ * offsets, E, N1 = K, N2, dt, dW, accumulate) in one persistent launch whose
+ * tile queue interleaves the two kinds evenly (dgrad reads W, wgrad writes dW).
+ * lrmoe_pruned_backward does not use it: on a B200 the two separate launches
+ * are faster for the shapes measured.  The two pairs of the path are:
+ *   (DYp; W_down, SWIGLU -> dGUp; Ap -> dW_down)   K = H, N = I, N2 = I
+ *   (dGUp; W_gu, STORE -> dXp;  Xp -> dW_gu)       K = 2I, N = H, N2 = H
+ * Layouts, outputs and errors as the two calls.  bf16 only (fp32 returns
+ * LRMOE_ERR_UNSUPPORTED: use the two calls).
+ * ------------------------------------------------------------------------- */
+int lrmoe_grouped_dgrad_wgrad(const void* grad_rows, int rows_cap, const void* W,
+                              const int32_t* offsets, int E, int K, int N, lrmoe_dtype dt,
+                              lrmoe_epilogue epi, const void* Gp, const void* Up, void* out,
+                              const void* in_rows, int N2, float* dW, int accumulate,
+                              uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * a5  Back to the original layout.  RU-B bullet 5, last sentence; FR-B
  * bullet 5, last sentence.
  *

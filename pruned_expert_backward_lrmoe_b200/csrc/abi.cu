@@ -351,6 +351,38 @@ int lrmoe_grouped_wgrad(const void* grad_rows, const void* in_rows, int rows_cap
   return LRMOE_OK;
 }
 
+int lrmoe_grouped_dgrad_wgrad(const void* grad_rows, int rows_cap, const void* W,
+                              const int32_t* offsets, int E, int K, int N, lrmoe_dtype dt,
+                              lrmoe_epilogue epi, const void* Gp, const void* Up, void* out,
+                              const void* in_rows, int N2, float* dW, int accumulate,
+                              uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  if (dt != LRMOE_BF16)
+    return fail(LRMOE_ERR_UNSUPPORTED, "the fused launch is bf16 only; use the two calls");
+  REQUIRE(epi == LRMOE_EPI_STORE || epi == LRMOE_EPI_SWIGLU_BWD, "unknown epilogue %d", (int)epi);
+  REQUIRE(E > 0 && rows_cap > 0, "E and rows_cap must be positive");
+  if (E > kMaxGroupedExperts) return fail(LRMOE_ERR_UNSUPPORTED, "E=%d > %d", E, kMaxGroupedExperts);
+  if (int r = check_feature(K, dt, "K")) return r;
+  if (int r = check_feature(N, dt, "N")) return r;
+  if (int r = check_feature(N2, dt, "N2")) return r;
+  REQUIRE_PTR(grad_rows);
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(out);
+  REQUIRE_PTR(in_rows);
+  REQUIRE_PTR(dW);
+  if (epi == LRMOE_EPI_SWIGLU_BWD) {
+    REQUIRE_PTR(Gp);
+    REQUIRE_PTR(Up);
+  }
+  const char* why = "launch failed";
+  cudaError_t e = launch_dgrad_wgrad_tc(grad_rows, rows_cap, W, offsets, E, K, N, epi, Gp, Up, out,
+                                        in_rows, N2, dW, accumulate, status,
+                                        static_cast<cudaStream_t>(stream), &why);
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, why);
+}
+
 int lrmoe_unpack(const void* dXp, int rows_cap, const int32_t* pos, int T, int k, int H,
                  lrmoe_dtype dt, void* dX, uint32_t* status, void* stream) {
   g_last_error[0] = 0;

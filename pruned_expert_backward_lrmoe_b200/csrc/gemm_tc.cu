@@ -36,7 +36,10 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;  // TMA warp, MMA warp, 8 epilogue warps
 constexpr int kEpiThreads = 32 * kEpiWarps;
 
-enum Mode : int { kDgradStore = 0, kDgradSwiglu = 1, kWgrad = 2 };
+// kFused*: one launch runs a dgrad (store or SwiGLU epilogue) and a wgrad that
+// share their packed gradient rows.
+enum Mode : int { kDgradStore = 0, kDgradSwiglu = 1, kWgrad = 2, kFusedStore = 3, kFusedSwiglu = 4 };
+constexpr int kBNT = 256;  // tile N (TMEM columns per accumulator)
 
 // Dynamic tile scheduling.  Each CTA's producer takes the next tile index from a
 // global counter and hands it to the MMA and epilogue warps through a ring of
@@ -72,7 +75,31 @@ struct Layout {
 };
 constexpr int kSmemLimit = 232448;  // per-block dynamic shared memory on sm_100
 
+// Scalars of one launch.  dgrad: out_d[R_e] = rows[R_e] . W[e] (K x Nd); wgrad:
+// dW[e] = grad[R_e]^T . in[R_e] (N1 x N2, fp32).  A fused launch runs both over
+// the same packed gradient rows (dgrad K = wgrad N1).
+struct GemmParams {
+  const int32_t* offsets;
+  int E;
+  int Kd, Nd;           // dgrad
+  int N1, N2;           // wgrad
+  const uint16_t* Gp;   // SwiGLU epilogue: saved g, u [rows][Nd]
+  const uint16_t* Up;
+  void* out_d;          // dgrad output [rows][Nd] (SwiGLU: [rows][2 Nd])
+  int accumulate;       // wgrad: add into dW
+  uint32_t* status;
+  int sched_slot;
+};
+
+template <int MODE>
+struct Traits {
+  static constexpr bool kHasD = MODE != kWgrad;
+  static constexpr bool kHasW = MODE == kWgrad || MODE == kFusedStore || MODE == kFusedSwiglu;
+  static constexpr bool kSwiglu = MODE == kDgradSwiglu || MODE == kFusedSwiglu;
+};
+
 struct TileInfo {
+  int kind;    // 0: dgrad tile, 1: wgrad tile
   int e;       // expert
   int row0;    // dgrad: first packed row of the tile; wgrad: first packed row of the expert
   int row_end; // end of the expert's rows
@@ -80,29 +107,50 @@ struct TileInfo {
   int nk;      // number of K blocks
 };
 
-template <int MODE, int BN>
-__device__ __forceinline__ TileInfo decode_tile(int t, const int32_t* __restrict__ offsets,
-                                                const int* tab0, int E, int K, int n_tiles,
-                                                int m_tiles) {
+// Tile counts of a launch: dgrad (variable M) and wgrad (fixed per expert).
+struct TileCounts {
+  int td, tw, total;
+  int nt_d;        // dgrad N tiles
+  int mt_w, nt_w;  // wgrad M and N tiles
+};
+
+// Tile t of the launch.  A fused launch spreads its td dgrad tiles evenly over
+// the tw wgrad tiles (position t is a dgrad tile when floor((t+1) td / T) steps),
+// so that every SM alternates the read-bound and the write-bound kind.
+template <int MODE>
+__device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, const int* offs,
+                                                const int* tab_d, const int* tab_w,
+                                                const TileCounts& tc) {
+  using Tr = Traits<MODE>;
   TileInfo ti;
-  if constexpr (MODE == kWgrad) {
-    const int per_e = m_tiles * n_tiles;
-    const int oi = t / per_e, local = t - oi * per_e;
-    ti.e = tab0[oi];
-    ti.m0 = (local / n_tiles) * BM;
-    ti.n0 = (local % n_tiles) * BN;
-    ti.row0 = offsets[ti.e];
-    ti.row_end = offsets[ti.e + 1];
+  int idx;
+  if constexpr (Tr::kHasD && Tr::kHasW) {
+    const long long before = (long long)t * tc.td / tc.total;
+    const long long upto = ((long long)t + 1) * tc.td / tc.total;
+    ti.kind = upto > before ? 0 : 1;
+    idx = ti.kind == 0 ? (int)before : t - (int)upto;
+  } else {
+    ti.kind = Tr::kHasW ? 1 : 0;
+    idx = t;
+  }
+  if (ti.kind == 1) {
+    const int per_e = tc.mt_w * tc.nt_w;
+    const int oi = idx / per_e, local = idx - oi * per_e;
+    ti.e = tab_w[oi];
+    ti.m0 = (local / tc.nt_w) * BM;
+    ti.n0 = (local % tc.nt_w) * kBNT;
+    ti.row0 = offs[ti.e];
+    ti.row_end = offs[ti.e + 1];
     ti.nk = (ti.row_end - ti.row0 + BK - 1) / BK;
   } else {
-    const int e = find_group(tab0, E, t);
-    const int local = t - tab0[e];
+    const int e = find_group(tab_d, p.E, idx);
+    const int local = idx - tab_d[e];
     ti.e = e;
     ti.m0 = 0;
-    ti.n0 = (local % n_tiles) * BN;
-    ti.row0 = offsets[e] + (local / n_tiles) * BM;
-    ti.row_end = offsets[e + 1];
-    ti.nk = (K + BK - 1) / BK;
+    ti.n0 = (local % tc.nt_d) * kBNT;
+    ti.row0 = offs[e] + (local / tc.nt_d) * BM;
+    ti.row_end = offs[e + 1];
+    ti.nk = (p.Kd + BK - 1) / BK;
   }
   return ti;
 }
@@ -178,14 +226,20 @@ __device__ __forceinline__ void epi_swiglu(const uint32_t (&r)[32], const uint4 
   }
 }
 
-template <int MODE, int BN, int STAGES, int OUTBUFS>
+// STAGES = ring depth; OUTBUFS = fp32 staging buffers per epilogue warp (wgrad).
+template <int MODE, int STAGES, int OUTBUFS>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
-    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-    const __grid_constant__ CUtensorMap tmOut /* wgrad: dW [E][N1][N2] fp32 */,
-    const int32_t* __restrict__ offsets, int E, int K, int N /* dgrad N or wgrad N2 */,
-    int N1 /* wgrad only */, const uint16_t* __restrict__ Gp, const uint16_t* __restrict__ Up,
-    void* __restrict__ out, int accumulate, uint32_t* __restrict__ status, int sched_slot) {
+    const __grid_constant__ CUtensorMap tmAd /* dgrad rows, K-major boxes */,
+    const __grid_constant__ CUtensorMap tmBd /* dgrad W [E][K][N] */,
+    const __grid_constant__ CUtensorMap tmAw /* wgrad grad rows, MN-major boxes */,
+    const __grid_constant__ CUtensorMap tmBw /* wgrad in rows */,
+    const __grid_constant__ CUtensorMap tmOut /* wgrad dW [E][N1][N2] fp32 */,
+    const GemmParams p) {
+  using Tr = Traits<MODE>;
+  constexpr int BN = kBNT;
   using L = Layout<BN, STAGES, OUTBUFS>;
+  const int E = p.E;
+  uint32_t* status = p.status;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -200,11 +254,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   volatile int* ring = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 16);  // [kRing]
-  unsigned int* sched = g_sched[sched_slot];
-  int* tab0 = reinterpret_cast<int*>(smem + L::kTableOff);
-  int* tab1 = tab0 + (E + 1);
-  int* scratch = tab1 + (E + 1);
-  int* offs_s = scratch + 33;  // offsets[0..E] in shared memory (read once per CTA)
+  unsigned int* sched = g_sched[p.sched_slot];
+  // tables: wgrad expert order [E+1]; dgrad tile starts [E+1] (first used as the
+  // wgrad build's size scratch); scan scratch [33]; offsets[0..E]
+  int* tab_w = reinterpret_cast<int*>(smem + L::kTableOff);
+  int* tab_d = tab_w + (E + 1);
+  int* scratch = tab_d + (E + 1);
+  int* offs_s = scratch + 33;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -226,8 +282,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    if constexpr (Tr::kHasD) {
+      tma_prefetch_desc(&tmAd);
+      tma_prefetch_desc(&tmBd);
+    }
+    if constexpr (Tr::kHasW) {
+      tma_prefetch_desc(&tmAw);
+      tma_prefetch_desc(&tmBw);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 2 * BN);
@@ -236,17 +298,20 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   // everything above touches no global memory; from here on, earlier kernels' outputs
   pdl_wait();
   pdl_trigger();
-  // tile table
-  const int n_tiles = (N + BN - 1) / BN;
-  int m_tiles = 0, total;
-  if constexpr (MODE == kWgrad) {
-    m_tiles = (N1 + BM - 1) / BM;
-    build_wgrad_order(offsets, E, tab0, tab1);
-    total = E * m_tiles * n_tiles;
-  } else {
-    total = build_dgrad_tiles(offsets, E, BM, n_tiles, tab0, scratch);
+  // tile tables
+  TileCounts tc{0, 0, 0, 0, 0, 0};
+  if constexpr (Tr::kHasW) {
+    tc.mt_w = (p.N1 + BM - 1) / BM;
+    tc.nt_w = (p.N2 + BN - 1) / BN;
+    build_wgrad_order(p.offsets, E, tab_w, tab_d);
+    tc.tw = E * tc.mt_w * tc.nt_w;
   }
-  for (int i = threadIdx.x; i <= E; i += blockDim.x) offs_s[i] = offsets[i];
+  if constexpr (Tr::kHasD) {
+    tc.nt_d = (p.Nd + BN - 1) / BN;
+    tc.td = build_dgrad_tiles(p.offsets, E, BM, tc.nt_d, tab_d, scratch);
+  }
+  tc.total = tc.td + tc.tw;
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) offs_s[i] = p.offsets[i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -274,12 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         int t = (int)next;
         if (!mbar_wait_bounded(&ring_empty[slot], ((uint32_t)(it / kRing) & 1u) ^ 1u, abort_flag,
                                status) ||
-            t >= total || *abort_flag)
+            t >= tc.total || *abort_flag)
           t = -1;
         ring[slot] = t;
         mbar_arrive(&ring_full[slot]);
         if (t < 0) break;
-        const TileInfo ti = decode_tile<MODE, BN>(t, offs_s, tab0, E, K, n_tiles, m_tiles);
+        const TileInfo ti = decode_tile<MODE>(t, p, offs_s, tab_d, tab_w, tc);
         if (ti.nk == 0) next = atomicAdd(&sched[0], 1u);
         for (int kb = 0; kb < ti.nk; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status)) break;
@@ -289,18 +354,22 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
           uint8_t* sa = smem + stage * L::kStageBytes;
           uint8_t* sb = sa + L::kABytes;
           mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
-          if constexpr (MODE == kWgrad) {
-            const int r = ti.row0 + kb * BK;
-            tma_load_2d(sa, &tmA, &full[stage], ti.m0, r);
-            tma_load_2d(sa + 8192, &tmA, &full[stage], ti.m0 + 64, r);
+          if (ti.kind == 1) {
+            if constexpr (Tr::kHasW) {
+              const int r = ti.row0 + kb * BK;
+              tma_load_2d(sa, &tmAw, &full[stage], ti.m0, r);
+              tma_load_2d(sa + 8192, &tmAw, &full[stage], ti.m0 + 64, r);
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              tma_load_2d(sb + c * 8192, &tmB, &full[stage], ti.n0 + c * 64, r);
+              for (int c = 0; c < BN / 64; ++c)
+                tma_load_2d(sb + c * 8192, &tmBw, &full[stage], ti.n0 + c * 64, r);
+            }
           } else {
-            tma_load_2d(sa, &tmA, &full[stage], kb * BK, ti.row0);
+            if constexpr (Tr::kHasD) {
+              tma_load_2d(sa, &tmAd, &full[stage], kb * BK, ti.row0);
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              tma_load_3d(sb + c * 8192, &tmB, &full[stage], ti.n0 + c * 64, kb * BK, ti.e);
+              for (int c = 0; c < BN / 64; ++c)
+                tma_load_3d(sb + c * 8192, &tmBd, &full[stage], ti.n0 + c * 64, kb * BK, ti.e);
+            }
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -311,15 +380,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, MODE == kWgrad, true);
+    constexpr uint32_t idesc_d = idesc_bf16_f32(BM, BN, false, true);  // A K-major
+    constexpr uint32_t idesc_w = idesc_bf16_f32(BM, BN, true, true);   // A MN-major
     int stage = 0;
     uint32_t phase = 0;
     uint32_t acc_iter = 0;
     for (int it = 0;; ++it) {
       const int t = next_tile(it);
       if (t < 0) break;
-      const TileInfo ti = decode_tile<MODE, BN>(t, offs_s, tab0, E, K, n_tiles, m_tiles);
+      const TileInfo ti = decode_tile<MODE>(t, p, offs_s, tab_d, tab_w, tc);
       if (ti.nk == 0) continue;
+      const bool wg = ti.kind == 1;
       const uint32_t b = acc_iter & 1u, bphase = (acc_iter >> 1) & 1u;
       if (!__all_sync(kFull, mbar_wait_bounded(&tempty[b], bphase ^ 1u, abort_flag, status)))
         break;
@@ -335,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         uint8_t* sa = smem + stage * L::kStageBytes;
         uint8_t* sb = sa + L::kABytes;
         int nkk = BK / UK;  // MMAs of this K block
-        if constexpr (MODE == kWgrad) {
+        if (Tr::kHasW && wg) {
           const int valid = ti.row_end - (ti.row0 + kb * BK);
           if (valid < BK) {
             // Last K block of the expert: only the 16-row groups that hold valid rows
@@ -363,13 +434,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk) {
             if (kk >= nkk) break;
-            uint64_t adesc, bdesc;
-            if constexpr (MODE == kWgrad)
-              adesc = smem_desc_sw128(a_addr + kk * 2048, 8192, 1024);
-            else
-              adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-            bdesc = smem_desc_sw128(b_addr + kk * 2048, 8192, 1024);
-            tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t adesc = wg ? smem_desc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                      : smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, 8192, 1024);
+            tc_mma_f16(d_tmem, adesc, bdesc, wg ? idesc_w : idesc_d, (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
         }
@@ -400,16 +468,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     const int row_in_tile = q * 32 + lane;
     const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
     uint32_t acc_iter = 0;
-    // wgrad output staging: this warp's two 32 x 32 fp32 buffers (128-byte swizzled rows)
+    // wgrad output staging: this warp's OUTBUFS 32 x 32 fp32 buffers (128-byte swizzled rows)
     uint8_t* obuf = smem + L::kOutOff + ew * OUTBUFS * L::kOutBufBytes;
     uint32_t obuf_iter = 0;
     uint32_t ra[32], rb[32];
     for (int it = 0;; ++it) {
       const int t = next_tile(it);
       if (t < 0) break;
-      const TileInfo ti = decode_tile<MODE, BN>(t, offs_s, tab0, E, K, n_tiles, m_tiles);
-      const bool zero_tile = (MODE == kWgrad) && ti.nk == 0;
-      if (zero_tile && accumulate) continue;  // adding zero changes nothing
+      const TileInfo ti = decode_tile<MODE>(t, p, offs_s, tab_d, tab_w, tc);
+      const bool wg = Tr::kHasW && ti.kind == 1;
+      const bool zero_tile = wg && ti.nk == 0;
+      if (zero_tile && p.accumulate) continue;  // adding zero changes nothing
       uint32_t b = 0;
       if (!zero_tile) {
         b = acc_iter & 1u;
@@ -428,10 +497,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         for (int i = 0; i < 32; ++i) ra[i] = rb[i] = 0u;
       }
       const int row = ti.row0 + row_in_tile;  // dgrad output row
-      const bool row_ok = row < ti.row_end;
+      const bool row_ok = !wg && row < ti.row_end;
       uint4 ga[4], ua[4], gb[4], ub[4];        // SwiGLU: saved g, u of the current / next chunk
-      if constexpr (MODE == kDgradSwiglu) {
-        if (row_ok) load_gu(ga, ua, Gp, Up, row, ti.n0 + cbase * 32, N);
+      if constexpr (Tr::kSwiglu) {
+        if (row_ok) load_gu(ga, ua, p.Gp, p.Up, row, ti.n0 + cbase * 32, p.Nd);
       }
       auto step = [&](uint32_t (&cur)[32], uint32_t (&nxt)[32], uint4 (&gc)[4], uint4 (&uc)[4],
                       uint4 (&gn)[4], uint4 (&un)[4], int i) {
@@ -439,37 +508,42 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         const bool more = i + 1 < kCW;
         if (more && !zero_tile) tmem_ld_32x32b_x32(lane_base + b * BN + (ch + 1) * 32, nxt);
         const int nb = ti.n0 + ch * 32;
-        if constexpr (MODE == kWgrad) {
-          const int mrow = ti.m0 + q * 32;
-          if (mrow < N1 && nb < N) {
-            uint8_t* buf = obuf + (obuf_iter % OUTBUFS) * L::kOutBufBytes;
-            ++obuf_iter;
-            // the store that last used `buf` has read it
-            if (lane == 0) bulk_wait_group_read<OUTBUFS - 1>();
-            __syncwarp();
+        if (wg) {
+          if constexpr (Tr::kHasW) {
+            const int mrow = ti.m0 + q * 32;
+            if (mrow < p.N1 && nb < p.N2) {
+              uint8_t* buf = obuf + (obuf_iter % OUTBUFS) * L::kOutBufBytes;
+              ++obuf_iter;
+              // the store that last used `buf` has read it
+              if (lane == 0) bulk_wait_group_read<OUTBUFS - 1>();
+              __syncwarp();
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int slot = j ^ (lane & 7);
-              *reinterpret_cast<uint4*>(buf + lane * 128 + slot * 16) =
-                  make_uint4(cur[4 * j], cur[4 * j + 1], cur[4 * j + 2], cur[4 * j + 3]);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              if (accumulate)
-                tma_reduce_add_3d(&tmOut, buf, nb, mrow, ti.e);
-              else
-                tma_store_3d(&tmOut, buf, nb, mrow, ti.e);
-              bulk_commit_group();
+              for (int j = 0; j < 8; ++j) {
+                const int slot = j ^ (lane & 7);
+                *reinterpret_cast<uint4*>(buf + lane * 128 + slot * 16) =
+                    make_uint4(cur[4 * j], cur[4 * j + 1], cur[4 * j + 2], cur[4 * j + 3]);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                if (p.accumulate)
+                  tma_reduce_add_3d(&tmOut, buf, nb, mrow, ti.e);
+                else
+                  tma_store_3d(&tmOut, buf, nb, mrow, ti.e);
+                bulk_commit_group();
+              }
             }
           }
-        } else if constexpr (MODE == kDgradStore) {
-          if (row_ok) epi_store_bf16(cur, static_cast<uint16_t*>(out) + (size_t)row * N, nb, N);
-        } else {
-          if (more && row_ok) load_gu(gn, un, Gp, Up, row, nb + 32, N);
-          if (row_ok) {
-            uint16_t* og = static_cast<uint16_t*>(out) + (size_t)row * 2 * N;
-            epi_swiglu(cur, gc, uc, og, og + N, nb, N);
+        } else if constexpr (Tr::kHasD) {
+          if constexpr (Tr::kSwiglu) {
+            if (more && row_ok) load_gu(gn, un, p.Gp, p.Up, row, nb + 32, p.Nd);
+            if (row_ok) {
+              uint16_t* og = static_cast<uint16_t*>(p.out_d) + (size_t)row * 2 * p.Nd;
+              epi_swiglu(cur, gc, uc, og, og + p.Nd, nb, p.Nd);
+            }
+          } else {
+            if (row_ok)
+              epi_store_bf16(cur, static_cast<uint16_t*>(p.out_d) + (size_t)row * p.Nd, nb, p.Nd);
           }
         }
         if (more && !zero_tile) {
@@ -491,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
       if (!zero_tile) ++acc_iter;
     }
   }
-  if constexpr (MODE == kWgrad) {
+  if constexpr (Tr::kHasW) {
     // shared memory must outlive the bulk stores that read it
     if (warp >= 2 && lane == 0) bulk_wait_group<0>();  // every epilogue warp
     __syncwarp();
@@ -577,54 +651,57 @@ bool make_map_out_f32(CUtensorMap* m, void* base, uint64_t E, uint64_t N1, uint6
 // Launch counter of all grouped-GEMM kernels (picks the scheduling slot).
 std::atomic<unsigned int> g_launches{0};
 
-constexpr int kBN = 256;
+struct Maps {
+  CUtensorMap ad, bd, aw, bw, out;
+};
 
 // Launch one instantiation; the dynamic shared memory depends on E.
 template <int MODE, int S, int OB>
-cudaError_t launch_variant(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
-                           const int32_t* offsets, int E, int K, int N, int N1, const void* Gp,
-                           const void* Up, void* out, int accumulate, uint32_t* status,
-                           cudaStream_t s, int grid) {
-  using L = Layout<kBN, S, OB>;
+cudaError_t launch_variant(const Maps& m, GemmParams prm, cudaStream_t s, int grid) {
+  using L = Layout<kBNT, S, OB>;
   static_assert(L::alloc(kMaxExperts) <= kSmemLimit || OB == 1,
                 "shared memory over the sm_100 per-block limit");
-  const int smem = L::alloc(E);
+  const int smem = L::alloc(prm.E);
   if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
   static unsigned long long attr_done = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tc<MODE, kBN, S, OB>,
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tc<MODE, S, OB>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            kSmemLimit);
     if (err != cudaSuccess) return err;
     attr_done |= 1ull << dev;
   }
-  const int slot = (int)(g_launches.fetch_add(1u) % kSchedSlots);
-  return launch_pdl(grouped_gemm_tc<MODE, kBN, S, OB>, dim3(grid), dim3(kThreads), (size_t)smem,
-                    s, ta, tb, tout, offsets, E, K, N, N1, static_cast<const uint16_t*>(Gp),
-                    static_cast<const uint16_t*>(Up), out, accumulate, status, slot);
+  prm.sched_slot = (int)(g_launches.fetch_add(1u) % kSchedSlots);
+  return launch_pdl(grouped_gemm_tc<MODE, S, OB>, dim3(grid), dim3(kThreads), (size_t)smem, s,
+                    m.ad, m.bd, m.aw, m.bw, m.out, prm);
 }
 
-// dgrad K loops are long (K = H or 2I): 4 stages.  wgrad K loops are short
-// (K = m_e) and its fp32 output goes through shared memory: 4 stages with one
-// staging buffer per epilogue warp when that fits for this E (E <= ~130), else
-// 3 stages with two buffers.
+// dgrad K loops are long (K = H or 2I): 4 stages.  Launches with wgrad tiles
+// stage their fp32 output in shared memory: 4 stages with one staging buffer
+// per epilogue warp when that fits for this E (E <= ~140), else 3 stages with two.
 template <int MODE>
-cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
-                        const int32_t* offsets, int E, int K, int N, int N1, const void* Gp,
-                        const void* Up, void* out, int accumulate, uint32_t* status,
-                        cudaStream_t s, int grid) {
-  if constexpr (MODE == kWgrad) {
-    if (Layout<kBN, 4, 1>::alloc(E) <= kSmemLimit)
-      return launch_variant<MODE, 4, 1>(ta, tb, tout, offsets, E, K, N, N1, Gp, Up, out,
-                                        accumulate, status, s, grid);
-    return launch_variant<MODE, 3, 2>(ta, tb, tout, offsets, E, K, N, N1, Gp, Up, out, accumulate,
-                                      status, s, grid);
+cudaError_t launch_mode(const Maps& m, const GemmParams& prm, cudaStream_t s, int grid) {
+  if constexpr (Traits<MODE>::kHasW) {
+    if (Layout<kBNT, 4, 1>::alloc(prm.E) <= kSmemLimit)
+      return launch_variant<MODE, 4, 1>(m, prm, s, grid);
+    return launch_variant<MODE, 3, 2>(m, prm, s, grid);
   } else {
-    return launch_variant<MODE, 4, 0>(ta, tb, tout, offsets, E, K, N, N1, Gp, Up, out, accumulate,
-                                      status, s, grid);
+    return launch_variant<MODE, 4, 0>(m, prm, s, grid);
   }
+}
+
+bool dgrad_maps(Maps* m, const void* rows, int rows_cap, const void* W, int E, int K, int N) {
+  return make_map_2d(&m->ad, rows, (uint64_t)rows_cap, (uint64_t)K, 64, 128) &&
+         make_map_3d(&m->bd, W, (uint64_t)E, (uint64_t)K, (uint64_t)N);
+}
+
+bool wgrad_maps(Maps* m, const void* grad_rows, const void* in_rows, int rows_cap, int E, int N1,
+                int N2, float* dW) {
+  return make_map_2d(&m->aw, grad_rows, (uint64_t)rows_cap, (uint64_t)N1, 64, 64) &&
+         make_map_2d(&m->bw, in_rows, (uint64_t)rows_cap, (uint64_t)N2, 64, 64) &&
+         make_map_out_f32(&m->out, dW, (uint64_t)E, (uint64_t)N1, (uint64_t)N2);
 }
 
 }  // namespace
@@ -633,36 +710,49 @@ cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
                             const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
                             const void* Gp, const void* Up, void* out, uint32_t* status,
                             cudaStream_t s, const char** why) {
-  CUtensorMap ta, tb;
-  if (!make_map_2d(&ta, rows, (uint64_t)rows_cap, (uint64_t)K, 64, 128) ||
-      !make_map_3d(&tb, W, (uint64_t)E, (uint64_t)K, (uint64_t)N)) {
+  Maps m;
+  if (!dgrad_maps(&m, rows, rows_cap, W, E, K, N)) {
     *why = "cuTensorMapEncodeTiled failed for a dgrad operand";
     return cudaErrorInvalidValue;
   }
-  const int grid = num_sms();
-  if (epi == LRMOE_EPI_SWIGLU_BWD)
-    return launch_mode<kDgradSwiglu>(ta, tb, ta, offsets, E, K, N, 0, Gp, Up, out, 0, status, s,
-                                     grid);
-  return launch_mode<kDgradStore>(ta, tb, ta, offsets, E, K, N, 0, nullptr, nullptr, out, 0, status,
-                                  s, grid);
+  m.aw = m.bw = m.out = m.ad;  // unused
+  GemmParams prm{offsets, E, K, N, 0, 0, static_cast<const uint16_t*>(Gp),
+                 static_cast<const uint16_t*>(Up), out, 0, status, 0};
+  if (epi == LRMOE_EPI_SWIGLU_BWD) return launch_mode<kDgradSwiglu>(m, prm, s, num_sms());
+  return launch_mode<kDgradStore>(m, prm, s, num_sms());
 }
 
 cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows_cap,
                             const int32_t* offsets, int E, int N1, int N2, float* dW,
                             int accumulate, uint32_t* status, cudaStream_t s, const char** why) {
-  CUtensorMap ta, tb, tout;
-  if (!make_map_2d(&ta, grad_rows, (uint64_t)rows_cap, (uint64_t)N1, 64, 64) ||
-      !make_map_2d(&tb, in_rows, (uint64_t)rows_cap, (uint64_t)N2, 64, 64) ||
-      !make_map_out_f32(&tout, dW, (uint64_t)E, (uint64_t)N1, (uint64_t)N2)) {
+  Maps m;
+  if (!wgrad_maps(&m, grad_rows, in_rows, rows_cap, E, N1, N2, dW)) {
     *why = "cuTensorMapEncodeTiled failed for a wgrad operand";
     return cudaErrorInvalidValue;
   }
-  const long long total =
-      (long long)E * ((N1 + BM - 1) / BM) * ((N2 + kBN - 1) / kBN);
+  m.ad = m.bd = m.aw;  // unused
+  const long long total = (long long)E * ((N1 + BM - 1) / BM) * ((N2 + kBNT - 1) / kBNT);
   int grid = num_sms();
   if (total < grid) grid = (int)total;
-  return launch_mode<kWgrad>(ta, tb, tout, offsets, E, 0, N2, N1, nullptr, nullptr, dW, accumulate,
-                             status, s, grid);
+  GemmParams prm{offsets, E, 0, 0, N1, N2, nullptr, nullptr, nullptr, accumulate, status, 0};
+  return launch_mode<kWgrad>(m, prm, s, grid);
+}
+
+cudaError_t launch_dgrad_wgrad_tc(const void* grad_rows, int rows_cap, const void* W,
+                                  const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
+                                  const void* Gp, const void* Up, void* out, const void* in_rows,
+                                  int N2, float* dW, int accumulate, uint32_t* status,
+                                  cudaStream_t s, const char** why) {
+  Maps m;
+  if (!dgrad_maps(&m, grad_rows, rows_cap, W, E, K, N) ||
+      !wgrad_maps(&m, grad_rows, in_rows, rows_cap, E, K, N2, dW)) {
+    *why = "cuTensorMapEncodeTiled failed for a fused dgrad/wgrad operand";
+    return cudaErrorInvalidValue;
+  }
+  GemmParams prm{offsets, E, K, N, K, N2, static_cast<const uint16_t*>(Gp),
+                 static_cast<const uint16_t*>(Up), out, accumulate, status, 0};
+  if (epi == LRMOE_EPI_SWIGLU_BWD) return launch_mode<kFusedSwiglu>(m, prm, s, num_sms());
+  return launch_mode<kFusedStore>(m, prm, s, num_sms());
 }
 
 }  // namespace lrmoe

@@ -105,6 +105,21 @@ def test_split_by_destination_rejects_bad_arguments(lib):
     assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
 
 
+def test_fused_gemm_rejects_bad_arguments(lib):
+    f = lib.lrmoe_grouped_dgrad_wgrad
+    args = [FAKE, 64, FAKE, FAKE, 4, 64, 64, 1, 0, NULL, NULL, FAKE, FAKE, 64, FAKE, 0, NULL, NULL]
+    bad = list(args); bad[7] = 0                          # fp32: the fused launch is bf16 only
+    assert f(*bad) == L.LRMOE_ERR_UNSUPPORTED
+    bad = list(args); bad[14] = NULL                      # dW
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG and b"dW" in lib.lrmoe_last_error()
+    bad = list(args); bad[8] = 1                          # SwiGLU epilogue without g, u
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
+    bad = list(args); bad[13] = 12                        # N2 not a multiple of 8
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
+    bad = list(args); bad[4] = 5000                       # E above the grouped-GEMM limit
+    assert f(*bad) == L.LRMOE_ERR_UNSUPPORTED
+
+
 def test_select_rejects_small_workspace(lib):
     f = lib.lrmoe_select_quota
     need = L.lrmoe_select_workspace_bytes(64, 2, 4)
