@@ -83,7 +83,8 @@ def algorithmic(T, k, E, H, I, M, b):
     by = {
         "score": T * H * b + P * I * b + 8 * P + 4 * P,
         "select": 4 * P + 4 * P + 4 * E + 12 * E + 4 * M + 4 * P,
-        "pack": 2 * M * (2 * H + 3 * I) * b + 8 * M,
+        # X_p, DY_p, A_p (bf16 path: g, u are read in place by the SwiGLU epilogue)
+        "pack": 2 * M * (2 * H + (I if b == 2 else 3 * I)) * b + 8 * M,
         "dgrad_swiglu": M * H * b + E * H * I * b + 2 * M * I * b + 2 * M * I * b,
         "wgrad_down": M * H * b + M * I * b + E * H * I * 4,
         "wgrad_gu": 2 * M * I * b + M * H * b + E * 2 * I * H * 4,
@@ -385,6 +386,7 @@ def make_runner(layer, dev):
     def step(ev=None, a_sqnorm=None, fused=False):
         """One pass of the path; with a_sqnorm (||a_p||^2 saved by the forward) the
         score reads dY and the saved norms instead of a."""
+        gather = s.dtype == "bf16" and not fused   # the path's g, u handling
         score_call = (
             (lambda: L.lrmoe_score(inp["topk_idx"], inp["topk_w"], inp["dY"], inp["a"], s.E,
                                    out["score"], st, stream)) if a_sqnorm is None else
@@ -395,15 +397,22 @@ def make_runner(layer, dev):
             lambda: L.lrmoe_select_quota(inp["topk_idx"], out["score"], inp["quota"], out["counts"],
                                          out["kept"], out["offsets"], out["perm"], out["pos"],
                                          out["workspace"], st, stream),
-            lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], inp["x"], inp["dY"],
-                                 inp["a"], inp["g"], inp["u"], out["Xp"], out["DYp"], out["Ap"],
-                                 out["Gp"], out["Up"], st, stream),
+            # bf16: G_p, U_p are not packed; the SwiGLU epilogue reads g, u in place
+            (lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], inp["x"], inp["dY"],
+                                  inp["a"], None, None, out["Xp"], out["DYp"], out["Ap"], None,
+                                  None, st, stream)) if gather else
+            (lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], inp["x"], inp["dY"],
+                                  inp["a"], inp["g"], inp["u"], out["Xp"], out["DYp"], out["Ap"],
+                                  out["Gp"], out["Up"], st, stream)),
         )
         if not fused:  # the four grouped GEMMs as separate launches
             gemms = (
-                lambda: L.lrmoe_grouped_dgrad(out["DYp"], inp["W_down"], out["offsets"],
-                                              L.LRMOE_EPI_SWIGLU_BWD, out["dGUp"], Gp=out["Gp"],
-                                              Up=out["Up"], status=st, stream=stream),
+                (lambda: L.lrmoe_grouped_dgrad_swiglu_gather(
+                    out["DYp"], inp["W_down"], out["offsets"], out["perm"], inp["g"], inp["u"],
+                    out["dGUp"], status=st, stream=stream)) if gather else
+                (lambda: L.lrmoe_grouped_dgrad(out["DYp"], inp["W_down"], out["offsets"],
+                                               L.LRMOE_EPI_SWIGLU_BWD, out["dGUp"], Gp=out["Gp"],
+                                               Up=out["Up"], status=st, stream=stream)),
                 lambda: L.lrmoe_grouped_wgrad(out["DYp"], out["Ap"], out["offsets"],
                                               out["dW_down"], status=st, stream=stream),
                 lambda: L.lrmoe_grouped_wgrad(out["dGUp"], out["Xp"], out["offsets"],

@@ -282,7 +282,9 @@ int lrmoe_select_quota_noalloc(const int32_t* topk_idx, const float* score, int 
  *   Ap[r] = a[p] (I)      Gp[r] = g[p] (I)       Up[r] = u[p] (I)
  * x, dY [T][H]; a, g, u [T*k][I]; outputs [rows_cap][.] with rows_cap >= M
  * (T*k always suffices).  Rows >= M are not touched.  A perm entry outside
- * [0, T*k) is skipped and sets LRMOE_ST_BAD_INDEX.
+ * [0, T*k) is skipped and sets LRMOE_ST_BAD_INDEX.  Gp and Up may both be NULL
+ * (then g, u may be NULL too): G_p, U_p are not packed, for the SwiGLU
+ * epilogue that reads g, u in place (lrmoe_grouped_dgrad_swiglu_gather).
  * ------------------------------------------------------------------------- */
 int lrmoe_pack(const int32_t* perm, const int32_t* offsets, const float* topk_w, int T, int k, int E,
                const void* x, const void* dY, int H, const void* a, const void* g, const void* u,
@@ -324,6 +326,21 @@ int lrmoe_grouped_wgrad(const void* grad_rows, const void* in_rows, int rows_cap
                         float* dW, int accumulate, uint32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * a4 dgrad with the SwiGLU-backward epilogue, gathering g and u in place (the
+ * pages' dense per-expert blocks are what the tensor cores read; the
+ * epilogue's per-row operands need no copy).  As lrmoe_grouped_dgrad with
+ * epi = LRMOE_EPI_SWIGLU_BWD, except that packed row r reads g, u [gu_rows][N]
+ * at row perm[r] (perm from lrmoe_select_quota, gu_rows = T*k) instead of
+ * Gp[r], Up[r]; bit-identical results.  perm entries outside [0, gu_rows) set
+ * LRMOE_ST_BAD_INDEX and leave that output row unwritten.  bf16 only (fp32:
+ * LRMOE_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------- */
+int lrmoe_grouped_dgrad_swiglu_gather(const void* rows, int rows_cap, const void* W,
+                                      const int32_t* offsets, int E, int K, int N, lrmoe_dtype dt,
+                                      const int32_t* perm, const void* g, const void* u, int gu_rows,
+                                      void* out, uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * a4, two GEMMs that share their gradient rows in one launch (same passages).
  * Exactly lrmoe_grouped_dgrad(grad_rows, rows_cap, W, offsets, E, K, N, dt,
  * epi, Gp, Up, out) plus lrmoe_grouped_wgrad(grad_rows, in_rows, rows_cap,
@@ -358,7 +375,9 @@ int lrmoe_unpack(const void* dXp, int rows_cap, const int32_t* pos, int T, int k
  * The whole path a1..a5 on one stream (RU-B bullets 3-5): score, selection,
  * compaction, the four grouped GEMMs and the return to the token layout, as
  * one enqueue with no host synchronisation.  All buffers are caller-owned
- * device memory; rows_cap >= M (T*k always suffices).
+ * device memory; rows_cap >= M (T*k always suffices).  For bf16 the SwiGLU
+ * epilogue reads g, u in place, so Gp and Up are neither written nor needed
+ * (they may be NULL); fp32 packs them.
  * ------------------------------------------------------------------------- */
 typedef struct {
   /* inputs */

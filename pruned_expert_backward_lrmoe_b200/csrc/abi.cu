@@ -280,13 +280,16 @@ int lrmoe_pack(const int32_t* perm, const int32_t* offsets, const float* topk_w,
   REQUIRE_PTR(x);
   REQUIRE_PTR(dY);
   REQUIRE_PTR(a);
-  REQUIRE_PTR(g);
-  REQUIRE_PTR(u);
   REQUIRE_PTR(Xp);
   REQUIRE_PTR(DYp);
   REQUIRE_PTR(Ap);
-  REQUIRE_PTR(Gp);
-  REQUIRE_PTR(Up);
+  REQUIRE((Gp == nullptr) == (Up == nullptr), "Gp and Up must both be given or both be NULL");
+  if (Gp) {  // G_p, U_p are optional (the gathering SwiGLU epilogue reads g, u in place)
+    REQUIRE_PTR(g);
+    REQUIRE_PTR(u);
+    REQUIRE_PTR(Gp);
+    REQUIRE_PTR(Up);
+  }
   cudaError_t e = launch_pack(perm, offsets, topk_w, T, k, E, x, dY, H, a, g, u, I, dt, Xp, DYp, Ap,
                               Gp, Up, rows_cap, status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_pack launch");
@@ -321,6 +324,32 @@ int lrmoe_grouped_dgrad(const void* rows, int rows_cap, const void* W, const int
     if (e != cudaSuccess) return cuda_fail(e, "lrmoe_grouped_dgrad launch");
   }
   return LRMOE_OK;
+}
+
+int lrmoe_grouped_dgrad_swiglu_gather(const void* rows, int rows_cap, const void* W,
+                                      const int32_t* offsets, int E, int K, int N, lrmoe_dtype dt,
+                                      const int32_t* perm, const void* g, const void* u, int gu_rows,
+                                      void* out, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  if (dt != LRMOE_BF16)
+    return fail(LRMOE_ERR_UNSUPPORTED, "the gathering epilogue is bf16 only; pack G_p, U_p");
+  REQUIRE(E > 0 && rows_cap > 0 && gu_rows > 0, "E, rows_cap and gu_rows must be positive");
+  if (E > kMaxGroupedExperts) return fail(LRMOE_ERR_UNSUPPORTED, "E=%d > %d", E, kMaxGroupedExperts);
+  if (int r = check_feature(K, dt, "K")) return r;
+  if (int r = check_feature(N, dt, "N")) return r;
+  REQUIRE_PTR(rows);
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(perm);
+  REQUIRE_PTR(g);
+  REQUIRE_PTR(u);
+  REQUIRE_PTR(out);
+  const char* why = "launch failed";
+  cudaError_t e = launch_dgrad_tc(rows, rows_cap, W, offsets, E, K, N, LRMOE_EPI_SWIGLU_BWD, g, u,
+                                  out, status, static_cast<cudaStream_t>(stream), &why, perm,
+                                  gu_rows);
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, why);
 }
 
 int lrmoe_grouped_wgrad(const void* grad_rows, const void* in_rows, int rows_cap,
@@ -420,13 +449,26 @@ int lrmoe_pruned_backward(const lrmoe_buffers* b, int T, int k, int E, int H, in
                               b->offsets, b->perm, b->pos, b->workspace, b->workspace_bytes,
                               b->status, stream)))
     return r;
-  if ((r = lrmoe_pack(b->perm, b->offsets, b->topk_w, T, k, E, b->x, b->dY, H, b->a, b->g, b->u, I,
-                      dt, b->Xp, b->DYp, b->Ap, b->Gp, b->Up, rows_cap, b->status, stream)))
-    return r;
-  // dA -> [dG | dU]  (m_e x H) . (H x I), SwiGLU backward in the epilogue
-  if ((r = lrmoe_grouped_dgrad(b->DYp, rows_cap, b->W_down, b->offsets, E, H, I, dt,
-                               LRMOE_EPI_SWIGLU_BWD, b->Gp, b->Up, b->dGUp, b->status, stream)))
-    return r;
+  if (dt == LRMOE_BF16) {
+    // g, u are read in place by the SwiGLU epilogue (row perm[r]); only the
+    // operands the tensor cores load with TMA are packed
+    if ((r = lrmoe_pack(b->perm, b->offsets, b->topk_w, T, k, E, b->x, b->dY, H, b->a, nullptr,
+                        nullptr, I, dt, b->Xp, b->DYp, b->Ap, nullptr, nullptr, rows_cap, b->status,
+                        stream)))
+      return r;
+    if ((r = lrmoe_grouped_dgrad_swiglu_gather(b->DYp, rows_cap, b->W_down, b->offsets, E, H, I, dt,
+                                               b->perm, b->g, b->u, T * k, b->dGUp, b->status,
+                                               stream)))
+      return r;
+  } else {
+    if ((r = lrmoe_pack(b->perm, b->offsets, b->topk_w, T, k, E, b->x, b->dY, H, b->a, b->g, b->u,
+                        I, dt, b->Xp, b->DYp, b->Ap, b->Gp, b->Up, rows_cap, b->status, stream)))
+      return r;
+    // dA -> [dG | dU]  (m_e x H) . (H x I), SwiGLU backward in the epilogue
+    if ((r = lrmoe_grouped_dgrad(b->DYp, rows_cap, b->W_down, b->offsets, E, H, I, dt,
+                                 LRMOE_EPI_SWIGLU_BWD, b->Gp, b->Up, b->dGUp, b->status, stream)))
+      return r;
+  }
   // dW_down = DY_p^T A_p
   if ((r = lrmoe_grouped_wgrad(b->DYp, b->Ap, rows_cap, b->offsets, E, H, I, dt, b->dW_down, 0,
                                b->status, stream)))

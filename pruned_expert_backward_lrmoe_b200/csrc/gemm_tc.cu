@@ -83,8 +83,10 @@ struct GemmParams {
   int E;
   int Kd, Nd;           // dgrad
   int N1, N2;           // wgrad
-  const uint16_t* Gp;   // SwiGLU epilogue: saved g, u [rows][Nd]
-  const uint16_t* Up;
+  const uint16_t* Gp;   // SwiGLU epilogue: saved g, u [rows][Nd] (packed), or [gu_rows][Nd]
+  const uint16_t* Up;   // read at row perm[r] when perm is given
+  const int32_t* perm;
+  int gu_rows;
   void* out_d;          // dgrad output [rows][Nd] (SwiGLU: [rows][2 Nd])
   int accumulate;       // wgrad: add into dW
   uint32_t* status;
@@ -497,10 +499,20 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         for (int i = 0; i < 32; ++i) ra[i] = rb[i] = 0u;
       }
       const int row = ti.row0 + row_in_tile;  // dgrad output row
-      const bool row_ok = !wg && row < ti.row_end;
+      bool row_ok = !wg && row < ti.row_end;
+      int gu_row = row;                        // SwiGLU: row of g, u
+      if constexpr (Tr::kSwiglu) {
+        if (row_ok && p.perm != nullptr) {
+          gu_row = p.perm[row];
+          if (gu_row < 0 || gu_row >= p.gu_rows) {
+            raise_status(status, LRMOE_ST_BAD_INDEX);
+            row_ok = false;
+          }
+        }
+      }
       uint4 ga[4], ua[4], gb[4], ub[4];        // SwiGLU: saved g, u of the current / next chunk
       if constexpr (Tr::kSwiglu) {
-        if (row_ok) load_gu(ga, ua, p.Gp, p.Up, row, ti.n0 + cbase * 32, p.Nd);
+        if (row_ok) load_gu(ga, ua, p.Gp, p.Up, gu_row, ti.n0 + cbase * 32, p.Nd);
       }
       auto step = [&](uint32_t (&cur)[32], uint32_t (&nxt)[32], uint4 (&gc)[4], uint4 (&uc)[4],
                       uint4 (&gn)[4], uint4 (&un)[4], int i) {
@@ -536,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
           }
         } else if constexpr (Tr::kHasD) {
           if constexpr (Tr::kSwiglu) {
-            if (more && row_ok) load_gu(gn, un, p.Gp, p.Up, row, nb + 32, p.Nd);
+            if (more && row_ok) load_gu(gn, un, p.Gp, p.Up, gu_row, nb + 32, p.Nd);
             if (row_ok) {
               uint16_t* og = static_cast<uint16_t*>(p.out_d) + (size_t)row * 2 * p.Nd;
               epi_swiglu(cur, gc, uc, og, og + p.Nd, nb, p.Nd);
@@ -709,7 +721,7 @@ bool wgrad_maps(Maps* m, const void* grad_rows, const void* in_rows, int rows_ca
 cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
                             const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
                             const void* Gp, const void* Up, void* out, uint32_t* status,
-                            cudaStream_t s, const char** why) {
+                            cudaStream_t s, const char** why, const int32_t* perm, int gu_rows) {
   Maps m;
   if (!dgrad_maps(&m, rows, rows_cap, W, E, K, N)) {
     *why = "cuTensorMapEncodeTiled failed for a dgrad operand";
@@ -717,7 +729,7 @@ cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
   }
   m.aw = m.bw = m.out = m.ad;  // unused
   GemmParams prm{offsets, E, K, N, 0, 0, static_cast<const uint16_t*>(Gp),
-                 static_cast<const uint16_t*>(Up), out, 0, status, 0};
+                 static_cast<const uint16_t*>(Up), perm, gu_rows, out, 0, status, 0};
   if (epi == LRMOE_EPI_SWIGLU_BWD) return launch_mode<kDgradSwiglu>(m, prm, s, num_sms());
   return launch_mode<kDgradStore>(m, prm, s, num_sms());
 }
@@ -734,7 +746,8 @@ cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows
   const long long total = (long long)E * ((N1 + BM - 1) / BM) * ((N2 + kBNT - 1) / kBNT);
   int grid = num_sms();
   if (total < grid) grid = (int)total;
-  GemmParams prm{offsets, E, 0, 0, N1, N2, nullptr, nullptr, nullptr, accumulate, status, 0};
+  GemmParams prm{offsets, E, 0, 0, N1, N2, nullptr, nullptr, nullptr, 0, nullptr, accumulate,
+                 status, 0};
   return launch_mode<kWgrad>(m, prm, s, grid);
 }
 
@@ -750,7 +763,7 @@ cudaError_t launch_dgrad_wgrad_tc(const void* grad_rows, int rows_cap, const voi
     return cudaErrorInvalidValue;
   }
   GemmParams prm{offsets, E, K, N, K, N2, static_cast<const uint16_t*>(Gp),
-                 static_cast<const uint16_t*>(Up), out, accumulate, status, 0};
+                 static_cast<const uint16_t*>(Up), nullptr, 0, out, accumulate, status, 0};
   if (epi == LRMOE_EPI_SWIGLU_BWD) return launch_mode<kFusedSwiglu>(m, prm, s, num_sms());
   return launch_mode<kFusedStore>(m, prm, s, num_sms());
 }

@@ -98,10 +98,12 @@ cudaError_t launch_quota(const int32_t* idx, int P, int E, int cap, long long bu
 cudaError_t launch_selftest_wait(uint32_t limit_us, uint32_t* status, cudaStream_t s);
 
 // tcgen05 grouped GEMMs (bf16 storage)
+// perm != nullptr: the SwiGLU epilogue reads g, u ([gu_rows][N]) at row perm[r]
 cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
                             const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
                             const void* Gp, const void* Up, void* out, uint32_t* status,
-                            cudaStream_t s, const char** why);
+                            cudaStream_t s, const char** why, const int32_t* perm = nullptr,
+                            int gu_rows = 0);
 cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows_cap,
                             const int32_t* offsets, int E, int N1, int N2, float* dW,
                             int accumulate, uint32_t* status, cudaStream_t s, const char** why);

@@ -93,8 +93,8 @@ __global__ void __launch_bounds__(256) pack_kernel(
     copy_row(Xp + rr * VH, x + (size_t)t * VH, VH, lane);
     scale_row<DT>(DYp + rr * VH, dY + (size_t)t * VH, VH, wp, lane);
     copy_row(Ap + rr * VI, a + (size_t)p * VI, VI, lane);
-    copy_row(Gp + rr * VI, g + (size_t)p * VI, VI, lane);
-    copy_row(Up + rr * VI, u + (size_t)p * VI, VI, lane);
+    if (Gp) copy_row(Gp + rr * VI, g + (size_t)p * VI, VI, lane);  // optional: the SwiGLU
+    if (Up) copy_row(Up + rr * VI, u + (size_t)p * VI, VI, lane);  // epilogue can gather g, u
   }
 }
 

@@ -27,7 +27,8 @@ EXPORTS = ("lrmoe_version", "lrmoe_status_string", "lrmoe_last_error", "lrmoe_sc
            "lrmoe_grouped_dgrad", "lrmoe_grouped_wgrad", "lrmoe_unpack", "lrmoe_pruned_backward",
            "lrmoe_select_quota_noalloc", "lrmoe_selftest_bounded_wait", "lrmoe_quota_controller",
            "lrmoe_row_sqnorm", "lrmoe_score_from_norms", "lrmoe_router_grad",
-           "lrmoe_redistribute", "lrmoe_split_by_destination", "lrmoe_grouped_dgrad_wgrad")
+           "lrmoe_redistribute", "lrmoe_split_by_destination", "lrmoe_grouped_dgrad_wgrad",
+           "lrmoe_grouped_dgrad_swiglu_gather")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -77,6 +78,7 @@ def load() -> ctypes.CDLL:
     lib.lrmoe_pack.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, I, I, P, P, P, P, P, I, P, P]
     lib.lrmoe_grouped_dgrad.argtypes = [P, I, P, P, I, I, I, I, I, P, P, P, P, P]
     lib.lrmoe_grouped_wgrad.argtypes = [P, P, I, P, I, I, I, I, P, I, P, P]
+    lib.lrmoe_grouped_dgrad_swiglu_gather.argtypes = [P, I, P, P, I, I, I, I, P, P, P, I, P, P, P]
     lib.lrmoe_grouped_dgrad_wgrad.argtypes = [P, I, P, P, I, I, I, I, I, P, P, P, P, I, P, I, P, P]
     lib.lrmoe_unpack.argtypes = [P, I, P, I, I, I, I, P, P, P]
     lib.lrmoe_pruned_backward.argtypes = [ctypes.POINTER(lrmoe_buffers), I, I, I, I, I, I, I, P]
@@ -236,6 +238,16 @@ def lrmoe_grouped_wgrad(grad_rows, in_rows, offsets, dW, accumulate: bool = Fals
     _check(load().lrmoe_grouped_wgrad(_ptr(grad_rows), _ptr(in_rows), grad_rows.shape[0],
                                       _ptr(offsets), E, N1, N2, _dt(grad_rows), _ptr(dW),
                                       int(accumulate), _ptr(status), _stream(stream)))
+
+
+def lrmoe_grouped_dgrad_swiglu_gather(rows, W, offsets, perm, g, u, out, status=None,
+                                      stream=None) -> None:
+    """dgrad with the SwiGLU-backward epilogue reading g, u [T*k][N] at row perm[r] (bf16)."""
+    E, K, N = W.shape
+    _check(load().lrmoe_grouped_dgrad_swiglu_gather(_ptr(rows), rows.shape[0], _ptr(W),
+                                                    _ptr(offsets), E, K, N, _dt(rows), _ptr(perm),
+                                                    _ptr(g), _ptr(u), g.shape[0], _ptr(out),
+                                                    _ptr(status), _stream(stream)))
 
 
 def lrmoe_grouped_dgrad_wgrad(grad_rows, W, offsets, epilogue: int, out, in_rows, dW, Gp=None,

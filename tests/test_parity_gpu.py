@@ -74,7 +74,7 @@ def test_chain_entry_point_equals_steps_and_is_deterministic():
     for name in ("score", "counts", "kept", "offsets", "pos", "dW_down", "dW_gu", "dX"):
         assert _same_bytes(a[name], b[name]), name
         assert _same_bytes(b[name], c[name]), name
-    for name in ("perm", "Xp", "DYp", "Ap", "Gp", "Up", "dGUp", "dXp"):
+    for name in ("perm", "dGUp", "dXp") + PT.chain_packed(layer):
         assert _same_bytes(a[name][:M], b[name][:M]), name
         assert _same_bytes(b[name][:M], c[name][:M]), name
 
@@ -177,7 +177,8 @@ def test_full_size_parity(name):
     M = PT.check_selection(layer, out, ref)
     Xp, DYp, Ap, Gp, Up = O.pack(perm, layer.topk_w, s.k, layer.x, layer.dY, layer.a, layer.g,
                                  layer.u, dt)
-    PT.check_pack(layer, out, dict(Xp=Xp, DYp=DYp, Ap=Ap, Gp=Gp, Up=Up), M)
+    PT.check_pack(layer, out, dict(Xp=Xp, DYp=DYp, Ap=Ap, Gp=Gp, Up=Up), M,
+                  PT.chain_packed(layer))
     rng = np.random.default_rng(0)
     experts = sampled_experts(kept, rng)
     dWd, dWgu, _, _ = O.expert_backward(Xp, DYp, Ap, Gp, Up, offsets, layer.W_gu, layer.W_down, dt,
