@@ -83,7 +83,8 @@ def algorithmic(T, k, E, H, I, M, b):
     by = {
         "score": T * H * b + P * I * b + 8 * P + 4 * P,
         "select": 4 * P + 4 * P + 4 * E + 12 * E + 4 * M + 4 * P,
-        # X_p, DY_p, A_p (bf16 path: g, u are read in place by the SwiGLU epilogue)
+        # bf16 path: X_p, DY_p, A_p (g, u are read in place at row perm[r]);
+        # fp32: X_p, DY_p, A_p, G_p, U_p
         "pack": 2 * M * (2 * H + (I if b == 2 else 3 * I)) * b + 8 * M,
         "dgrad_swiglu": M * H * b + E * H * I * b + 2 * M * I * b + 2 * M * I * b,
         "wgrad_down": M * H * b + M * I * b + E * H * I * 4,
@@ -383,7 +384,7 @@ def make_runner(layer, dev):
         flush.sum()
     st = out["status"]
 
-    def step(ev=None, a_sqnorm=None, fused=False):
+    def step(ev=None, a_sqnorm=None, fused=False, wgrad_gather=False):
         """One pass of the path; with a_sqnorm (||a_p||^2 saved by the forward) the
         score reads dY and the saved norms instead of a."""
         gather = s.dtype == "bf16" and not fused   # the path's g, u handling
@@ -397,7 +398,10 @@ def make_runner(layer, dev):
             lambda: L.lrmoe_select_quota(inp["topk_idx"], out["score"], inp["quota"], out["counts"],
                                          out["kept"], out["offsets"], out["perm"], out["pos"],
                                          out["workspace"], st, stream),
-            # bf16: G_p, U_p are not packed; the SwiGLU epilogue reads g, u in place
+            # bf16: g, u are read in place at row perm[r] (and, with wgrad_gather, a, x)
+            (lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], None, inp["dY"],
+                                  None, None, None, None, out["DYp"], None, None, None, st,
+                                  stream, I=s.I)) if gather and wgrad_gather else
             (lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], inp["x"], inp["dY"],
                                   inp["a"], None, None, out["Xp"], out["DYp"], out["Ap"], None,
                                   None, st, stream)) if gather else
@@ -413,10 +417,16 @@ def make_runner(layer, dev):
                 (lambda: L.lrmoe_grouped_dgrad(out["DYp"], inp["W_down"], out["offsets"],
                                                L.LRMOE_EPI_SWIGLU_BWD, out["dGUp"], Gp=out["Gp"],
                                                Up=out["Up"], status=st, stream=stream)),
-                lambda: L.lrmoe_grouped_wgrad(out["DYp"], out["Ap"], out["offsets"],
-                                              out["dW_down"], status=st, stream=stream),
-                lambda: L.lrmoe_grouped_wgrad(out["dGUp"], out["Xp"], out["offsets"],
-                                              out["dW_gu"], status=st, stream=stream),
+                (lambda: L.lrmoe_grouped_wgrad_gather(
+                    out["DYp"], out["perm"], inp["a"], 1, s.P, out["offsets"], out["dW_down"],
+                    status=st, stream=stream)) if gather and wgrad_gather else
+                (lambda: L.lrmoe_grouped_wgrad(out["DYp"], out["Ap"], out["offsets"],
+                                               out["dW_down"], status=st, stream=stream)),
+                (lambda: L.lrmoe_grouped_wgrad_gather(
+                    out["dGUp"], out["perm"], inp["x"], s.k, s.P, out["offsets"], out["dW_gu"],
+                    status=st, stream=stream)) if gather and wgrad_gather else
+                (lambda: L.lrmoe_grouped_wgrad(out["dGUp"], out["Xp"], out["offsets"],
+                                               out["dW_gu"], status=st, stream=stream)),
                 lambda: L.lrmoe_grouped_dgrad(out["dGUp"], inp["W_gu"], out["offsets"],
                                               L.LRMOE_EPI_STORE, out["dXp"], status=st,
                                               stream=stream),
@@ -526,7 +536,7 @@ def run_gpu(args):
                                                     FALLBACK_PEAKS["bf16_tflops_sustained"]))
         breakdown[kname] = e
 
-    controller_us = controller_matches = fused_step_ms = None
+    controller_us = controller_matches = fused_step_ms = wgrad_gather_step_ms = None
     saved_norms = router = redistribution = None
     e2e_value = e2e_ms = None
     h2d = d2h = 0
@@ -595,6 +605,17 @@ def run_gpu(args):
         torch.cuda.synchronize(dev)
         fused_step_ms = max_over_ranks(
             statistics.fmean(a_.elapsed_time(b_) for a_, b_ in fu_steps), dist)
+        # ... and with the wgrads gathering a, x in place (only DY_p packed)
+        wg_steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(n_bd)]
+        for i in range(n_bd):
+            flush_l2()
+            wg_steps[i][0].record(stream)
+            step(wgrad_gather=True)
+            wg_steps[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        wgrad_gather_step_ms = max_over_ranks(
+            statistics.fmean(a_.elapsed_time(b_) for a_, b_ in wg_steps), dist)
         saved_norms = {
             "row_sqnorm_us": sn_us["row_sqnorm"], "score_from_norms_us": sn_us["score_from_norms"],
             "score_us": sn_us["score"],
@@ -730,6 +751,7 @@ def run_gpu(args):
         "quota_controller_us": controller_us,
         "quota_controller_equals_capacity_rule": controller_matches,
         "fused_gemm_step_ms": fused_step_ms,
+        "gathered_wgrad_step_ms": wgrad_gather_step_ms,
         "saved_norms": saved_norms,
         "router_grad": router,
         "redistribution": redistribution,

@@ -282,9 +282,10 @@ int lrmoe_select_quota_noalloc(const int32_t* topk_idx, const float* score, int 
  *   Ap[r] = a[p] (I)      Gp[r] = g[p] (I)       Up[r] = u[p] (I)
  * x, dY [T][H]; a, g, u [T*k][I]; outputs [rows_cap][.] with rows_cap >= M
  * (T*k always suffices).  Rows >= M are not touched.  A perm entry outside
- * [0, T*k) is skipped and sets LRMOE_ST_BAD_INDEX.  Gp and Up may both be NULL
- * (then g, u may be NULL too): G_p, U_p are not packed, for the SwiGLU
- * epilogue that reads g, u in place (lrmoe_grouped_dgrad_swiglu_gather).
+ * [0, T*k) is skipped and sets LRMOE_ST_BAD_INDEX.  Only DYp is required:
+ * Gp and Up may both be NULL (then g, u may be NULL too), and Xp or Ap may be
+ * NULL (then x or a may be NULL), for the kernels that read those rows in
+ * place (lrmoe_grouped_dgrad_swiglu_gather, lrmoe_grouped_wgrad_gather).
  * ------------------------------------------------------------------------- */
 int lrmoe_pack(const int32_t* perm, const int32_t* offsets, const float* topk_w, int T, int k, int E,
                const void* x, const void* dY, int H, const void* a, const void* g, const void* u,
@@ -324,6 +325,23 @@ int lrmoe_grouped_dgrad(const void* rows, int rows_cap, const void* W, const int
 int lrmoe_grouped_wgrad(const void* grad_rows, const void* in_rows, int rows_cap,
                         const int32_t* offsets, int E, int N1, int N2, lrmoe_dtype dt,
                         float* dW, int accumulate, uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a4 wgrad gathering its second operand in place (same passages as
+ * lrmoe_grouped_wgrad): dW[e] = grad[R_e]^T . B[R_e] with the row of B for
+ * packed row r being src[perm[r] / src_div], src [n_pairs / src_div][N2]:
+ *   dW_down: grad = DY_p, src = a [T*k][I], src_div = 1
+ *   dW_gu:   grad = dGU_p, src = x [T][H],  src_div = k
+ * Bit-identical to lrmoe_grouped_wgrad on the packed rows.  perm entries
+ * outside [0, n_pairs) set LRMOE_ST_BAD_INDEX and read as zero rows.  bf16 only
+ * (fp32: LRMOE_ERR_UNSUPPORTED).  The rows come in through 16-byte cp.async
+ * copies issued by one producer warp, which on a B200 is about half as fast as
+ * the TMA loads of packed rows, so lrmoe_pruned_backward packs X_p and A_p.
+ * ------------------------------------------------------------------------- */
+int lrmoe_grouped_wgrad_gather(const void* grad_rows, int rows_cap, const int32_t* perm,
+                               const void* src, int src_div, int n_pairs, const int32_t* offsets,
+                               int E, int N1, int N2, lrmoe_dtype dt, float* dW, int accumulate,
+                               uint32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------
  * a4 dgrad with the SwiGLU-backward epilogue, gathering g and u in place (the

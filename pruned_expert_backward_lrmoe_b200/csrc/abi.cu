@@ -277,12 +277,16 @@ int lrmoe_pack(const int32_t* perm, const int32_t* offsets, const float* topk_w,
   REQUIRE_PTR(perm);
   REQUIRE_PTR(offsets);
   REQUIRE_PTR(topk_w);
-  REQUIRE_PTR(x);
   REQUIRE_PTR(dY);
-  REQUIRE_PTR(a);
-  REQUIRE_PTR(Xp);
   REQUIRE_PTR(DYp);
-  REQUIRE_PTR(Ap);
+  if (Xp) {  // X_p and A_p are optional too (the gathering wgrad reads x, a in place)
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(Xp);
+  }
+  if (Ap) {
+    REQUIRE_PTR(a);
+    REQUIRE_PTR(Ap);
+  }
   REQUIRE((Gp == nullptr) == (Up == nullptr), "Gp and Up must both be given or both be NULL");
   if (Gp) {  // G_p, U_p are optional (the gathering SwiGLU epilogue reads g, u in place)
     REQUIRE_PTR(g);
@@ -349,6 +353,32 @@ int lrmoe_grouped_dgrad_swiglu_gather(const void* rows, int rows_cap, const void
   cudaError_t e = launch_dgrad_tc(rows, rows_cap, W, offsets, E, K, N, LRMOE_EPI_SWIGLU_BWD, g, u,
                                   out, status, static_cast<cudaStream_t>(stream), &why, perm,
                                   gu_rows);
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, why);
+}
+
+int lrmoe_grouped_wgrad_gather(const void* grad_rows, int rows_cap, const int32_t* perm,
+                               const void* src, int src_div, int n_pairs, const int32_t* offsets,
+                               int E, int N1, int N2, lrmoe_dtype dt, float* dW, int accumulate,
+                               uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  if (dt != LRMOE_BF16)
+    return fail(LRMOE_ERR_UNSUPPORTED, "the gathering wgrad is bf16 only; pack the rows");
+  REQUIRE(E > 0 && rows_cap > 0 && n_pairs > 0, "E, rows_cap and n_pairs must be positive");
+  REQUIRE(src_div > 0 && n_pairs % src_div == 0, "src_div=%d must divide n_pairs=%d", src_div,
+          n_pairs);
+  if (E > kMaxGroupedExperts) return fail(LRMOE_ERR_UNSUPPORTED, "E=%d > %d", E, kMaxGroupedExperts);
+  if (int r = check_feature(N1, dt, "N1")) return r;
+  if (int r = check_feature(N2, dt, "N2")) return r;
+  REQUIRE_PTR(grad_rows);
+  REQUIRE_PTR(perm);
+  REQUIRE_PTR(src);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(dW);
+  const char* why = "launch failed";
+  cudaError_t e = launch_wgrad_gather_tc(grad_rows, rows_cap, perm, src, src_div, n_pairs, offsets,
+                                         E, N1, N2, dW, accumulate, status,
+                                         static_cast<cudaStream_t>(stream), &why);
   return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, why);
 }
 

@@ -38,7 +38,9 @@ constexpr int kEpiThreads = 32 * kEpiWarps;
 
 // kFused*: one launch runs a dgrad (store or SwiGLU epilogue) and a wgrad that
 // share their packed gradient rows.
-enum Mode : int { kDgradStore = 0, kDgradSwiglu = 1, kWgrad = 2, kFusedStore = 3, kFusedSwiglu = 4 };
+// kWgradGather: wgrad whose B rows are gathered from an unpacked tensor.
+enum Mode : int { kDgradStore = 0, kDgradSwiglu = 1, kWgrad = 2, kFusedStore = 3, kFusedSwiglu = 4,
+                  kWgradGather = 5 };
 constexpr int kBNT = 256;  // tile N (TMEM columns per accumulator)
 
 // Dynamic tile scheduling.  Each CTA's producer takes the next tile index from a
@@ -89,15 +91,21 @@ struct GemmParams {
   int gu_rows;
   void* out_d;          // dgrad output [rows][Nd] (SwiGLU: [rows][2 Nd])
   int accumulate;       // wgrad: add into dW
+  // kWgradGather: B row of packed row r = gsrc[perm[r] / gdiv] ([*][N2]); perm
+  // entries must lie in [0, gperm_max)
+  const uint16_t* gsrc;
+  int gdiv, gperm_max;
   uint32_t* status;
   int sched_slot;
 };
 
 template <int MODE>
 struct Traits {
-  static constexpr bool kHasD = MODE != kWgrad;
-  static constexpr bool kHasW = MODE == kWgrad || MODE == kFusedStore || MODE == kFusedSwiglu;
+  static constexpr bool kHasD = MODE != kWgrad && MODE != kWgradGather;
+  static constexpr bool kHasW =
+      MODE == kWgrad || MODE == kFusedStore || MODE == kFusedSwiglu || MODE == kWgradGather;
   static constexpr bool kSwiglu = MODE == kDgradSwiglu || MODE == kFusedSwiglu;
+  static constexpr bool kGatherB = MODE == kWgradGather;
 };
 
 struct TileInfo {
@@ -268,7 +276,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full[i], 1);
+      // gathered B: the TMA arrival plus one cp.async arrival per producer lane
+      mbar_init(&full[i], Tr::kGatherB ? 33 : 1);
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -330,7 +339,85 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     return t;
   };
 
-  if (warp == 0) {
+  if (Tr::kGatherB && warp == 0) {
+    // ---------------- producer with gathered B (whole warp) ----------------
+    // lane 0 schedules tiles and loads A by TMA; all lanes gather B: 64 rows x 256
+    // columns per stage as 16-byte cp.async pieces written where a 128-byte
+    // swizzled TMA box would put them (row rr at rr * 128, piece c at c ^ (rr & 7))
+    if constexpr (Tr::kGatherB) {
+      int stage = 0;
+      uint32_t phase = 0;
+      unsigned int next = 0;
+      if (lane == 0) next = atomicAdd(&sched[0], 1u);
+      const int piece = lane & 7;
+      for (int it = 0;; ++it) {
+        const int slot = it % kRing;
+        int t = -1;
+        if (lane == 0) {
+          t = (int)next;
+          if (!mbar_wait_bounded(&ring_empty[slot], ((uint32_t)(it / kRing) & 1u) ^ 1u,
+                                 abort_flag, status) ||
+              t >= tc.total || *abort_flag)
+            t = -1;
+          ring[slot] = t;
+          mbar_arrive(&ring_full[slot]);
+        }
+        t = __shfl_sync(kFull, t, 0);
+        if (t < 0) break;
+        const TileInfo ti = decode_tile<MODE>(t, p, offs_s, tab_d, tab_w, tc);
+        if (ti.nk == 0 && lane == 0) next = atomicAdd(&sched[0], 1u);
+        bool ok = true;
+        for (int kb = 0; kb < ti.nk; ++kb) {
+          if (!__all_sync(kFull, mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag,
+                                                   status))) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * L::kStageBytes;
+          uint8_t* sb = sa + L::kABytes;
+          const int r0 = ti.row0 + kb * BK;
+          if (lane == 0) {
+            if (kb == ti.nk - 1) next = atomicAdd(&sched[0], 1u);
+            mbar_arrive_expect_tx(&full[stage], L::kABytes);
+            tma_load_2d(sa, &tmAw, &full[stage], ti.m0, r0);
+            tma_load_2d(sa + 8192, &tmAw, &full[stage], ti.m0 + 64, r0);
+          }
+          // perm of the block's 64 rows: lane l holds rows l and l + 32 (one round trip)
+          int pv[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int r = r0 + lane + 32 * h;
+            pv[h] = -1;
+            if (r < ti.row_end) {
+              const int pp = __ldg(p.perm + r);
+              if (pp >= 0 && pp < p.gperm_max)
+                pv[h] = pp / p.gdiv;
+              else
+                raise_status(status, LRMOE_ST_BAD_INDEX);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < BK / 4; ++i) {
+            const int rr = (lane >> 3) + 4 * i;  // row inside the K block
+            const long long srow = __shfl_sync(kFull, i < 8 ? pv[0] : pv[1], rr & 31);
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c) {
+              const int col = ti.n0 + c * 64 + piece * 8;
+              const bool in = srow >= 0 && col < p.N2;
+              const uint16_t* src = in ? p.gsrc + srow * p.N2 + col : p.gsrc;
+              cp_async_16(sb + c * 8192 + rr * 128 + ((piece ^ (rr & 7)) * 16), src, in ? 16u : 0u);
+            }
+          }
+          cp_async_arrive_noinc(&full[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 0) {
     // ---------------- TMA producer (and tile scheduler) ----------------
     if (lane == 0) {
       int stage = 0;
@@ -405,6 +492,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
           break;
         }
         tc_fence_after();
+        // gathered B was written by cp.async (generic proxy); the MMAs read it
+        // through the async proxy
+        if constexpr (Tr::kGatherB) fence_proxy_async_smem();
         uint8_t* sa = smem + stage * L::kStageBytes;
         uint8_t* sb = sa + L::kABytes;
         int nkk = BK / UK;  // MMAs of this K block
@@ -729,7 +819,7 @@ cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
   }
   m.aw = m.bw = m.out = m.ad;  // unused
   GemmParams prm{offsets, E, K, N, 0, 0, static_cast<const uint16_t*>(Gp),
-                 static_cast<const uint16_t*>(Up), perm, gu_rows, out, 0, status, 0};
+                 static_cast<const uint16_t*>(Up), perm, gu_rows, out, 0, nullptr, 1, 0, status, 0};
   if (epi == LRMOE_EPI_SWIGLU_BWD) return launch_mode<kDgradSwiglu>(m, prm, s, num_sms());
   return launch_mode<kDgradStore>(m, prm, s, num_sms());
 }
@@ -747,8 +837,28 @@ cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows
   int grid = num_sms();
   if (total < grid) grid = (int)total;
   GemmParams prm{offsets, E, 0, 0, N1, N2, nullptr, nullptr, nullptr, 0, nullptr, accumulate,
-                 status, 0};
+                 nullptr, 1, 0, status, 0};
   return launch_mode<kWgrad>(m, prm, s, grid);
+}
+
+cudaError_t launch_wgrad_gather_tc(const void* grad_rows, int rows_cap, const int32_t* perm,
+                                   const void* src, int src_div, int perm_max,
+                                   const int32_t* offsets, int E, int N1, int N2, float* dW,
+                                   int accumulate, uint32_t* status, cudaStream_t s,
+                                   const char** why) {
+  Maps m;
+  if (!make_map_2d(&m.aw, grad_rows, (uint64_t)rows_cap, (uint64_t)N1, 64, 64) ||
+      !make_map_out_f32(&m.out, dW, (uint64_t)E, (uint64_t)N1, (uint64_t)N2)) {
+    *why = "cuTensorMapEncodeTiled failed for a wgrad operand";
+    return cudaErrorInvalidValue;
+  }
+  m.ad = m.bd = m.bw = m.aw;  // unused
+  const long long total = (long long)E * ((N1 + BM - 1) / BM) * ((N2 + kBNT - 1) / kBNT);
+  int grid = num_sms();
+  if (total < grid) grid = (int)total;
+  GemmParams prm{offsets, E, 0, 0, N1, N2, nullptr, nullptr, perm, 0, nullptr, accumulate,
+                 static_cast<const uint16_t*>(src), src_div, perm_max, status, 0};
+  return launch_mode<kWgradGather>(m, prm, s, grid);
 }
 
 cudaError_t launch_dgrad_wgrad_tc(const void* grad_rows, int rows_cap, const void* W,
@@ -763,7 +873,8 @@ cudaError_t launch_dgrad_wgrad_tc(const void* grad_rows, int rows_cap, const voi
     return cudaErrorInvalidValue;
   }
   GemmParams prm{offsets, E, K, N, K, N2, static_cast<const uint16_t*>(Gp),
-                 static_cast<const uint16_t*>(Up), nullptr, 0, out, accumulate, status, 0};
+                 static_cast<const uint16_t*>(Up), nullptr, 0, out, accumulate, nullptr, 1, 0,
+                 status, 0};
   if (epi == LRMOE_EPI_SWIGLU_BWD) return launch_mode<kFusedSwiglu>(m, prm, s, num_sms());
   return launch_mode<kFusedStore>(m, prm, s, num_sms());
 }

@@ -107,6 +107,11 @@ cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
 cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows_cap,
                             const int32_t* offsets, int E, int N1, int N2, float* dW,
                             int accumulate, uint32_t* status, cudaStream_t s, const char** why);
+cudaError_t launch_wgrad_gather_tc(const void* grad_rows, int rows_cap, const int32_t* perm,
+                                   const void* src, int src_div, int perm_max,
+                                   const int32_t* offsets, int E, int N1, int N2, float* dW,
+                                   int accumulate, uint32_t* status, cudaStream_t s,
+                                   const char** why);
 cudaError_t launch_dgrad_wgrad_tc(const void* grad_rows, int rows_cap, const void* W,
                                   const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
                                   const void* Gp, const void* Up, void* out, const void* in_rows,

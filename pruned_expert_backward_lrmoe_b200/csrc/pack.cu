@@ -90,9 +90,9 @@ __global__ void __launch_bounds__(256) pack_kernel(
     const int t = p / k;
     const float wp = __ldg(w + p);
     const size_t rr = (size_t)r;
-    copy_row(Xp + rr * VH, x + (size_t)t * VH, VH, lane);
+    if (Xp) copy_row(Xp + rr * VH, x + (size_t)t * VH, VH, lane);  // X_p, A_p optional: the
     scale_row<DT>(DYp + rr * VH, dY + (size_t)t * VH, VH, wp, lane);
-    copy_row(Ap + rr * VI, a + (size_t)p * VI, VI, lane);
+    if (Ap) copy_row(Ap + rr * VI, a + (size_t)p * VI, VI, lane);  // wgrad can gather them
     if (Gp) copy_row(Gp + rr * VI, g + (size_t)p * VI, VI, lane);  // optional: the SwiGLU
     if (Up) copy_row(Up + rr * VI, u + (size_t)p * VI, VI, lane);  // epilogue can gather g, u
   }

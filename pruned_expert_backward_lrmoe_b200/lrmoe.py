@@ -28,7 +28,7 @@ EXPORTS = ("lrmoe_version", "lrmoe_status_string", "lrmoe_last_error", "lrmoe_sc
            "lrmoe_select_quota_noalloc", "lrmoe_selftest_bounded_wait", "lrmoe_quota_controller",
            "lrmoe_row_sqnorm", "lrmoe_score_from_norms", "lrmoe_router_grad",
            "lrmoe_redistribute", "lrmoe_split_by_destination", "lrmoe_grouped_dgrad_wgrad",
-           "lrmoe_grouped_dgrad_swiglu_gather")
+           "lrmoe_grouped_dgrad_swiglu_gather", "lrmoe_grouped_wgrad_gather")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -79,6 +79,7 @@ def load() -> ctypes.CDLL:
     lib.lrmoe_grouped_dgrad.argtypes = [P, I, P, P, I, I, I, I, I, P, P, P, P, P]
     lib.lrmoe_grouped_wgrad.argtypes = [P, P, I, P, I, I, I, I, P, I, P, P]
     lib.lrmoe_grouped_dgrad_swiglu_gather.argtypes = [P, I, P, P, I, I, I, I, P, P, P, I, P, P, P]
+    lib.lrmoe_grouped_wgrad_gather.argtypes = [P, I, P, P, I, I, P, I, I, I, I, P, I, P, P]
     lib.lrmoe_grouped_dgrad_wgrad.argtypes = [P, I, P, P, I, I, I, I, I, P, P, P, P, I, P, I, P, P]
     lib.lrmoe_unpack.argtypes = [P, I, P, I, I, I, I, P, P, P]
     lib.lrmoe_pruned_backward.argtypes = [ctypes.POINTER(lrmoe_buffers), I, I, I, I, I, I, I, P]
@@ -215,12 +216,16 @@ def lrmoe_select_quota_noalloc(topk_idx, score, quota, counts, kept, offsets, pe
 
 
 def lrmoe_pack(perm, offsets, topk_w, x, dY, a, g, u, Xp, DYp, Ap, Gp, Up, status=None,
-               stream=None) -> None:
+               stream=None, I: Optional[int] = None) -> None:
+    """Only dY/DYp are required; x/Xp, a/Ap and g, u/Gp, Up may be None (not packed)."""
     T, k = topk_w.shape
     E = offsets.numel() - 1
+    if I is None:
+        feat = next((t for t in (a, g, u, Ap, Gp, Up) if t is not None), None)
+        I = feat.shape[-1] if feat is not None else 8
     _check(load().lrmoe_pack(_ptr(perm), _ptr(offsets), _ptr(topk_w), T, k, E, _ptr(x), _ptr(dY),
-                             x.shape[-1], _ptr(a), _ptr(g), _ptr(u), a.shape[-1], _dt(x), _ptr(Xp),
-                             _ptr(DYp), _ptr(Ap), _ptr(Gp), _ptr(Up), Xp.shape[0], _ptr(status),
+                             dY.shape[-1], _ptr(a), _ptr(g), _ptr(u), I, _dt(dY), _ptr(Xp),
+                             _ptr(DYp), _ptr(Ap), _ptr(Gp), _ptr(Up), DYp.shape[0], _ptr(status),
                              _stream(stream)))
 
 
@@ -248,6 +253,16 @@ def lrmoe_grouped_dgrad_swiglu_gather(rows, W, offsets, perm, g, u, out, status=
                                                     _ptr(offsets), E, K, N, _dt(rows), _ptr(perm),
                                                     _ptr(g), _ptr(u), g.shape[0], _ptr(out),
                                                     _ptr(status), _stream(stream)))
+
+
+def lrmoe_grouped_wgrad_gather(grad_rows, perm, src, src_div: int, n_pairs: int, offsets, dW,
+                               accumulate: bool = False, status=None, stream=None) -> None:
+    """dW[e] = grad[R_e]^T . src[perm[r] / src_div] rows (bf16)."""
+    E, N1, N2 = dW.shape
+    _check(load().lrmoe_grouped_wgrad_gather(_ptr(grad_rows), grad_rows.shape[0], _ptr(perm),
+                                             _ptr(src), int(src_div), int(n_pairs), _ptr(offsets),
+                                             E, N1, N2, _dt(grad_rows), _ptr(dW), int(accumulate),
+                                             _ptr(status), _stream(stream)))
 
 
 def lrmoe_grouped_dgrad_wgrad(grad_rows, W, offsets, epilogue: int, out, in_rows, dW, Gp=None,

@@ -59,3 +59,56 @@ def test_pack_without_g_u_leaves_them_alone():
     M = int(out["offsets"][-1].item())
     for n in bufs:
         assert torch.equal(bufs[n][:M].view(torch.int16), out[n][:M].view(torch.int16)), n
+
+
+@pytest.mark.parametrize("name,over", [("qwen", dict(T=600, E=16, H=256, I=192)),
+                                       ("glm", dict(T=300, E=8, H=512, I=320)),
+                                       ("skew", dict(T=700, E=16, H=256, I=136)),
+                                       ("qwen", dict(T=64, E=32, H=128, I=64))])
+@pytest.mark.parametrize("accumulate", [False, True])
+def test_wgrad_gather_equals_packed(name, over, accumulate):
+    """dW_down from a[perm] and dW_gu from x[perm / k] equal the wgrads on packed rows."""
+    layer = inputs.make_layer(inputs.spec(name, **over), seed=19)
+    s = layer.spec
+    inp = PT.device_inputs(layer)
+    out = PT.run_steps(layer, inp)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for grad, src, div, packed, dw in (("DYp", inp["a"], 1, "Ap", "dW_down"),
+                                       ("dGUp", inp["x"], s.k, "Xp", "dW_gu")):
+        base = torch.randn_like(out[dw]) if accumulate else None
+        want = base.clone() if accumulate else torch.full_like(out[dw], float("nan"))
+        got = base.clone() if accumulate else torch.full_like(out[dw], float("nan"))
+        L.lrmoe_grouped_wgrad(out[grad], out[packed], out["offsets"], want, accumulate=accumulate,
+                              status=st)
+        L.lrmoe_grouped_wgrad_gather(out[grad], out["perm"], src, div, s.P, out["offsets"], got,
+                                     accumulate=accumulate, status=st)
+        torch.cuda.synchronize()
+        assert torch.equal(got.view(torch.int32), want.view(torch.int32)), dw
+    assert int(st.item()) == 0
+
+
+def test_wgrad_gather_flags_bad_perm_entries():
+    layer = inputs.make_layer(inputs.spec("qwen", T=200, E=8, H=128, I=64), seed=20)
+    s = layer.spec
+    inp = PT.device_inputs(layer)
+    out = PT.run_steps(layer, inp)
+    perm = out["perm"].clone()
+    perm[1] = -3
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dw = torch.empty_like(out["dW_down"])
+    L.lrmoe_grouped_wgrad_gather(out["DYp"], perm, inp["a"], 1, s.P, out["offsets"], dw, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & L.ST_BAD_INDEX
+    assert torch.isfinite(dw).all()
+
+
+def test_pack_dy_only():
+    layer = inputs.make_layer(inputs.spec("qwen", T=200, E=8, H=128, I=64), seed=21)
+    inp = PT.device_inputs(layer)
+    out = PT.run_steps(layer, inp)
+    dyp = torch.full_like(out["DYp"], float("nan"))
+    L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], None, inp["dY"], None, None, None,
+                 None, dyp, None, None, None, out["status"])
+    torch.cuda.synchronize()
+    M = int(out["offsets"][-1].item())
+    assert torch.equal(dyp[:M].view(torch.int16), out["DYp"][:M].view(torch.int16))
