@@ -98,6 +98,36 @@ __global__ void __launch_bounds__(256) pack_kernel(
   }
 }
 
+// acc += the 16-byte vector v (fp32 adds, element by element)
+template <lrmoe_dtype DT>
+__device__ __forceinline__ void add_vec(float (&acc)[DT == LRMOE_BF16 ? 8 : 4], const uint4& v) {
+  if constexpr (DT == LRMOE_BF16) {
+    const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc[2 * q] = __fadd_rn(acc[2 * q], bf16_bits_to_f32(ww[q] & 0xffffu));
+      acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_bits_to_f32(ww[q] >> 16));
+    }
+  } else {
+    acc[0] = __fadd_rn(acc[0], __uint_as_float(v.x));
+    acc[1] = __fadd_rn(acc[1], __uint_as_float(v.y));
+    acc[2] = __fadd_rn(acc[2], __uint_as_float(v.z));
+    acc[3] = __fadd_rn(acc[3], __uint_as_float(v.w));
+  }
+}
+
+// the sums rounded once to the storage type
+template <lrmoe_dtype DT>
+__device__ __forceinline__ uint4 to_vec(const float (&acc)[DT == LRMOE_BF16 ? 8 : 4]) {
+  if constexpr (DT == LRMOE_BF16) {
+    return make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                      pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+  } else {
+    return make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
+                      __float_as_uint(acc[3]));
+  }
+}
+
 // dX[t] = sum over retained slots j (ascending) of dXp[pos[t*k+j]], fp32, rounded once.
 template <lrmoe_dtype DT>
 __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ dXp, int rows_cap,
@@ -128,45 +158,29 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ d
         todo &= todo - 1;
       }
     }
-    for (int c = lane; c < VH; c += 32) {
+    // one 32-vector column chunk per pass, the retained rows' loads in flight together
+    // (the trip count is the same for every lane: the loop body shuffles)
+    for (int cb = 0; cb < VH; cb += 32) {
+      const int c = cb + lane;
+      const bool has = c < VH;
       float acc[PER];
 #pragma unroll
       for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
       for (int base = 0; base < nrows; base += kUnpackMaxRows) {
-        // all loads of this batch in flight before any add
         uint4 v[kUnpackMaxRows];
 #pragma unroll
         for (int i = 0; i < kUnpackMaxRows; ++i) {
           const int row = __shfl_sync(kFull, comp, (base + i) & 31);
-          v[i] = base + i < nrows ? __ldg(dXp + (size_t)row * VH + c) : make_uint4(0, 0, 0, 0);
+          v[i] = base + i < nrows && has ? __ldg(dXp + (size_t)row * VH + c)
+                                         : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int i = 0; i < kUnpackMaxRows; ++i) {
           if (base + i >= nrows) break;
-          if constexpr (DT == LRMOE_BF16) {
-            const uint32_t ww[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              acc[2 * q] = __fadd_rn(acc[2 * q], bf16_bits_to_f32(ww[q] & 0xffffu));
-              acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_bits_to_f32(ww[q] >> 16));
-            }
-          } else {
-            acc[0] = __fadd_rn(acc[0], __uint_as_float(v[i].x));
-            acc[1] = __fadd_rn(acc[1], __uint_as_float(v[i].y));
-            acc[2] = __fadd_rn(acc[2], __uint_as_float(v[i].z));
-            acc[3] = __fadd_rn(acc[3], __uint_as_float(v[i].w));
-          }
+          add_vec<DT>(acc, v[i]);
         }
       }
-      uint4 o;
-      if constexpr (DT == LRMOE_BF16) {
-        o = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-      } else {
-        o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
-                       __float_as_uint(acc[3]));
-      }
-      dX[(size_t)t * VH + c] = o;
+      if (has) dX[(size_t)t * VH + c] = to_vec<DT>(acc);
     }
   }
 }
