@@ -384,7 +384,7 @@ def make_runner(layer, dev):
         flush.sum()
     st = out["status"]
 
-    def step(ev=None, a_sqnorm=None, fused=False, wgrad_gather=False):
+    def step(ev=None, a_sqnorm=None, fused=False, wgrad_gather=False, waits=None):
         """One pass of the path; with a_sqnorm (||a_p||^2 saved by the forward) the
         score reads dY and the saved norms instead of a."""
         gather = s.dtype == "bf16" and not fused   # the path's g, u handling
@@ -444,6 +444,8 @@ def make_runner(layer, dev):
         calls = head + gemms + (
             lambda: L.lrmoe_unpack(out["dXp"], out["pos"], s.T, s.k, out["dX"], st, stream),)
         for i, c in enumerate(calls):
+            if waits and i in waits:
+                stream.wait_event(waits[i])
             if ev is not None:
                 ev[i].record(stream)
             c()
@@ -710,14 +712,27 @@ def run_gpu(args):
         n_e2e = max(3, min(args.steps, 50))
         e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(n_e2e)]
+        # Inputs go up on a copy stream in the order the path consumes them; the
+        # compute stream waits only where it needs each group (score and select:
+        # routing, dY, a; pack: x; the SwiGLU dgrad: g, u).
+        copy_stream = torch.cuda.Stream(dev)
+        groups = (("topk_idx", "topk_w", "quota", "dY", "a"), ("x",), ("g", "u"))
+        need_at = (0, 2, 3)   # step call index before which each group must have landed
         for i in range(n_e2e + 2):
             timed = i >= 2
             flush_l2()
             if timed:
                 e2e_ev[i - 2][0].record(stream)
-            for k_, v in pin.items():
-                inp[k_].copy_(v, non_blocking=True)
-            L.lrmoe_pruned_backward(inp, out, stream)
+            copy_stream.wait_stream(stream)   # the previous step is done with its inputs
+            landed = []
+            with torch.cuda.stream(copy_stream):
+                for grp in groups:
+                    for k_ in grp:
+                        inp[k_].copy_(pin[k_], non_blocking=True)
+                    ev_ = torch.cuda.Event()
+                    ev_.record(copy_stream)
+                    landed.append(ev_)
+            step(waits=dict(zip(need_at, landed)))
             dX_host.copy_(out["dX"], non_blocking=True)
             st_host.copy_(out["status"], non_blocking=True)
             if timed:
