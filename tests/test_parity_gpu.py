@@ -30,6 +30,9 @@ SMALL = {
     "full-quota": inputs.spec("qwen", T=256, E=4, k=2, H=128, I=64, quota="full"),
     "over-quota": inputs.spec("qwen", T=256, E=4, k=2, H=128, I=64, quota="over"),
     "zero-quota": inputs.spec("qwen", T=128, E=4, k=2, H=64, I=64, quota="zero"),
+    # the limits: E = 1024 experts (grouped-GEMM maximum; the wgrad then uses its
+    # 3-stage / 2-buffer layout; most experts empty) and top-32 routing (k maximum)
+    "max-sizes": inputs.spec("qwen", T=512, E=1024, k=32, H=64, I=64),
 }
 
 
