@@ -621,3 +621,35 @@ def test_split_by_destination_covers_each_global_run_once():
     for g in range(3):
         for e in range(3):
             assert got[(g, e)] == plan[e, g]
+
+
+def test_pruned_backward_equals_torch_autograd_on_the_retained_pairs():
+    """The pruned oracle equals torch autograd (fp64) of a forward that contains only
+    the retained pairs: dropping a pair from the backward is the same as dropping
+    its term from the layer output, for dW and for dX (library routine pin)."""
+    layer = small_layer("qwen", seed=23, T=24, E=4, k=2, H=16, I=8, dtype="f32",
+                        quota="half_ceil")
+    s = layer.spec
+    ref = O.pruned_backward(layer)
+    keep = ref["pos"] >= 0
+    x = torch.tensor(O.decode(layer.x, s.dtype), dtype=torch.float64, requires_grad=True)
+    Wgu = torch.tensor(O.decode(layer.W_gu, s.dtype), dtype=torch.float64, requires_grad=True)
+    Wd = torch.tensor(O.decode(layer.W_down, s.dtype), dtype=torch.float64, requires_grad=True)
+    dY = torch.tensor(O.decode(layer.dY, s.dtype), dtype=torch.float64)
+    w = torch.tensor(layer.topk_w, dtype=torch.float64)
+    Y = torch.zeros(s.T, s.H, dtype=torch.float64)
+    for t in range(s.T):
+        for j in range(s.k):
+            p = t * s.k + j
+            if not keep[p]:
+                continue
+            e = int(layer.topk_idx[t, j])
+            g = Wgu[e, : s.I] @ x[t]
+            u = Wgu[e, s.I:] @ x[t]
+            Y[t] = Y[t] + w[t, j] * (Wd[e] @ (torch.nn.functional.silu(g) * u))
+    (dY * Y).sum().backward()
+    # the oracle's packed gradient rows are fp32-rounded w * dY (storage f32):
+    # compare at the fp32 rounding level of that one product
+    assert rel_fro(ref["dW_down"], Wd.grad.numpy()) < 1e-6
+    assert rel_fro(ref["dW_gu"], Wgu.grad.numpy()) < 1e-6
+    assert rel_fro(ref["dX"], x.grad.numpy()) < 1e-6
