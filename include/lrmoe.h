@@ -222,6 +222,16 @@ int lrmoe_split_by_destination(const int32_t* perm, const int32_t* offsets, cons
                                int32_t* dest_expert_offsets, uint32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Row gather for the exchange of retained rows (RU-B bullet 5: rows move in
+ * compact blocks and come back to their original layout): dst[i] = src[idx[i]]
+ * for i < n, rows of row_bytes bytes (a multiple of 16), src [n_src][.],
+ * dst [n][.], idx [n] int32 device.  idx outside [0, n_src) sets
+ * LRMOE_ST_BAD_INDEX and leaves that dst row unwritten.  n = 0 is a no-op.
+ * ------------------------------------------------------------------------- */
+int lrmoe_gather_rows(const void* src, int n_src, int row_bytes, const int32_t* idx, int n,
+                      void* dst, uint32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Quota controller.  RU-B bullet 2, FR-B bullet 2, DE paragraph 3: before the
  * backward a controller sees how many tokens came to each expert and, within
  * the memory limit, fixes how many pairs of each expert stay for the layer

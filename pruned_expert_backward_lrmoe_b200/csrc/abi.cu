@@ -442,6 +442,21 @@ int lrmoe_grouped_dgrad_wgrad(const void* grad_rows, int rows_cap, const void* W
   return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, why);
 }
 
+int lrmoe_gather_rows(const void* src, int n_src, int row_bytes, const int32_t* idx, int n,
+                      void* dst, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(n >= 0 && n_src > 0, "n=%d must be >= 0 and n_src=%d positive", n, n_src);
+  REQUIRE(row_bytes > 0 && row_bytes % 16 == 0, "row_bytes=%d must be a positive multiple of 16",
+          row_bytes);
+  REQUIRE_PTR(src);
+  REQUIRE_PTR(idx);
+  REQUIRE_PTR(dst);
+  if (n == 0) return LRMOE_OK;
+  cudaError_t e = launch_gather_rows(src, n_src, row_bytes, idx, n, dst, status,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_gather_rows launch");
+}
+
 int lrmoe_unpack(const void* dXp, int rows_cap, const int32_t* pos, int T, int k, int H,
                  lrmoe_dtype dt, void* dX, uint32_t* status, void* stream) {
   g_last_error[0] = 0;

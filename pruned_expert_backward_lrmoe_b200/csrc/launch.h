@@ -47,6 +47,8 @@ cudaError_t launch_split_by_destination(const int32_t* perm, const int32_t* offs
                                         int rows_cap, int32_t* perm_dest, int32_t* dest_offsets,
                                         int32_t* dest_expert_offsets, uint32_t* status,
                                         cudaStream_t s);
+cudaError_t launch_gather_rows(const void* src, int n_src, int row_bytes, const int32_t* idx,
+                               int n, void* dst, uint32_t* status, cudaStream_t s);
 cudaError_t launch_row_sqnorm(const void* rows, int n, int D, lrmoe_dtype dt, float* out,
                               cudaStream_t s);
 cudaError_t launch_score_from_norms(const int32_t* idx, const float* w, int T, int k, int E,

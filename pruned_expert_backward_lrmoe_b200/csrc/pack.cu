@@ -185,7 +185,38 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ d
   }
 }
 
+// dst[i] = src[idx[i]] (rows of V 16-byte vectors); bad indices flagged, row skipped.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, int n_src,
+                                                          const int32_t* __restrict__ idx, int n,
+                                                          int V, uint4* __restrict__ dst,
+                                                          uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  pdl_wait();
+  pdl_trigger();
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n; i += gridDim.x * wpb) {
+    const int r = idx[i];
+    if (r < 0 || r >= n_src) {
+      if (lane == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
+      continue;
+    }
+    copy_row(dst + (size_t)i * V, src + (size_t)r * V, V, lane);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_gather_rows(const void* src, int n_src, int row_bytes, const int32_t* idx,
+                               int n, void* dst, uint32_t* status, cudaStream_t s) {
+  const int V = row_bytes / 16;
+  int blocks = (n + 7) / 8;
+  const int maxb = num_sms() * 8;
+  if (blocks > maxb) blocks = maxb;
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(256), 0, s,
+                    static_cast<const uint4*>(src), n_src, idx, n, V, static_cast<uint4*>(dst),
+                    status);
+}
 
 cudaError_t launch_pack(const int32_t* perm, const int32_t* offsets, const float* w, int T,
                         int k, int E, const void* x, const void* dY, int H, const void* a,

@@ -28,7 +28,7 @@ EXPORTS = ("lrmoe_version", "lrmoe_status_string", "lrmoe_last_error", "lrmoe_sc
            "lrmoe_select_quota_noalloc", "lrmoe_selftest_bounded_wait", "lrmoe_quota_controller",
            "lrmoe_row_sqnorm", "lrmoe_score_from_norms", "lrmoe_router_grad",
            "lrmoe_redistribute", "lrmoe_split_by_destination", "lrmoe_grouped_dgrad_wgrad",
-           "lrmoe_grouped_dgrad_swiglu_gather", "lrmoe_grouped_wgrad_gather")
+           "lrmoe_grouped_dgrad_swiglu_gather", "lrmoe_grouped_wgrad_gather", "lrmoe_gather_rows")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -80,6 +80,7 @@ def load() -> ctypes.CDLL:
     lib.lrmoe_grouped_wgrad.argtypes = [P, P, I, P, I, I, I, I, P, I, P, P]
     lib.lrmoe_grouped_dgrad_swiglu_gather.argtypes = [P, I, P, P, I, I, I, I, P, P, P, I, P, P, P]
     lib.lrmoe_grouped_wgrad_gather.argtypes = [P, I, P, P, I, I, P, I, I, I, I, P, I, P, P]
+    lib.lrmoe_gather_rows.argtypes = [P, I, I, P, I, P, P, P]
     lib.lrmoe_grouped_dgrad_wgrad.argtypes = [P, I, P, P, I, I, I, I, I, P, P, P, P, I, P, I, P, P]
     lib.lrmoe_unpack.argtypes = [P, I, P, I, I, I, I, P, P, P]
     lib.lrmoe_pruned_backward.argtypes = [ctypes.POINTER(lrmoe_buffers), I, I, I, I, I, I, I, P]
@@ -263,6 +264,15 @@ def lrmoe_grouped_wgrad_gather(grad_rows, perm, src, src_div: int, n_pairs: int,
                                              _ptr(src), int(src_div), int(n_pairs), _ptr(offsets),
                                              E, N1, N2, _dt(grad_rows), _ptr(dW), int(accumulate),
                                              _ptr(status), _stream(stream)))
+
+
+def lrmoe_gather_rows(src, idx, dst, status=None, stream=None) -> None:
+    """dst[i] = src[idx[i]] for the rows of 2-D tensors (row bytes a multiple of 16)."""
+    n = idx.numel()
+    if n == 0:
+        return
+    _check(load().lrmoe_gather_rows(_ptr(src), src.shape[0], src.shape[1] * src.element_size(),
+                                    _ptr(idx), n, _ptr(dst), _ptr(status), _stream(stream)))
 
 
 def lrmoe_grouped_dgrad_wgrad(grad_rows, W, offsets, epilogue: int, out, in_rows, dW, Gp=None,

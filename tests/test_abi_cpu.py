@@ -120,6 +120,14 @@ def test_fused_gemm_rejects_bad_arguments(lib):
     assert f(*bad) == L.LRMOE_ERR_UNSUPPORTED
 
 
+def test_gather_rows_rejects_bad_arguments(lib):
+    f = lib.lrmoe_gather_rows
+    assert f(FAKE, 10, 24, FAKE, 4, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG  # 24 % 16
+    assert f(NULL, 10, 32, FAKE, 4, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert f(FAKE, 0, 32, FAKE, 4, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+    assert f(FAKE, 10, 32, FAKE, 0, FAKE, NULL, NULL) == L.LRMOE_OK              # nothing to do
+
+
 def test_select_rejects_small_workspace(lib):
     f = lib.lrmoe_select_quota
     need = L.lrmoe_select_workspace_bytes(64, 2, 4)
