@@ -302,6 +302,20 @@ def host_cores() -> int:
         return os.cpu_count() or 1
 
 
+def host_cpu() -> dict:
+    """nproc and the CPU model name, reported beside every oracle timing."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count() or 1, "cpu_model": model}
+
+
 def run_reference(args):
     """The oracle on the host cores, one bounded expert sample per step."""
     rank = int(os.environ.get("RANK", "0"))
@@ -335,7 +349,8 @@ def run_reference(args):
         "config": config_block(s, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{group} expert(s) per step as standalone k=1 layers "
-                                   f"(score, selection, compaction, fp64 backward, unpack)"},
+                                   f"(score, selection, compaction, fp64 backward, unpack)",
+                         **host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -747,7 +762,7 @@ def run_gpu(args):
         secs, m_cpu = oracle_full_pass(layer)
         cpu = {"value": m_cpu / secs, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
                "sample": f"one full oracle pass over the {s.name} layer "
-                         f"({m_cpu} retained of {s.P} pairs), {secs:.1f} s"}
+                         f"({m_cpu} retained of {s.P} pairs), {secs:.1f} s", **host_cpu()}
 
     if dist is not None:
         dist.destroy_process_group()
