@@ -31,6 +31,8 @@ expert_backward  [RU-B] bullet 5: variable-size grouped GEMMs on those blocks
                  with no zero padding (here: plain fp64 matmuls per expert).
 unpack           [RU-B] bullet 5, last sentence: the result goes back to the
                  original layout.
+unpack_storage   the same return in the storage arithmetic the device uses
+                 (R12): fp32 sum in ascending slot order, one rounding.
 dense_backward   the ordinary unpruned SwiGLU MoE expert backward (textbook
                  calculus); used only to pin the pruned functions.
 forward          the ordinary SwiGLU MoE forward in fp64, used only by the
@@ -67,6 +69,9 @@ Readings where the pages are silent:
       for, it is <dY_t, y_p> with y_p saved by the forward, for every routed
       pair, or for the retained pairs only when pos is given (dropped pairs
       then get 0), in the canonical order below with x*x replaced by dY*y.
+  R12 returning dX_p to the token layout sums a token's retained rows in fp32,
+      starting from +0, in ascending slot order, and rounds once to the
+      storage dtype; a token with nothing retained gets +0.
 
 Canonical score order (R3), for one row v of D = V * VEC elements
 (VEC = 8 for bf16 storage, 4 for fp32):
@@ -525,6 +530,20 @@ def unpack(dXp, pos, T: int, k: int):
         keep = r >= 0
         dX[keep] += dXp[r[keep]]
     return dX
+
+
+def unpack_storage(dXp_stored, pos, T: int, k: int, dtype: str):
+    """dX in storage form from dX_p in storage form (R12): per token, acc = +0
+    in fp32, then acc = fl(acc + row) for the retained slots j = 0..k-1 in
+    order, then one round-to-nearest-even to the storage dtype."""
+    rows = decode(np.asarray(dXp_stored), dtype).astype(np.float32)
+    pos = np.asarray(pos).reshape(T, k)
+    acc = np.zeros((T, rows.shape[1]), dtype=np.float32)
+    for j in range(k):
+        r = pos[:, j]
+        keep = r >= 0
+        acc[keep] = acc[keep] + rows[r[keep]]    # float32 + float32: one IEEE rounding
+    return encode_rne(acc, dtype)
 
 
 # ----------------------------------------------------------------------------

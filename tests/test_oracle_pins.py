@@ -653,3 +653,58 @@ def test_pruned_backward_equals_torch_autograd_on_the_retained_pairs():
     assert rel_fro(ref["dW_down"], Wd.grad.numpy()) < 1e-6
     assert rel_fro(ref["dW_gu"], Wgu.grad.numpy()) < 1e-6
     assert rel_fro(ref["dX"], x.grad.numpy()) < 1e-6
+
+
+# ----------------------------------------------------------------------------
+# unpack in storage arithmetic (R12)
+# ----------------------------------------------------------------------------
+def _random_pos(rng, T, k, keep_frac):
+    """pos[T*k]: each kept slot gets a distinct packed row, the rest -1."""
+    keep = rng.random(T * k) < keep_frac
+    pos = np.full(T * k, -1, np.int32)
+    pos[keep] = rng.permutation(int(keep.sum())).astype(np.int32)
+    return pos, int(keep.sum())
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_unpack_storage_exact_on_dyadic_inputs(dtype):
+    """Multiples of 1/8 in [-1/2, 1/2]: every fp32 partial sum of up to 8 rows is
+    exact and so is its bf16 rounding, so the result equals the fp64 return."""
+    rng = np.random.default_rng(5)
+    T, k, H = 37, 8, 24
+    pos, M = _random_pos(rng, T, k, 0.4)
+    vals = (rng.integers(-4, 5, size=(M, H)) / 8.0).astype(np.float32)
+    stored = O.encode_rne(vals, dtype)
+    got = O.decode(O.unpack_storage(stored, pos, T, k, dtype), dtype)
+    want = O.unpack(vals.astype(np.float64), pos, T, k)
+    np.testing.assert_array_equal(got.astype(np.float64), want)
+
+
+def test_unpack_storage_sums_in_fp32_in_slot_order():
+    """1 + 2^-24 rounds to 1 (tie to even) in fp32, twice; the small rows first,
+    or an fp64 sum, would give 1 + 2^-23."""
+    rows = np.array([[1.0], [2.0 ** -24], [2.0 ** -24]], np.float32)
+    ascending = np.array([0, 1, 2], np.int32)
+    small_first = np.array([1, 2, 0], np.int32)
+    assert O.unpack_storage(rows, ascending, 1, 3, "f32")[0, 0] == np.float32(1.0)
+    assert O.unpack_storage(rows, small_first, 1, 3, "f32")[0, 0] == np.float32(1 + 2.0 ** -23)
+
+
+def test_unpack_storage_rounds_once_to_bf16():
+    """1 + 2^-8 + 2^-8 = 1 + 2^-7 exactly in fp32, a bf16 value; rounding after
+    each add would tie 1 + 2^-8 down to 1 and stay there."""
+    rows = O.encode_rne(np.array([[1.0], [2.0 ** -8], [2.0 ** -8]], np.float32), "bf16")
+    got = O.unpack_storage(rows, np.array([0, 1, 2], np.int32), 1, 3, "bf16")
+    assert O.decode(got, "bf16")[0, 0] == np.float32(1 + 2.0 ** -7)
+
+
+def test_unpack_storage_special_cases():
+    """k = 1 copies the row; nothing retained gives +0 bits; -0 rows give +0."""
+    rng = np.random.default_rng(6)
+    rows = O.encode_rne(rng.standard_normal((5, 16)).astype(np.float32), "bf16")
+    pos = np.array([3, -1, 0, 4, 1, 2], np.int32)
+    got = O.unpack_storage(rows, pos, 6, 1, "bf16")
+    for t, r in enumerate(pos):
+        np.testing.assert_array_equal(got[t], rows[r] if r >= 0 else np.zeros(16, np.uint16))
+    neg0 = np.full((1, 8), 0x8000, np.uint16)                 # bf16 -0.0
+    assert not O.unpack_storage(neg0, np.array([0], np.int32), 1, 1, "bf16").any()
