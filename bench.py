@@ -40,7 +40,7 @@ METRIC = "retained pairs/s + expert-bwd TFLOP/s on 1 B200; % of HBM / bf16 roofl
 UNIT = "retained pairs/s"
 DEFAULT_CONFIG = "qwen"
 KERNELS = ("score", "select", "pack", "dgrad_swiglu", "wgrad_down", "wgrad_gu", "dgrad_x", "unpack")
-KERNEL_LAUNCHES = {"score": 2, "select": 4, "pack": 1, "dgrad_swiglu": 1, "wgrad_down": 1,
+KERNEL_LAUNCHES = {"score": 1, "select": 4, "pack": 1, "dgrad_swiglu": 1, "wgrad_down": 1,
                    "wgrad_gu": 1, "dgrad_x": 1, "unpack": 1}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 

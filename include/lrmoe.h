@@ -114,7 +114,7 @@ int lrmoe_score(const int32_t* topk_idx, const float* topk_w, int T, int k, int 
  * the backward's score then reads dY and the saved norms instead of all of a
  * (T*H + 4*T*k bytes instead of T*H + T*k*I elements).  The pages describe no
  * such split; it changes no value: the two calls below give, bit for bit,
- * what lrmoe_score gives (which is itself these two kernels back to back).
+ * what lrmoe_score gives (every row norm takes the same order in each kernel).
  *
  * lrmoe_row_sqnorm: out[r] = ||rows[r]||^2 for r < n_rows, rows [n_rows][D] in
  *   dtype dt, out [n_rows] fp32, in the canonical order of lrmoe_score.

@@ -14,7 +14,7 @@
 namespace lrmoe {
 namespace {
 
-constexpr int kUnpackMaxRows = 8;  // retained rows of a token loaded together per column
+constexpr int kUnpackLoads = 8;  // a token's (column chunk, row) loads in flight together
 
 __device__ __forceinline__ void copy_row(uint4* __restrict__ dst, const uint4* __restrict__ src,
                                          int V, int lane) {
@@ -129,6 +129,10 @@ __device__ __forceinline__ uint4 to_vec(const float (&acc)[DT == LRMOE_BF16 ? 8 
 }
 
 // dX[t] = sum over retained slots j (ascending) of dXp[pos[t*k+j]], fp32, rounded once.
+// A token's loads form one list, column chunk by column chunk (32 vectors each),
+// retained rows in ascending slot order inside a chunk; the warp issues
+// kUnpackLoads of them at once, so a token with n retained rows needs about
+// ceil(n * chunks / kUnpackLoads) memory round trips rather than one per chunk.
 template <lrmoe_dtype DT>
 __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ dXp, int rows_cap,
                                                      const int32_t* __restrict__ pos, int T,
@@ -147,7 +151,6 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ d
       r = -1;
     }
     const unsigned have = __ballot_sync(kFull, r >= 0);
-    // retained rows in ascending slot order, compacted: rows[i] for i < nrows
     const int nrows = __popc(have);
     int comp = 0;  // lane i: packed row of the i-th retained slot (ascending slot order)
     {
@@ -158,29 +161,46 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ d
         todo &= todo - 1;
       }
     }
-    // one 32-vector column chunk per pass, the retained rows' loads in flight together
-    // (the trip count is the same for every lane: the loop body shuffles)
-    for (int cb = 0; cb < VH; cb += 32) {
-      const int c = cb + lane;
-      const bool has = c < VH;
-      float acc[PER];
+    uint4* __restrict__ out = dX + (size_t)t * VH;
+    if (nrows == 0) {
+      for (int c = lane; c < VH; c += 32) out[c] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    // item i = (chunk i / nrows, row i % nrows); nrows, items, ch and ri are warp-uniform
+    const int items = ((VH + 31) >> 5) * nrows;
+    float acc[PER];
 #pragma unroll
-      for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
-      for (int base = 0; base < nrows; base += kUnpackMaxRows) {
-        uint4 v[kUnpackMaxRows];
+    for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+    int ch = 0, ri = 0;  // chunk and row of item i0
+    for (int i0 = 0; i0 < items; i0 += kUnpackLoads) {
+      uint4 v[kUnpackLoads];
+      {
+        int c2 = ch, r2 = ri;
 #pragma unroll
-        for (int i = 0; i < kUnpackMaxRows; ++i) {
-          const int row = __shfl_sync(kFull, comp, (base + i) & 31);
-          v[i] = base + i < nrows && has ? __ldg(dXp + (size_t)row * VH + c)
-                                         : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int i = 0; i < kUnpackMaxRows; ++i) {
-          if (base + i >= nrows) break;
-          add_vec<DT>(acc, v[i]);
+        for (int q = 0; q < kUnpackLoads; ++q) {
+          const int row = __shfl_sync(kFull, comp, r2);
+          const int c = (c2 << 5) + lane;
+          v[q] = (i0 + q < items && c < VH) ? __ldg(dXp + (size_t)row * VH + c)
+                                            : make_uint4(0, 0, 0, 0);
+          if (++r2 == nrows) {
+            r2 = 0;
+            ++c2;
+          }
         }
       }
-      if (has) dX[(size_t)t * VH + c] = to_vec<DT>(acc);
+#pragma unroll
+      for (int q = 0; q < kUnpackLoads; ++q) {
+        if (i0 + q >= items) break;
+        add_vec<DT>(acc, v[q]);
+        if (++ri == nrows) {  // the chunk's last retained row: store, start the next chunk
+          const int c = (ch << 5) + lane;
+          if (c < VH) out[c] = to_vec<DT>(acc);
+#pragma unroll
+          for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+          ri = 0;
+          ++ch;
+        }
+      }
     }
   }
 }

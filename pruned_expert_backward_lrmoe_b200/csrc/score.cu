@@ -4,12 +4,15 @@
 // bullet 3: the squared norm of a pair's outer-product contribution factorises,
 // so each pair needs two row norms and three multiplies, never the H x I matrix.
 //
-// Two HBM-bound kernels:
-//   row_sqnorm        ||row||^2 of every row of a matrix (the saved a, T*k rows);
-//   score_from_norms  ||dY_t||^2 per token, then w^2 * ||dY_t||^2 * ||a_p||^2 per slot.
-// lrmoe_score runs both, parking ||a_p||^2 in the score buffer, which the second
-// kernel then overwrites slot by slot.  When the forward has saved ||a_p||^2
-// (it owns a when a is produced), only the second kernel runs and a is not read.
+// Three HBM-bound kernels:
+//   score_fused       lrmoe_score: per token ||dY_t||^2, then its k rows' ||a_p||^2,
+//                     then w^2 * ||dY_t||^2 * ||a_p||^2 per slot, in one pass;
+//   row_sqnorm        ||row||^2 of every row of a matrix (the forward can save
+//                     ||a_p||^2 with it while it owns a);
+//   score_from_norms  ||dY_t||^2 per token, then the product with a saved ||a_p||^2,
+//                     so that a is not read at all.
+// Every row norm takes the same order whichever kernel computes it, so the two
+// routes give the same bits.
 //
 // A warp reduces RPW rows at once with every 16-byte load of a row chunk in
 // flight together.  The order is fixed so that results are bit-reproducible:
@@ -94,6 +97,65 @@ __global__ void __launch_bounds__(256) score_norms_kernel(const int32_t* __restr
   }
 }
 
+// One warp per token: ||dY_t||^2 (8 vectors per lane per chunk), then the token's
+// k saved rows a_p, RA at a time (RA * VLI <= 24 vectors per lane in flight),
+// lane j keeping ||a_{t,j}||^2; then the product as in score_norms_kernel.
+template <lrmoe_dtype DT, int VLI, int RA>
+__global__ void __launch_bounds__(256) score_fused_kernel(const int32_t* __restrict__ idx,
+                                                          const float* __restrict__ w, int T,
+                                                          int k, int E,
+                                                          const uint4* __restrict__ dY, int VH,
+                                                          const uint4* __restrict__ a, int VI,
+                                                          float* __restrict__ score,
+                                                          uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  pdl_wait();
+  pdl_trigger();
+  for (long long t = gw; t < T; t += nw) {
+    const bool slot = lane < k;
+    const size_t p = (size_t)t * k + lane;
+    const int e = slot ? __ldg(idx + p) : -1;
+    const float wv = slot ? __ldg(w + p) : 0.0f;
+    float ny[1];
+    warp_row_norms<DT, 8, 1>(dY + t * VH, VH, 1, lane, ny);
+    float na = 0.0f;
+    for (int j0 = 0; j0 < k; j0 += RA) {
+      const int here = k - j0 < RA ? k - j0 : RA;
+      float nrm[RA];
+      warp_row_norms<DT, VLI, RA>(a + ((size_t)t * k + j0) * VI, VI, here, lane, nrm);
+#pragma unroll
+      for (int i = 0; i < RA; ++i)
+        if (lane == j0 + i) na = nrm[i];
+    }
+    if (__any_sync(kFull, slot && e >= E) && lane == 0) raise_status(status, LRMOE_ST_BAD_EXPERT);
+    float sc = 0.0f;
+    if (slot && e >= 0 && e < E) {
+      sc = __fmul_rn(__fmul_rn(__fmul_rn(wv, wv), ny[0]), na);
+      if (!isfinite(sc)) {
+        raise_status(status, LRMOE_ST_NONFINITE);
+        if (isnan(sc)) sc = __uint_as_float(0x7fffffffu);
+      }
+    }
+    if (slot) score[p] = sc;
+  }
+}
+
+template <lrmoe_dtype DT, int VLI>
+struct FusedF {
+  static cudaError_t run(const int32_t* idx, const float* w, int T, int k, int E, const void* dY,
+                         int VH, const void* a, int VI, float* score, uint32_t* status,
+                         cudaStream_t s) {
+    constexpr int RA = rpw_of<VLI>();
+    auto kern = score_fused_kernel<DT, VLI, RA>;
+    const int grid = grid_for(kern, T);
+    return launch_pdl(kern, dim3(grid), dim3(256), 0, s, idx, w, T, k, E,
+                      static_cast<const uint4*>(dY), VH, static_cast<const uint4*>(a), VI, score,
+                      status);
+  }
+};
+
 template <lrmoe_dtype DT, int VL>
 struct NormsF {
   static cudaError_t run(const void* rows, int n, int V, float* out, cudaStream_t s) {
@@ -138,9 +200,11 @@ cudaError_t launch_score_from_norms(const int32_t* idx, const float* w, int T, i
 cudaError_t launch_score(const int32_t* idx, const float* w, int T, int k, int E, const void* dY,
                          int H, const void* a, int D, lrmoe_dtype dt, float* score,
                          uint32_t* status, cudaStream_t s) {
-  cudaError_t e = launch_row_sqnorm(a, T * k, D, dt, score, s);
-  if (e != cudaSuccess) return e;
-  return launch_score_from_norms(idx, w, T, k, E, dY, H, score, dt, score, status, s);
+  const int per = dt == LRMOE_BF16 ? 8 : 4;
+  const int VH = H / per, VI = D / per;
+  if (dt == LRMOE_BF16)
+    return by_vl<LRMOE_BF16, FusedF>(VI, idx, w, T, k, E, dY, VH, a, VI, score, status, s);
+  return by_vl<LRMOE_F32, FusedF>(VI, idx, w, T, k, E, dY, VH, a, VI, score, status, s);
 }
 
 }  // namespace lrmoe
