@@ -90,8 +90,8 @@ struct RouterF {
                          cudaStream_t s) {
     // two rows (dY, y) per pair in flight: RPW*VL*2 <= 24 vectors per lane
     constexpr int RPW = rpw_of<2 * VL>();
-    auto kern = router_grad_kernel<DT, VL, RPW>;
-    const int grid = grid_for(kern, ((long long)P + 31) / 32);
+    constexpr auto kern = router_grad_kernel<DT, VL, RPW>;
+    const int grid = grid_for<kern>(((long long)P + 31) / 32);
     return launch_pdl(kern, dim3(grid), dim3(256), 0, s, idx, P, k, E,
                       static_cast<const uint4*>(dY), VH, static_cast<const uint4*>(y), pos, dw,
                       status);

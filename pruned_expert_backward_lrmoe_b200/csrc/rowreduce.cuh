@@ -6,6 +6,8 @@
 // o = 16, 8, 4, 2, 1; lane 0 (every lane) then holds the result.
 #pragma once
 
+#include <atomic>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -91,20 +93,19 @@ constexpr int rpw_of() {
 }
 
 // Grid: enough 8-warp blocks for the work, at most what is resident at once.
-template <typename Kern>
-int grid_for(Kern kern, long long warps_needed) {
-  static int per_sm[64] = {0};  // resident 256-thread blocks per SM, per device
+// The occupancy is looked up once per kernel (the template argument) and device.
+template <auto Kern>
+int grid_for(long long warps_needed) {
+  static std::atomic<int> per_sm[64];  // resident 256-thread blocks per SM; 0 = not known yet
   int dev = 0;
-  cudaGetDevice(&dev);
-  int occ = 1;
-  if (dev >= 0 && dev < 64) {
-    if (per_sm[dev] == 0) {
-      int n = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 256, 0) != cudaSuccess || n < 1)
-        n = 1;
-      per_sm[dev] = n;
-    }
-    occ = per_sm[dev];
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = -1;
+  int occ = dev >= 0 ? per_sm[dev].load(std::memory_order_relaxed) : 0;
+  if (occ == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kern, 256, 0) != cudaSuccess || n < 1)
+      n = 1;
+    occ = n;
+    if (dev >= 0) per_sm[dev].store(n, std::memory_order_relaxed);
   }
   const long long need = (warps_needed + 7) / 8;
   const long long cap = (long long)num_sms() * occ;

@@ -148,8 +148,8 @@ struct FusedF {
                          int VH, const void* a, int VI, float* score, uint32_t* status,
                          cudaStream_t s) {
     constexpr int RA = rpw_of<VLI>();
-    auto kern = score_fused_kernel<DT, VLI, RA>;
-    const int grid = grid_for(kern, T);
+    constexpr auto kern = score_fused_kernel<DT, VLI, RA>;
+    const int grid = grid_for<kern>(T);
     return launch_pdl(kern, dim3(grid), dim3(256), 0, s, idx, w, T, k, E,
                       static_cast<const uint4*>(dY), VH, static_cast<const uint4*>(a), VI, score,
                       status);
@@ -160,8 +160,8 @@ template <lrmoe_dtype DT, int VL>
 struct NormsF {
   static cudaError_t run(const void* rows, int n, int V, float* out, cudaStream_t s) {
     constexpr int RPW = rpw_of<VL>();
-    auto kern = row_sqnorm_kernel<DT, VL, RPW>;
-    const int grid = grid_for(kern, ((long long)n + RPW - 1) / RPW);
+    constexpr auto kern = row_sqnorm_kernel<DT, VL, RPW>;
+    const int grid = grid_for<kern>(((long long)n + RPW - 1) / RPW);
     return launch_pdl(kern, dim3(grid), dim3(256), 0, s, static_cast<const uint4*>(rows), n, V,
                       out);
   }
@@ -172,8 +172,8 @@ struct ScoreF {
   static cudaError_t run(const int32_t* idx, const float* w, int T, int k, int E, const void* dY,
                          int VH, const float* na, float* score, uint32_t* status, cudaStream_t s) {
     constexpr int RPW = rpw_of<VL>();
-    auto kern = score_norms_kernel<DT, VL, RPW>;
-    const int grid = grid_for(kern, ((long long)T + RPW - 1) / RPW);
+    constexpr auto kern = score_norms_kernel<DT, VL, RPW>;
+    const int grid = grid_for<kern>(((long long)T + RPW - 1) / RPW);
     return launch_pdl(kern, dim3(grid), dim3(256), 0, s, idx, w, T, k, E,
                       static_cast<const uint4*>(dY), VH, na, score, status);
   }
