@@ -1,6 +1,6 @@
 """Benchmark of the pruned MoE expert backward (LRMoE) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config qwen] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config sweep100] [--impl reference]
 
 A step is one pass of the whole hot path over one synthetic layer: LRM score,
 per-expert top-quota selection, compaction, the four grouped GEMMs (SwiGLU
@@ -9,6 +9,12 @@ C-ABI calls of liblrmoe.so on one stream.  The metric is retained pairs per
 second (plus expert-backward TFLOP/s of the grouped GEMMs), measured with CUDA
 events on the launching stream; inputs are resident in HBM and L2 is flushed
 between timed steps (a 512 MiB buffer written, then read back), outside the events.
+
+The headline layer is the largest single-GPU configuration: the GLM4.5-106B-A12B-
+shaped MoE layer with T = 16384 tokens, E = 128 experts, top-8, H = 4096,
+I = 1408, bf16, every routed pair kept (quota = count).  The Qwen3-30B-A3B- and
+GLM-shaped T = 8192 layers and the heavy-skew layer are timed after it in the
+same run and reported under "other_configs".
 
 N > 1 (torchrun, one process per GPU): every rank runs its own replica of the
 layer (the single-GPU path has no exchange step), the timed region is bracketed
@@ -38,10 +44,16 @@ if ROOT not in sys.path:
 
 METRIC = "retained pairs/s + expert-bwd TFLOP/s on 1 B200; % of HBM / bf16 roofline"
 UNIT = "retained pairs/s"
-DEFAULT_CONFIG = "qwen"
+DEFAULT_CONFIG = "sweep100"
+OTHER_CONFIGS = ("qwen", "glm", "skew")
 KERNELS = ("score", "select", "pack", "dgrad_swiglu", "wgrad_down", "wgrad_gu", "dgrad_x", "unpack")
 KERNEL_LAUNCHES = {"score": 1, "select": 4, "pack": 1, "dgrad_swiglu": 1, "wgrad_down": 1,
                    "wgrad_gu": 1, "dgrad_x": 1, "unpack": 1}
+# C-ABI call of each step position (NVTX range names)
+CALL_NAMES = ("lrmoe_score", "lrmoe_select_quota", "lrmoe_pack", "lrmoe_grouped_dgrad[swiglu]",
+              "lrmoe_grouped_wgrad[down]", "lrmoe_grouped_wgrad[gate|up]",
+              "lrmoe_grouped_dgrad[dX]", "lrmoe_unpack")
+FUSED_NAMES = ("lrmoe_grouped_dgrad_wgrad[swiglu,down]", "lrmoe_grouped_dgrad_wgrad[dX,gate|up]")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -60,6 +72,8 @@ def parse_args(argv=None):
     p.add_argument("--no-extras", action="store_true",
                    help="time only the step (profiling runs): no controller, fused-GEMM, "
                         "saved-norm, routing-gradient, redistribution or end-to-end blocks")
+    p.add_argument("--cpu-budget", type=float, default=20.0,
+                   help="seconds of host time for the bounded oracle sample (cpu_baseline)")
     p.add_argument("--override", default="",
                    help="layer fields to replace, e.g. T=4096,E=64 (smaller profiling cases)")
     return p.parse_args(argv)
@@ -117,38 +131,61 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def recorded_traffic(kernel: str, config: str):
-    """DRAM bytes per launch of `kernel` from a committed ncu summary, or None.
+# the sources that define each kernel whose DRAM traffic is recorded
+_GEMM_SOURCES = ("gemm_tc.cu", "common.cuh", "grouped.cuh", "launch.h")
+KERNEL_SOURCES = {
+    "score": ("score.cu", "rowreduce.cuh", "common.cuh"),
+    "select": ("select.cu", "common.cuh"),
+    "pack": ("pack.cu", "common.cuh"),
+    "unpack": ("pack.cu", "common.cuh"),
+    "dgrad_swiglu": _GEMM_SOURCES, "wgrad_down": _GEMM_SOURCES,
+    "wgrad_gu": _GEMM_SOURCES, "dgrad_x": _GEMM_SOURCES,
+}
+GEMM_SOURCES = _GEMM_SOURCES
 
-    profiles/traffic.json maps "<kernel>@<config>" to {"bytes": B, "source_sha1": S};
-    the figure is dropped when the kernel's sources (GEMM_SOURCES) changed since the
-    capture.
+
+def kernel_source_sha1(kernel: str = "wgrad_gu") -> str:
+    """sha1 over the source files that define `kernel` (name and bytes of each)."""
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "pruned_expert_backward_lrmoe_b200", "csrc")
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, config: str, algorithmic_bytes: float | None = None):
+    """DRAM bytes per launch of `kernel` on layer `config` from a committed ncu summary.
+
+    profiles/traffic.json maps "<kernel>@<layer>" to {"bytes": B, "source_sha1": S}
+    (captured on that layer), or to {"bytes": B, "algorithmic_bytes": A,
+    "scale_to": [layers], ...} for a capture on a smaller case of the same kernel,
+    which is scaled to a full launch of each listed layer as B / A x that launch's
+    algorithmic bytes.  Returns (bytes, how) or (None, reason); a figure is dropped
+    when the kernel's own sources changed since the capture.
     """
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             table = json.load(f)
     except (OSError, ValueError):
-        return None
+        return None, "no profiles/traffic.json"
+    sha = kernel_source_sha1(kernel)
     ent = table.get(f"{kernel}@{config}")
-    if not ent:
-        return None
-    if ent.get("source_sha1") != kernel_source_sha1():
-        return None
-    return ent.get("bytes")
-
-
-# the sources that define the grouped-GEMM kernels whose traffic is recorded
-GEMM_SOURCES = ("gemm_tc.cu", "common.cuh", "grouped.cuh", "launch.h")
-
-
-def kernel_source_sha1() -> str:
-    h = hashlib.sha1()
-    csrc = os.path.join(ROOT, "pruned_expert_backward_lrmoe_b200", "csrc")
-    for name in GEMM_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
-            h.update(f.read())
-    return h.hexdigest()
+    if ent:
+        if ent.get("source_sha1") != sha:
+            return None, "kernel changed since the capture"
+        return ent.get("bytes"), "ncu capture of this launch"
+    for key, ent in table.items():
+        if key.split("@")[0] != kernel or config not in ent.get("scale_to", ()):
+            continue
+        if ent.get("source_sha1") != sha:
+            return None, "kernel changed since the capture"
+        if algorithmic_bytes is None or not ent.get("algorithmic_bytes"):
+            return None, "no algorithmic bytes to scale by"
+        ratio = ent["bytes"] / ent["algorithmic_bytes"]
+        return ratio * algorithmic_bytes, f"scaled from the ncu capture {key} (traffic/algorithmic {ratio:.3f})"
+    return None, "not captured"
 
 
 # ---------------------------------------------------------------------------
@@ -295,11 +332,38 @@ def oracle_expert_sample(layer, experts):
 
 
 def host_cores() -> int:
+    """Threads the oracle's arithmetic runs on: numpy's BLAS pool (its matmuls are
+    the oracle's heavy steps), else torch's CPU thread count."""
+    try:
+        import threadpoolctl
+        for pool in threadpoolctl.threadpool_info():
+            if pool.get("user_api") == "blas":
+                return int(pool["num_threads"])
+    except Exception:
+        pass
     try:
         import torch
         return int(torch.get_num_threads())
     except Exception:
         return os.cpu_count() or 1
+
+
+def oracle_bounded_sample(layer, budget_s: float = 20.0):
+    """The oracle on a bounded sample of the layer: whole experts as standalone k = 1
+    layers (score, selection, compaction, fp64 backward, unpack), taken in the
+    order e = E/2, E/2 + 1, ... (wrapping), until about `budget_s` seconds of host
+    time are spent.  Returns (seconds, retained pairs, experts done)."""
+    E = layer.spec.E
+    tot_s, tot_m, done = 0.0, 0, []
+    for i in range(E):
+        if tot_s >= budget_s:
+            break
+        e = (E // 2 + i) % E
+        dt_, m = oracle_expert_sample(layer, [e])
+        tot_s += dt_
+        tot_m += m
+        done.append(e)
+    return tot_s, tot_m, done
 
 
 def host_cpu() -> dict:
@@ -357,9 +421,27 @@ def run_reference(args):
     return 0
 
 
+LAYER_SHAPES = {"tiny": "tiny fp32 MoE layer", "qwen": "Qwen3-30B-A3B-shaped MoE layer",
+                "glm": "GLM4.5-106B-A12B-shaped MoE layer",
+                "skew": "heavy-skew (Zipf 1.5) Qwen3-30B-A3B-shaped MoE layer",
+                "sweep": "GLM4.5-106B-A12B-shaped MoE layer"}
+
+
+def quota_rule(q: str) -> str:
+    if q.startswith("keep:"):
+        n, d = q[5:].split("/")
+        return "every routed pair kept (quota = count)" if n == d else \
+            f"keep {n}/{d} of each expert's pairs (quota = ceil({n}*count/{d}))"
+    return {"capacity": "quota = min(count, T*k/E)",
+            "skew": "quota = min(ceil(0.4*count), T*k/E)",
+            "half_ceil": "quota = ceil(count/2)"}.get(q, f"quota rule '{q}'")
+
+
 def config_block(s, n_gpus):
-    return {"workload": f"{s.name} MoE layer expert backward: T={s.T} E={s.E} top-{s.k} "
-                        f"H={s.H} I={s.I} {s.dtype}, quota rule '{s.quota}'",
+    base = next((v for k_, v in LAYER_SHAPES.items() if s.name.startswith(k_)), "MoE layer")
+    return {"workload": f"{base} ({s.name}), pruned expert backward: T={s.T} E={s.E} top-{s.k} "
+                        f"H={s.H} I={s.I} {s.dtype}, {quota_rule(s.quota)}",
+            "layer": s.name, "quota": s.quota,
             "T": s.T, "E": s.E, "k": s.k, "H": s.H, "I": s.I, "global_batch": s.T * n_gpus,
             "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
             "l2": "flushed between timed steps (512 MiB written, then read back); inputs also exceed L2"}
@@ -376,6 +458,7 @@ def make_runner(layer, dev):
 
     s = layer.spec
     tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
+    nvtx = torch.cuda.nvtx
 
     def storage(arr):
         if s.dtype == "bf16":
@@ -458,56 +541,74 @@ def make_runner(layer, dev):
             )
         calls = head + gemms + (
             lambda: L.lrmoe_unpack(out["dXp"], out["pos"], s.T, s.k, out["dX"], st, stream),)
+        names = CALL_NAMES if not fused else CALL_NAMES[:3] + FUSED_NAMES + CALL_NAMES[-1:]
         for i, c in enumerate(calls):
             if waits and i in waits:
                 stream.wait_event(waits[i])
             if ev is not None:
                 ev[i].record(stream)
+            nvtx.range_push(names[i])   # one NVTX range per C-ABI call
             c()
+            nvtx.range_pop()
         if ev is not None:
             ev[len(calls)].record(stream)
 
     return host, inp, out, stream, flush_l2, step
 
 
-def run_gpu(args):
+def roofline_of(kname, ms, by, fl, peaks, peak_src, layer_name):
+    """Roofline entry of one kernel: the bound (tensor when its flops per algorithmic
+    byte exceed the ridge of the peaks, else HBM), achieved = algorithmic flops or
+    bytes per launch / measured launch time, and the recorded DRAM traffic."""
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    ridge = tf * 1e12 / (hbm * 1e9)
+    flops, nbytes = fl.get(kname, 0), by[kname]
+    if flops and flops / nbytes > ridge:
+        ach = flops / (ms * 1e-3) / 1e12
+        bound, peak, unit, src = "tensor", tf, "TFLOP/s", f"{peak_src} bf16_tflops_sustained"
+    else:
+        ach = nbytes / (ms * 1e-3) / 1e9
+        bound, peak, unit, src = "hbm", hbm, "GB/s", f"{peak_src} hbm_gbs"
+    traffic, how = recorded_traffic(kname, layer_name, nbytes)
+    return {"kernel": kname, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+            "frac": ach / peak, "traffic": traffic, "traffic_source": how,
+            "peak_source": src, "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+            "flop_per_byte": flops / nbytes, "ridge_flop_per_byte": ridge, "ms": ms}
+
+
+def measure_layer(layer, dev, steps, warmup, dist, peaks, peak_src, breakdown_steps=None):
+    """Time K steps of the path on one layer (L2 flushed between steps), then a
+    second pass with events between the calls for per-kernel durations."""
     import torch
 
-    from pruned_expert_backward_lrmoe_b200 import inputs
-    from pruned_expert_backward_lrmoe_b200 import lrmoe as L
-
-    rank, world, local, dist = dist_setup(args.gpus)
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    layer = inputs.make_layer(layer_spec(args), seed=args.seed)
     s = layer.spec
-    tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
     b = 2 if s.dtype == "bf16" else 4
-    host, inp, out, stream, flush_l2, step = make_runner(layer, dev)
+    runner = make_runner(layer, dev)
+    host, inp, out, stream, flush_l2, step = runner
     st = out["status"]
     st.zero_()
-    for _ in range(max(1, args.warmup)):
+    for _ in range(max(1, warmup)):
         step()
     torch.cuda.synchronize(dev)
     if int(st.item()) != 0:
-        raise SystemExit(f"device status {int(st.item())} after warm-up")
+        raise SystemExit(f"device status {int(st.item())} after warm-up ({s.name})")
     M = int(out["offsets"][-1].item())
     counts = out["kept"].cpu().numpy()
 
-    # ---------------- device-timed region ----------------
     # Headline: K steps with events only around each step (events between the
     # kernels would stop each kernel's launch from overlapping its predecessor's
     # tail).  Then a second timed pass with events between the eight calls gives
     # the per-kernel durations used for the breakdown and the roofline.
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    n_bd = max(3, min(args.steps, 50))
+           for _ in range(steps)]
+    n_bd = breakdown_steps or max(3, min(steps, 50))
     evs_bd = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS) + 1)]
               for _ in range(n_bd)]
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index or 0) as clk:
         barrier(dist)
         torch.cuda.synchronize(dev)
-        for i in range(args.steps):
+        for i in range(steps):
             flush_l2()
             evs[i][0].record(stream)
             step()
@@ -519,6 +620,8 @@ def run_gpu(args):
             step(evs_bd[i])
         torch.cuda.synchronize(dev)
         barrier(dist)
+    if int(st.item()) != 0:
+        raise SystemExit(f"device status {int(st.item())} after the timed steps ({s.name})")
     per_kernel = {kname: [] for kname in KERNELS}
     for ev in evs_bd:
         for j, kname in enumerate(KERNELS):
@@ -527,272 +630,296 @@ def run_gpu(args):
     mean_step = statistics.fmean(step_ms)
     mean_step_max = max_over_ranks(mean_step, dist)
     M_all = sum_over_ranks(float(M), dist)
-    value = M_all / (mean_step_max * 1e-3)
     kern_ms = {kname: statistics.fmean(v) for kname, v in per_kernel.items()}
-
     by, fl = algorithmic(s.T, s.k, s.E, s.H, s.I, M, b)
     gemm_ms = sum(kern_ms[n] for n in step_gemms(fl))
     gemm_flops = sum(fl[n] for n in step_gemms(fl))
-    peaks, peak_src = load_peaks()
-    dominant = max(kern_ms, key=kern_ms.get)
-    dom_bytes = by[dominant]
-    achieved_gbs = dom_bytes / (kern_ms[dominant] * 1e-3) / 1e9
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    traffic = recorded_traffic(dominant, s.name)
-    roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
-                "unit": "GB/s", "frac": achieved_gbs / hbm_peak, "traffic": traffic,
-                "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes": dom_bytes}
+    tf_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     breakdown = {}
     for kname in KERNELS:
-        gbs = by[kname] / (kern_ms[kname] * 1e-3) / 1e9
-        e = {"ms": kern_ms[kname], "GB/s": gbs, "hbm_frac": gbs / hbm_peak}
+        r = roofline_of(kname, kern_ms[kname], by, fl, peaks, peak_src, s.name)
+        e = {"ms": kern_ms[kname], "bound": r["bound"], "frac": r["frac"],
+             "GB/s": by[kname] / (kern_ms[kname] * 1e-3) / 1e9}
+        e["hbm_frac"] = e["GB/s"] / hbm_peak
         if kname in fl:
-            tf = fl[kname] / (kern_ms[kname] * 1e-3) / 1e12
-            e["TFLOP/s"] = tf
-            e["tensor_frac"] = tf / float(peaks.get("bf16_tflops_sustained",
-                                                    FALLBACK_PEAKS["bf16_tflops_sustained"]))
+            e["TFLOP/s"] = fl[kname] / (kern_ms[kname] * 1e-3) / 1e12
+            e["tensor_frac"] = e["TFLOP/s"] / tf_peak
+        if r["traffic"] is not None:
+            e["traffic"] = r["traffic"]
         breakdown[kname] = e
+    dominant = max(kern_ms, key=kern_ms.get)
+    return {
+        "runner": runner, "M": M, "M_all": M_all, "counts": counts,
+        "ms_per_step": mean_step_max, "value": M_all / (mean_step_max * 1e-3),
+        "kern_ms": kern_ms, "breakdown": breakdown, "breakdown_steps": n_bd,
+        "breakdown_step_ms": sum(kern_ms.values()),
+        "gemm_ms": gemm_ms, "expert_bwd_tflops": gemm_flops / (gemm_ms * 1e-3) / 1e12,
+        "roofline": roofline_of(dominant, kern_ms[dominant], by, fl, peaks, peak_src, s.name),
+        "clocks": clk.summary(), "by": by, "fl": fl,
+    }
 
-    controller_us = controller_matches = fused_step_ms = wgrad_gather_step_ms = None
-    saved_norms = router = redistribution = None
-    e2e_value = e2e_ms = None
-    h2d = d2h = 0
-    if not args.no_extras:
-        # ---------------- quota controller (runs before the backward; not in the step) ----------------
-        q_dev = torch.empty(s.E, dtype=torch.int32, device=dev)
-        c_dev = torch.empty(s.E, dtype=torch.int32, device=dev)
-        cap = (s.T * s.k) // s.E
-        ctl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(20)]
-        for i in range(23):
-            if i >= 3:
-                ctl_ev[i - 3][0].record(stream)
-            L.lrmoe_quota_controller(inp["topk_idx"], s.E, cap, -1, q_dev, c_dev, st, stream)
-            if i >= 3:
-                ctl_ev[i - 3][1].record(stream)
-        torch.cuda.synchronize(dev)
-        controller_us = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in ctl_ev)
-        controller_matches = bool(torch.equal(q_dev, inp["quota"])) if s.quota == "capacity" else None
 
-        # ---------------- score from forward-saved ||a_p||^2 ----------------
-        # The forward can save ||a_p||^2 when it writes a; the backward's score then
-        # reads dY and 4 bytes per pair.  Timed per call after an L2 flush, and as
-        # whole steps with that score in place of the full one.
-        a2d = inp["a"].view(s.P, s.I)
-        na = torch.empty(s.P, dtype=torch.float32, device=dev)
-        L.lrmoe_row_sqnorm(a2d, na, stream)
-        sn_calls = {
-            "row_sqnorm": lambda: L.lrmoe_row_sqnorm(a2d, na, stream),
-            "score_from_norms": lambda: L.lrmoe_score_from_norms(
-                inp["topk_idx"], inp["topk_w"], inp["dY"], na, s.E, out["score"], st, stream),
-            "score": lambda: L.lrmoe_score(inp["topk_idx"], inp["topk_w"], inp["dY"], inp["a"], s.E,
-                                           out["score"], st, stream),
-        }
-        sn_us = {}
-        for name_, fn in sn_calls.items():
-            evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(20)]
-            for i in range(23):
-                flush_l2()
-                if i >= 3:
-                    evp[i - 3][0].record(stream)
-                fn()
-                if i >= 3:
-                    evp[i - 3][1].record(stream)
-            torch.cuda.synchronize(dev)
-            sn_us[name_] = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp)
-        sn_steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                    for _ in range(n_bd)]
-        for i in range(n_bd):
-            flush_l2()
-            sn_steps[i][0].record(stream)
-            step(a_sqnorm=na)
-            sn_steps[i][1].record(stream)
-        torch.cuda.synchronize(dev)
-        sn_step_ms = max_over_ranks(statistics.fmean(a_.elapsed_time(b_) for a_, b_ in sn_steps), dist)
-        sn_bytes = s.T * s.H * b + 16 * s.P          # dY, idx, w, saved norm, score
-        # the same steps with each dgrad and its wgrad fused into one launch
-        fu_steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                    for _ in range(n_bd)]
-        for i in range(n_bd):
-            flush_l2()
-            fu_steps[i][0].record(stream)
-            step(fused=True)
-            fu_steps[i][1].record(stream)
-        torch.cuda.synchronize(dev)
-        fused_step_ms = max_over_ranks(
-            statistics.fmean(a_.elapsed_time(b_) for a_, b_ in fu_steps), dist)
-        # ... and with the wgrads gathering a, x in place (only DY_p packed)
-        wg_steps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                    for _ in range(n_bd)]
-        for i in range(n_bd):
-            flush_l2()
-            wg_steps[i][0].record(stream)
-            step(wgrad_gather=True)
-            wg_steps[i][1].record(stream)
-        torch.cuda.synchronize(dev)
-        wgrad_gather_step_ms = max_over_ranks(
-            statistics.fmean(a_.elapsed_time(b_) for a_, b_ in wg_steps), dist)
-        saved_norms = {
-            "row_sqnorm_us": sn_us["row_sqnorm"], "score_from_norms_us": sn_us["score_from_norms"],
-            "score_us": sn_us["score"],
-            "score_from_norms_GB/s": sn_bytes / (sn_us["score_from_norms"] * 1e-6) / 1e9,
-            "score_from_norms_hbm_frac": sn_bytes / (sn_us["score_from_norms"] * 1e-6) / 1e9
-            / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
-            "step_ms": sn_step_ms, "value": M_all / (sn_step_ms * 1e-3), "unit": UNIT,
-            "steps": n_bd,
-        }
-        if int(st.item()) != 0:
-            raise SystemExit(f"device status {int(st.item())} after the saved-norm steps")
+def run_extras(layer, res, dev, args, dist, peaks):
+    """Blocks timed on the headline layer after the step: quota controller, score from
+    saved norms, fused and gathering GEMM variants, routing-weight gradient,
+    redistribution split, and the end-to-end number through host buffers."""
+    import torch
 
-        # ---------------- routing-weight gradient from saved expert outputs ----------------
-        # y_p = W_down[e] a_p is what the forward saves; it is generated here with torch
-        # (input generation, not part of the path), then dw = <dY_t, y_p> is timed for
-        # the retained pairs (pos from the selection) and for every routed pair.
-        y_dev = torch.empty(s.P, s.H, dtype=tdt, device=dev)
-        flat_idx = inp["topk_idx"].view(-1)
-        for e in range(s.E):
-            sel = (flat_idx == e).nonzero().squeeze(1)
-            if sel.numel():
-                y_dev[sel] = a2d[sel] @ inp["W_down"][e].T
-        dw = torch.empty(s.P, dtype=torch.float32, device=dev)
-        router = {}
-        for mode, pos_arg, nbytes in (
-                ("retained", out["pos"], M * s.H * b + s.T * s.H * b + 12 * s.P),
-                ("all", None, s.P * s.H * b + s.T * s.H * b + 8 * s.P)):
-            evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(20)]
-            for i in range(23):
-                flush_l2()
-                if i >= 3:
-                    evp[i - 3][0].record(stream)
-                L.lrmoe_router_grad(inp["topk_idx"], inp["dY"], y_dev, s.E, dw, pos=pos_arg,
-                                    status=st, stream=stream)
-                if i >= 3:
-                    evp[i - 3][1].record(stream)
-            torch.cuda.synchronize(dev)
-            us = 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp)
-            gbs = nbytes / (us * 1e-6) / 1e9
-            router[mode] = {"us": us, "GB/s": gbs,
-                            "hbm_frac": gbs / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
-                            "algorithmic_bytes": nbytes}
-        del y_dev
-        if int(st.item()) != 0:
-            raise SystemExit(f"device status {int(st.item())} after the router gradient")
+    from pruned_expert_backward_lrmoe_b200 import lrmoe as L
 
-        # ---------------- redistribution over expert copies (one rank's view) ----------------
-        # An 8-GPU copy map: expert e at home on GPU e % 8, the 16 most loaded experts with
-        # a second copy three GPUs on.  The host planner's time and peak against an even
-        # split and against home-only placement; then this rank's rows cut by the plan.
-        G_plan = 8
-        m_np = out["kept"].cpu().numpy().astype(np.int64)
-        adm = np.zeros((s.E, G_plan), bool)
-        adm[np.arange(s.E), np.arange(s.E) % G_plan] = True
-        hot = np.argsort(-m_np, kind="stable")[:16]
-        adm[hot, (hot + 3) % G_plan] = True
-        t0 = time.perf_counter()
-        plan, peak = L.lrmoe_redistribute(m_np, adm)
-        planner_us = (time.perf_counter() - t0) * 1e6
-        home = np.bincount(np.arange(s.E) % G_plan, weights=m_np, minlength=G_plan)
-        plan_dev = torch.from_numpy(plan.astype(np.int32)).to(dev)
-        pd = torch.empty(s.P, dtype=torch.int32, device=dev)
-        do = torch.empty(G_plan + 1, dtype=torch.int32, device=dev)
-        deo = torch.empty(G_plan, s.E + 1, dtype=torch.int32, device=dev)
+    s = layer.spec
+    b = 2 if s.dtype == "bf16" else 4
+    tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
+    host, inp, out, stream, flush_l2, step = res["runner"]
+    st = out["status"]
+    M, M_all, n_bd = res["M"], res["M_all"], res["breakdown_steps"]
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    x = {}
+
+    def timed(fn, n=20, warm=3, flush=True):
         evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(20)]
-        for i in range(23):
-            flush_l2()
-            if i >= 3:
-                evp[i - 3][0].record(stream)
-            L.lrmoe_split_by_destination(out["perm"], out["offsets"], plan_dev, pd, do, deo,
-                                         status=st, stream=stream)
-            if i >= 3:
-                evp[i - 3][1].record(stream)
+               for _ in range(n)]
+        for i in range(n + warm):
+            if flush:
+                flush_l2()
+            if i >= warm:
+                evp[i - warm][0].record(stream)
+            fn()
+            if i >= warm:
+                evp[i - warm][1].record(stream)
         torch.cuda.synchronize(dev)
-        redistribution = {
-            "gpus_in_plan": G_plan, "copies": int(adm.sum()), "planner_us": planner_us,
-            "peak": int(peak), "even_split": int(-(-int(m_np.sum()) // G_plan)),
-            "home_only_peak": int(home.max()),
-            "split_us": 1e3 * statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp),
-        }
-        if int(st.item()) != 0:
-            raise SystemExit(f"device status {int(st.item())} after the destination split")
+        return statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp)
 
-        # ---------------- end to end through host buffers ----------------
-        pin = {k_: v.pin_memory() for k_, v in host.items()}
-        dX_host = torch.empty(s.T, s.H, dtype=tdt).pin_memory()
-        st_host = torch.empty(1, dtype=torch.int32).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in pin.values())
-        d2h = dX_host.numel() * dX_host.element_size() + 4
-        n_e2e = max(3, min(args.steps, 50))
-        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(n_e2e)]
-        # Inputs go up on a copy stream in the order the path consumes them; the
-        # compute stream waits only where it needs each group (score and select:
-        # routing, dY, a; pack: x; the SwiGLU dgrad: g, u).
-        copy_stream = torch.cuda.Stream(dev)
-        groups = (("topk_idx", "topk_w", "quota", "dY", "a"), ("x",), ("g", "u"))
-        need_at = (0, 2, 3)   # step call index before which each group must have landed
-        for i in range(n_e2e + 2):
-            timed = i >= 2
+    # ---------------- quota controller (runs before the backward; not in the step) ----------------
+    q_dev = torch.empty(s.E, dtype=torch.int32, device=dev)
+    c_dev = torch.empty(s.E, dtype=torch.int32, device=dev)
+    cap = (s.T * s.k) // s.E
+    x["quota_controller_us"] = 1e3 * timed(
+        lambda: L.lrmoe_quota_controller(inp["topk_idx"], s.E, cap, -1, q_dev, c_dev, st, stream),
+        flush=False)
+    x["quota_controller_equals_capacity_rule"] = (
+        bool(torch.equal(q_dev, inp["quota"])) if s.quota == "capacity" else None)
+
+    # ---------------- score from forward-saved ||a_p||^2 ----------------
+    # The forward can save ||a_p||^2 when it writes a; the backward's score then
+    # reads dY and 4 bytes per pair.  Timed per call after an L2 flush, and as
+    # whole steps with that score in place of the full one.
+    a2d = inp["a"].view(s.P, s.I)
+    na = torch.empty(s.P, dtype=torch.float32, device=dev)
+    L.lrmoe_row_sqnorm(a2d, na, stream)
+    sn_us = {
+        "row_sqnorm": 1e3 * timed(lambda: L.lrmoe_row_sqnorm(a2d, na, stream)),
+        "score_from_norms": 1e3 * timed(lambda: L.lrmoe_score_from_norms(
+            inp["topk_idx"], inp["topk_w"], inp["dY"], na, s.E, out["score"], st, stream)),
+        "score": 1e3 * timed(lambda: L.lrmoe_score(inp["topk_idx"], inp["topk_w"], inp["dY"],
+                                                   inp["a"], s.E, out["score"], st, stream)),
+    }
+
+    def step_ms(**kw):
+        evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_bd)]
+        for i in range(n_bd):
             flush_l2()
-            if timed:
-                e2e_ev[i - 2][0].record(stream)
-            copy_stream.wait_stream(stream)   # the previous step is done with its inputs
-            landed = []
-            with torch.cuda.stream(copy_stream):
-                for grp in groups:
-                    for k_ in grp:
-                        inp[k_].copy_(pin[k_], non_blocking=True)
-                    ev_ = torch.cuda.Event()
-                    ev_.record(copy_stream)
-                    landed.append(ev_)
-            step(waits=dict(zip(need_at, landed)))
-            dX_host.copy_(out["dX"], non_blocking=True)
-            st_host.copy_(out["status"], non_blocking=True)
-            if timed:
-                e2e_ev[i - 2][1].record(stream)
+            evp[i][0].record(stream)
+            step(**kw)
+            evp[i][1].record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = statistics.fmean(a_.elapsed_time(b_) for a_, b_ in e2e_ev)
-        e2e_value = M_all / (max_over_ranks(e2e_ms, dist) * 1e-3)
+        return max_over_ranks(statistics.fmean(a_.elapsed_time(b_) for a_, b_ in evp), dist)
+
+    sn_step = step_ms(a_sqnorm=na)
+    sn_bytes = s.T * s.H * b + 16 * s.P          # dY, idx, w, saved norm, score
+    x["saved_norms"] = {
+        "row_sqnorm_us": sn_us["row_sqnorm"], "score_from_norms_us": sn_us["score_from_norms"],
+        "score_us": sn_us["score"],
+        "score_from_norms_GB/s": sn_bytes / (sn_us["score_from_norms"] * 1e-6) / 1e9,
+        "score_from_norms_hbm_frac": sn_bytes / (sn_us["score_from_norms"] * 1e-6) / 1e9 / hbm_peak,
+        "step_ms": sn_step, "value": M_all / (sn_step * 1e-3), "unit": UNIT, "steps": n_bd,
+    }
+    # the same steps with each dgrad and its wgrad fused into one launch, and with
+    # the wgrads gathering a, x in place (only DY_p packed)
+    x["fused_gemm_step_ms"] = step_ms(fused=True)
+    x["gathered_wgrad_step_ms"] = step_ms(wgrad_gather=True)
+    if int(st.item()) != 0:
+        raise SystemExit(f"device status {int(st.item())} after the variant steps")
+
+    # ---------------- routing-weight gradient from saved expert outputs ----------------
+    # y_p = W_down[e] a_p is what the forward saves; it is generated here with torch
+    # (input generation, not part of the path), then dw = <dY_t, y_p> is timed for
+    # the retained pairs (pos from the selection) and for every routed pair.
+    y_dev = torch.empty(s.P, s.H, dtype=tdt, device=dev)
+    flat_idx = inp["topk_idx"].view(-1)
+    for e in range(s.E):
+        sel = (flat_idx == e).nonzero().squeeze(1)
+        if sel.numel():
+            y_dev[sel] = a2d[sel] @ inp["W_down"][e].T
+    dw = torch.empty(s.P, dtype=torch.float32, device=dev)
+    router = {}
+    for mode, pos_arg, nbytes in (
+            ("retained", out["pos"], M * s.H * b + s.T * s.H * b + 12 * s.P),
+            ("all", None, s.P * s.H * b + s.T * s.H * b + 8 * s.P)):
+        us = 1e3 * timed(lambda: L.lrmoe_router_grad(inp["topk_idx"], inp["dY"], y_dev, s.E, dw,
+                                                     pos=pos_arg, status=st, stream=stream))
+        gbs = nbytes / (us * 1e-6) / 1e9
+        router[mode] = {"us": us, "GB/s": gbs, "hbm_frac": gbs / hbm_peak,
+                        "algorithmic_bytes": nbytes}
+    x["router_grad"] = router
+    del y_dev
+    if int(st.item()) != 0:
+        raise SystemExit(f"device status {int(st.item())} after the router gradient")
+
+    # ---------------- redistribution over expert copies (one rank's view) ----------------
+    # An 8-GPU copy map: expert e at home on GPU e % 8, the 16 most loaded experts with
+    # a second copy three GPUs on.  The host planner's time and peak against an even
+    # split and against home-only placement; then this rank's rows cut by the plan.
+    G_plan = 8
+    m_np = out["kept"].cpu().numpy().astype(np.int64)
+    adm = np.zeros((s.E, G_plan), bool)
+    adm[np.arange(s.E), np.arange(s.E) % G_plan] = True
+    hot = np.argsort(-m_np, kind="stable")[:16]
+    adm[hot, (hot + 3) % G_plan] = True
+    t0 = time.perf_counter()
+    plan, peak = L.lrmoe_redistribute(m_np, adm)
+    planner_us = (time.perf_counter() - t0) * 1e6
+    home = np.bincount(np.arange(s.E) % G_plan, weights=m_np, minlength=G_plan)
+    plan_dev = torch.from_numpy(plan.astype(np.int32)).to(dev)
+    pd = torch.empty(s.P, dtype=torch.int32, device=dev)
+    do = torch.empty(G_plan + 1, dtype=torch.int32, device=dev)
+    deo = torch.empty(G_plan, s.E + 1, dtype=torch.int32, device=dev)
+    split_ms = timed(lambda: L.lrmoe_split_by_destination(out["perm"], out["offsets"], plan_dev,
+                                                          pd, do, deo, status=st, stream=stream))
+    x["redistribution"] = {
+        "gpus_in_plan": G_plan, "copies": int(adm.sum()), "planner_us": planner_us,
+        "peak": int(peak), "even_split": int(-(-int(m_np.sum()) // G_plan)),
+        "home_only_peak": int(home.max()), "split_us": 1e3 * split_ms,
+    }
+    if int(st.item()) != 0:
+        raise SystemExit(f"device status {int(st.item())} after the destination split")
+    return x
+
+
+def run_e2e(layer, res, dev, args, dist):
+    """The same metric end to end: every step uploads its inputs from pinned host
+    memory (on a copy stream, in the order the path consumes them), runs the path
+    and reads dX and the status word back, all inside the timed region."""
+    import torch
+
+    s = layer.spec
+    tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
+    host, inp, out, stream, flush_l2, step = res["runner"]
+    pin = {k_: v.pin_memory() for k_, v in host.items()}
+    dX_host = torch.empty(s.T, s.H, dtype=tdt).pin_memory()
+    st_host = torch.empty(1, dtype=torch.int32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = dX_host.numel() * dX_host.element_size() + 4
+    n_e2e = max(3, min(args.steps, 50))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_e2e)]
+    # The compute stream waits only where it needs each group (score and select:
+    # routing, dY, a; pack: x; the SwiGLU dgrad: g, u).
+    copy_stream = torch.cuda.Stream(dev)
+    groups = (("topk_idx", "topk_w", "quota", "dY", "a"), ("x",), ("g", "u"))
+    need_at = (0, 2, 3)   # step call index before which each group must have landed
+    for i in range(n_e2e + 2):
+        timed = i >= 2
+        flush_l2()
+        if timed:
+            e2e_ev[i - 2][0].record(stream)
+        copy_stream.wait_stream(stream)   # the previous step is done with its inputs
+        landed = []
+        with torch.cuda.stream(copy_stream):
+            for grp in groups:
+                for k_ in grp:
+                    inp[k_].copy_(pin[k_], non_blocking=True)
+                ev_ = torch.cuda.Event()
+                ev_.record(copy_stream)
+                landed.append(ev_)
+        step(waits=dict(zip(need_at, landed)))
+        dX_host.copy_(out["dX"], non_blocking=True)
+        st_host.copy_(out["status"], non_blocking=True)
+        if timed:
+            e2e_ev[i - 2][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if int(st_host.item()) != 0:
+        raise SystemExit(f"device status {int(st_host.item())} after the end-to-end steps")
+    e2e_ms = max_over_ranks(statistics.fmean(a_.elapsed_time(b_) for a_, b_ in e2e_ev), dist)
+    return {"value": res["M_all"] / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e}
+
+
+def run_gpu(args):
+    import gc
+
+    import torch
+
+    from pruned_expert_backward_lrmoe_b200 import inputs
+
+    rank, world, local, dist = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    layer = inputs.make_layer(layer_spec(args), seed=args.seed)
+    s = layer.spec
+    res = measure_layer(layer, dev, args.steps, args.warmup, dist, peaks, peak_src)
+    extras = run_extras(layer, res, dev, args, dist, peaks) if not args.no_extras and world == 1 else {}
+    e2e = run_e2e(layer, res, dev, args, dist) if not args.no_extras else None
 
     # ---------------- CPU baseline (rank 0 at N = 1) ----------------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        secs, m_cpu = oracle_full_pass(layer)
+        secs, m_cpu, experts = oracle_bounded_sample(layer, budget_s=args.cpu_budget)
         cpu = {"value": m_cpu / secs, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
-               "sample": f"one full oracle pass over the {s.name} layer "
-                         f"({m_cpu} retained of {s.P} pairs), {secs:.1f} s", **host_cpu()}
+               "sample": f"{len(experts)} of the {s.E} experts of the {s.name} layer "
+                         f"(experts {experts[0]}..{experts[-1]}, {m_cpu} retained pairs), each "
+                         f"run as a standalone k=1 layer: score, selection, compaction, fp64 "
+                         f"backward, unpack; {secs:.1f} s", **host_cpu()}
+
+    # ---------------- the other configurations, after the headline ----------------
+    others = {}
+    if not args.no_extras and world == 1 and args.config == DEFAULT_CONFIG and not args.override:
+        del res["runner"]
+        gc.collect()
+        torch.cuda.empty_cache()
+        for name in OTHER_CONFIGS:
+            lay = inputs.make_layer(inputs.spec(name), seed=args.seed)
+            r = measure_layer(lay, dev, max(3, min(args.steps, 50)), max(3, args.warmup), dist,
+                              peaks, peak_src)
+            others[name] = {
+                "workload": config_block(lay.spec, world)["workload"],
+                "value": r["value"], "unit": UNIT, "ms_per_step": r["ms_per_step"],
+                "retained_pairs": r["M"], "routed_pairs": lay.spec.P,
+                "expert_bwd_tflops": r["expert_bwd_tflops"], "gemm_ms": r["gemm_ms"],
+                "roofline": r["roofline"],
+                "breakdown": {k_: {kk: v[kk] for kk in ("ms", "bound", "frac") if kk in v}
+                              for k_, v in r["breakdown"].items()},
+                "clocks": r["clocks"], "empty_experts": int((r["counts"] == 0).sum()),
+            }
+            del r, lay
+            gc.collect()
+            torch.cuda.empty_cache()
 
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return 0
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": mean_step_max, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
-        "config": config_block(s, world),
-        "retained_pairs": M, "routed_pairs": s.P,
-        "expert_bwd_tflops": gemm_flops / (gemm_ms * 1e-3) / 1e12,
-        "gemm_ms": gemm_ms,
-        "roofline": roofline,
-        "breakdown": breakdown,
-        "quota_controller_us": controller_us,
-        "quota_controller_equals_capacity_rule": controller_matches,
-        "fused_gemm_step_ms": fused_step_ms,
-        "gathered_wgrad_step_ms": wgrad_gather_step_ms,
-        "saved_norms": saved_norms,
-        "router_grad": router,
-        "redistribution": redistribution,
-        "breakdown_steps": n_bd,
-        "breakdown_step_ms": sum(kern_ms.values()),
+        "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": s.dtype,
+        "data": "synthetic", "config": config_block(s, world),
+        "retained_pairs": res["M"], "routed_pairs": s.P,
+        "expert_bwd_tflops": res["expert_bwd_tflops"], "gemm_ms": res["gemm_ms"],
+        "roofline": res["roofline"], "breakdown": res["breakdown"],
+        "breakdown_steps": res["breakdown_steps"], "breakdown_step_ms": res["breakdown_step_ms"],
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "e2e": e2e if e2e is not None else {"value": None, "unit": UNIT, "h2d_bytes_per_step": 0,
+                                            "d2h_bytes_per_step": 0},
         "gpu_launches": args.steps * sum(KERNEL_LAUNCHES.values()),
-        "clocks": clk.summary(),
-        "empty_experts": int((counts == 0).sum()),
+        "clocks": res["clocks"], "empty_experts": int((res["counts"] == 0).sum()),
+        "peaks": {k_: peaks.get(k_) for k_ in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")},
+        "peaks_source": peak_src,
+        **extras,
+        "other_configs": others,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -851,7 +978,7 @@ def run_sweep(args):
             "gemm_flop_per_byte": gemm_fl / gemm_bytes,
             "peaks": f"{peak_src}: bf16 {tf_peak} TFLOP/s sustained, HBM {hbm_peak} GB/s",
             "kernels_ms": kern, "clocks": clk.summary(), "steps": args.steps,
-            "config": config_block(s, 1)}), flush=True)
+            "config": config_block(inputs.spec(f"sweep{25 * n}"), 1)}), flush=True)
     xs = np.array([p[0] for p in points], np.float64)
     ys = np.array([p[1] for p in points], np.float64)
     slope, intercept = np.polyfit(xs, ys, 1)

@@ -262,11 +262,13 @@ int lrmoe_quota_controller(const int32_t* topk_idx, int T, int k, int E, int32_t
  * Same arguments (minus the workspace), same outputs and the same guarantees
  * as lrmoe_select_quota.  The scratch is a fixed array of
  * LRMOE_NOALLOC_SCRATCH_BYTES that the library keeps in device memory: every
- * GPU that loads the library holds it until the process exits.  The first
- * call on a device looks up that array's device address (once per device,
- * with the device current), so make the first call on each device before any
- * stream capture.  The call itself allocates nothing and calls no allocating
- * routine.  All calls on one device share the array: two calls whose kernels
+ * GPU that loads the library holds it until the process exits.  Every call
+ * asks the runtime for that array's device address in the context current on
+ * the calling thread (a host-side query that allocates nothing), so the
+ * address stays right across a reset of the device's context.  The first
+ * such query in a context also loads the library's device code, so make the
+ * first call on each device before any stream capture.  The call itself
+ * allocates nothing and calls no allocating routine.  All calls on one device share the array: two calls whose kernels
  * overlap on the GPU (different streams, no ordering between them) race and
  * give undefined results; calls on one stream are safe.  Nothing in the
  * array has to start at zero and its stale contents never affect a result.

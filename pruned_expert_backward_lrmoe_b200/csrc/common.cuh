@@ -120,6 +120,20 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Wait for phase `parity` of `bar` regardless of any abort flag, giving up after
+// `limit_ns`.  Used on the way out of a kernel to let asynchronous copies and
+// tensor-core work that are already in flight land before their shared or
+// tensor memory is released.  Returns false on give-up.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                                uint64_t limit_ns = 200000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0 && global_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tiled bulk tensor copies, no multicast)
 // ---------------------------------------------------------------------------
@@ -185,6 +199,11 @@ __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc, ui
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
                "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(src_bytes)
                : "memory");
+}
+
+// Wait until every cp.async this thread issued has landed.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // One arrival on `bar` once every cp.async this thread issued so far has landed

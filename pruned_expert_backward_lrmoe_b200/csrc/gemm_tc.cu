@@ -347,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     if constexpr (Tr::kGatherB) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and its phase
       unsigned int next = 0;
       if (lane == 0) next = atomicAdd(&sched[0], 1u);
       const int piece = lane & 7;
@@ -376,6 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
           uint8_t* sa = smem + stage * L::kStageBytes;
           uint8_t* sb = sa + L::kABytes;
           const int r0 = ti.row0 + kb * BK;
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (lane == 0) {
             if (kb == ti.nk - 1) next = atomicAdd(&sched[0], 1u);
             mbar_arrive_expect_tx(&full[stage], L::kABytes);
@@ -416,12 +419,20 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         }
         if (!ok) break;
       }
+      // Let every copy this warp started land before the CTA releases its shared
+      // memory (they are all consumed already unless a wait gave up).
+      cp_async_wait_all();
+      if (lane == 0)
+        for (int i = 0; i < STAGES; ++i)
+          if ((armed >> i) & 1u) mbar_wait_drain(&full[i], (armed_par >> i) & 1u);
+      __syncwarp();
     }
   } else if (warp == 0) {
     // ---------------- TMA producer (and tile scheduler) ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and its phase
       unsigned int next = atomicAdd(&sched[0], 1u);
       for (int it = 0;; ++it) {
         const int slot = it % kRing;
@@ -442,6 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
           if (kb == ti.nk - 1) next = atomicAdd(&sched[0], 1u);
           uint8_t* sa = smem + stage * L::kStageBytes;
           uint8_t* sb = sa + L::kABytes;
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
           if (ti.kind == 1) {
             if constexpr (Tr::kHasW) {
@@ -466,6 +479,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
           }
         }
       }
+      // Let every TMA load this CTA started land before its shared memory is
+      // released (after a normal run they have all been consumed already).
+      for (int i = 0; i < STAGES; ++i)
+        if ((armed >> i) & 1u) mbar_wait_drain(&full[i], (armed_par >> i) & 1u);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -544,10 +561,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
       __syncwarp();
       ++acc_iter;
     }
-    // make sure every issued MMA has finished before tensor memory is released
+    // make sure every issued MMA has finished before tensor memory is released,
+    // also when another role gave up a wait (the abort flag does not cut this short)
     if (lane == 0) tc_commit(mma_done);
     __syncwarp();
-    mbar_wait_bounded(mma_done, 0, abort_flag, status);
+    mbar_wait_drain(mma_done, 0);
   } else {
     // ---------------- epilogue (warps 2..9) ----------------
     // Two warps per TMEM lane quarter q = warp % 4; warp half h owns the 32-column
@@ -695,18 +713,19 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once per process.  The lookup runs
+// inside the initialiser of a function-local static, which C++ runs exactly
+// once even when several host threads make their first GEMM call together.
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -765,16 +784,11 @@ cudaError_t launch_variant(const Maps& m, GemmParams prm, cudaStream_t s, int gr
                 "shared memory over the sm_100 per-block limit");
   const int smem = L::alloc(prm.E);
   if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
-  static unsigned long long attr_done = 0;  // one bit per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tc<MODE, S, OB>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kSmemLimit);
-    if (err != cudaSuccess) return err;
-    attr_done |= 1ull << dev;
-  }
+  // Set on every launch (a host-side call, no device work): a cached "already
+  // set" flag would go stale when the device's context is reset and recreated.
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tc<MODE, S, OB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+  if (err != cudaSuccess) return err;
   prm.sched_slot = (int)(g_launches.fetch_add(1u) % kSchedSlots);
   return launch_pdl(grouped_gemm_tc<MODE, S, OB>, dim3(grid), dim3(kThreads), (size_t)smem, s,
                     m.ad, m.bd, m.aw, m.bw, m.out, prm);

@@ -17,8 +17,6 @@
 //                    largest key, then an ordered compaction that keeps keys
 //                    above the threshold and the first (m_e - #above) equal
 //                    keys in ascending p; writes perm and pos.
-#include <mutex>
-
 #include "common.cuh"
 #include "launch.h"
 
@@ -451,7 +449,19 @@ static cudaError_t enqueue_select(const SelectWs& L, const int32_t* idx, const f
                                   int32_t* offsets, int32_t* perm, int32_t* pos, int32_t* cc,
                                   int32_t* seg_start, int32_t* seg_p, uint32_t* seg_key,
                                   uint32_t* status, cudaStream_t s) {
-  cudaError_t e = launch_pdl(chunk_count, dim3(L.nchunks), dim3(kCountThreads), (size_t)E * 4, s,
+  // Shared-memory limits are set on every call (host-side calls, no device
+  // work), so that they hold in whatever context is current, also after a
+  // context reset, and no host-side flag is shared between threads.
+  cudaError_t e = cudaFuncSetAttribute(chunk_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (33 + 4096 + kScanSmemInts) * 4);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(chunk_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kScatterWarps * 4096 * 4);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(expert_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kTopkSmemKeys * 8);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(chunk_count, dim3(L.nchunks), dim3(kCountThreads), (size_t)E * 4, s,
                              idx, P, E, L.chunk, L.nchunks, cc, pos, status);
   if (e != cudaSuccess) return e;
   const bool fits = (size_t)E * L.nchunks <= (size_t)kScanSmemInts;
@@ -508,44 +518,21 @@ cudaError_t launch_select(const int32_t* idx, const float* score, int T, int k, 
   int32_t* seg_p = reinterpret_cast<int32_t*>(base + L.off_seg_p);
   uint32_t* seg_key = reinterpret_cast<uint32_t*>(base + L.off_seg_key);
 
-  static unsigned long long attrs_set = 0;  // one bit per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !((attrs_set >> dev) & 1ull)) {
-    cudaFuncSetAttribute(chunk_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (33 + 4096 + kScanSmemInts) * 4);
-    cudaFuncSetAttribute(chunk_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kScatterWarps * 4096 * 4);
-    cudaFuncSetAttribute(expert_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kTopkSmemKeys * 8);
-    attrs_set |= 1ull << dev;
-  }
   return enqueue_select(L, idx, score, P, E, quota, counts, kept, offsets, perm, pos, cc,
                         seg_start, seg_p, seg_key, status, s);
 }
 
-namespace {
-std::mutex g_scratch_mu;
-void* g_scratch_addr[64] = {nullptr};  // device address of g_select_scratch, per device ordinal
-}  // namespace
-
-// Device address of the built-in scratch array on the current device.  In
-// host code `g_select_scratch` names only a host-side stand-in, never device
-// memory; the real address comes from the runtime, once per device, with that
-// device current, and is cached here.
+// Device address of the built-in scratch array in the context current on this
+// thread.  In host code `g_select_scratch` names only a host-side stand-in,
+// never device memory; the real address comes from the runtime.  It is looked
+// up on every call (a host-side query that allocates nothing), so that it
+// stays right when the device's context is reset and the module is loaded
+// again at another address.  The first lookup in a context loads the module.
 static cudaError_t select_scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_select_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_select_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 
@@ -569,18 +556,6 @@ cudaError_t launch_select_noalloc(const int32_t* idx, const float* score, int T,
   int32_t* seg_p = reinterpret_cast<int32_t*>(base + L.off_seg_p);
   uint32_t* seg_key = reinterpret_cast<uint32_t*>(base + L.off_seg_key);
 
-  static unsigned long long attrs_set = 0;  // one bit per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !((attrs_set >> dev) & 1ull)) {
-    cudaFuncSetAttribute(chunk_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (33 + 4096 + kScanSmemInts) * 4);
-    cudaFuncSetAttribute(chunk_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kScatterWarps * 4096 * 4);
-    cudaFuncSetAttribute(expert_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kTopkSmemKeys * 8);
-    attrs_set |= 1ull << dev;
-  }
   return enqueue_select(L, idx, score, P, E, quota, counts, kept, offsets, perm, pos, cc,
                         seg_start, seg_p, seg_key, status, s);
 }

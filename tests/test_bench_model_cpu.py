@@ -25,21 +25,47 @@ def test_algorithmic_bytes_and_flops_hand_counted():
     assert by32["pack"] == 2 * M * (2 * H + 3 * I) * 4 + 8 * M
 
 
-def test_recorded_traffic_needs_the_current_gemm_sources(monkeypatch, tmp_path):
+def test_recorded_traffic_needs_the_kernels_current_sources(monkeypatch, tmp_path):
     prof = tmp_path / "profiles"
     prof.mkdir()
-    sha = bench.kernel_source_sha1()
-    (prof / "traffic.json").write_text(json.dumps(
-        {"wgrad_gu@qwen": {"bytes": 123, "source_sha1": sha}}))
-    monkeypatch.setattr(bench, "kernel_source_sha1", lambda: sha)
+    sha = bench.kernel_source_sha1("wgrad_gu")
+    (prof / "traffic.json").write_text(json.dumps({
+        "wgrad_gu@qwen": {"bytes": 123, "source_sha1": sha},
+        "unpack@qwen-T2048": {"bytes": 300, "algorithmic_bytes": 200, "source_sha1": "x",
+                              "scale_to": ["qwen"]}}))
+    assert bench.kernel_source_sha1("score") != bench.kernel_source_sha1("wgrad_gu")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.recorded_traffic("wgrad_gu", "qwen") == 123
-    assert bench.recorded_traffic("dgrad_x", "qwen") is None
-    monkeypatch.setattr(bench, "kernel_source_sha1", lambda: "0" * 40)
-    assert bench.recorded_traffic("wgrad_gu", "qwen") is None
+    monkeypatch.setattr(bench, "kernel_source_sha1", lambda k: sha if k == "wgrad_gu" else "x")
+    assert bench.recorded_traffic("wgrad_gu", "qwen")[0] == 123
+    assert bench.recorded_traffic("dgrad_x", "qwen")[0] is None
+    # a capture on a smaller case scales by the algorithmic bytes of the full launch
+    assert bench.recorded_traffic("unpack", "qwen", 1000.0)[0] == 1500.0
+    assert bench.recorded_traffic("unpack", "glm", 1000.0)[0] is None
+    monkeypatch.setattr(bench, "kernel_source_sha1", lambda k: "0" * 40)
+    assert bench.recorded_traffic("wgrad_gu", "qwen")[0] is None
+    assert bench.recorded_traffic("unpack", "qwen", 1000.0)[0] is None
 
 
-def test_committed_traffic_matches_the_committed_gemm_sources():
+def test_committed_traffic_entries_are_well_formed():
     with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
         table = json.load(f)
-    assert {e["source_sha1"] for e in table.values()} == {bench.kernel_source_sha1()}
+    for key, e in table.items():
+        kernel = key.split("@")[0]
+        assert kernel in bench.KERNEL_SOURCES, key
+        assert len(e["source_sha1"]) == 40 and e["bytes"] > 0, key
+        if "scale_to" in e:
+            assert e["algorithmic_bytes"] > 0, key
+
+
+def test_roofline_bound_follows_the_ridge():
+    peaks = dict(bench.FALLBACK_PEAKS)
+    T, k, E, H, I = 16384, 8, 128, 4096, 1408
+    by, fl = bench.algorithmic(T, k, E, H, I, T * k, 2)       # every pair kept
+    r = bench.roofline_of("wgrad_gu", 2.5, by, fl, peaks, "fallback", "sweep100")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["achieved"] - fl["wgrad_gu"] / 2.5e-3 / 1e12) < 1e-9
+    assert abs(r["frac"] - r["achieved"] / peaks["bf16_tflops_sustained"]) < 1e-12
+    by, fl = bench.algorithmic(8192, 8, 128, 2048, 768, 20427, 2)   # qwen-shaped, pruned
+    r = bench.roofline_of("wgrad_gu", 0.34, by, fl, peaks, "fallback", "qwen")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert bench.roofline_of("unpack", 0.03, by, fl, peaks, "fallback", "qwen")["bound"] == "hbm"

@@ -5,9 +5,11 @@ device scratch: a host framework or plugin host that owns all device memory
 and offers its extensions no allocator, or a latency-critical caller that must
 not call cudaMalloc/cudaFree because they can synchronise the device.  It uses
 a fixed scratch array inside the library instead.  Its outputs are integers, so
-the check against the workspace-taking entry point is bit-exact, on two calls
-in a row with different layers (stale scratch from the first call must not
-leak into the second), plus the refusal of a problem too large for the array.
+the check against the workspace-taking entry point is bit-exact, on calls in a
+row with different layers (stale scratch from an earlier call must not leak
+into a later one, also when a smaller layer follows a larger one), with the
+free device memory unchanged across them, plus the refusal of a problem too
+large for the array.
 
 This file is named so that pytest collects it last.
 """
@@ -47,9 +49,9 @@ def _reference(layer, inp, score):
     return ref
 
 
-def _noalloc(layer, inp, score):
+def _noalloc(layer, inp, score, out=None):
     s = layer.spec
-    out = _sel_buffers(s)
+    out = _sel_buffers(s) if out is None else out
     L.lrmoe_select_quota_noalloc(inp["topk_idx"], score, inp["quota"], out["counts"], out["kept"],
                                  out["offsets"], out["perm"], out["pos"], out["status"])
     return out
@@ -67,12 +69,23 @@ def test_noalloc_selection_matches_workspace_selection_twice():
     b = _scored(inputs.spec("qwen", T=4096, E=64, k=8, H=64, I=64), seed=1)
     ref_a = _reference(*a)
     ref_b = _reference(*b)
-    got_a = _noalloc(*a)          # first call: also looks up the scratch address
-    got_b = _noalloc(*b)          # second call in a row reuses the same scratch
+    # every output buffer exists before the no-alloc calls, so that the free
+    # device memory measured around them can only change if they allocate
+    outs = [_sel_buffers(a[0].spec), _sel_buffers(b[0].spec), _sel_buffers(a[0].spec)]
     torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    got_a = _noalloc(*a, out=outs[0])   # first call: also looks up the scratch address
+    got_b = _noalloc(*b, out=outs[1])   # second call in a row reuses the same scratch
+    # third call: the smaller layer again, after the larger one left its bytes
+    # beyond the smaller layout in the shared array
+    got_a2 = _noalloc(*a, out=outs[2])
+    torch.cuda.synchronize()
+    free_after = torch.cuda.mem_get_info()[0]
     _assert_same(got_a, ref_a)
     _assert_same(got_b, ref_b)
+    _assert_same(got_a2, ref_a)
     assert int(ref_b["offsets"][-1].item()) > 0
+    assert free_after == free_before, (free_before, free_after)
 
 
 def test_noalloc_refuses_problems_larger_than_its_array():
