@@ -211,15 +211,64 @@ int lrmoe_redistribute(const int64_t* m, const uint8_t* admissible, int E, int G
  *   dest_offsets [G+1]           start of each destination's block (last = M)
  *   dest_expert_offsets [G][E+1] expert offsets inside each block (the
  *                                receiver's grouped-GEMM offsets for this source)
- * lrmoe_pack(perm_dest, dest_offsets, ..., E = G, ...) then gathers the send
- * buffer (pack reads only offsets[E], the row count).  Rows that the plan
- * does not cover, and negative plan entries, set LRMOE_ST_BAD_INDEX; such rows
- * are left out.
+ *   row_dest [rows_cap]          (optional, NULL = not written) the send slot
+ *                                of each local packed row r < offsets[E]:
+ *                                perm_dest[row_dest[r]] = perm[r]; rows that come
+ *                                back in send order return to the packed layout
+ *                                with lrmoe_gather_rows(back, row_dest, ...)
+ * lrmoe_pack(perm_dest, dest_offsets, ..., E = G, ...) or lrmoe_pack_wide then
+ * gathers the send buffer (pack reads only offsets[E], the row count).  Rows
+ * that the plan does not cover, and negative plan entries, set
+ * LRMOE_ST_BAD_INDEX; such rows are left out.
  * ------------------------------------------------------------------------- */
 int lrmoe_split_by_destination(const int32_t* perm, const int32_t* offsets, const int32_t* plan,
                                const int32_t* global_start, int E, int G, int rows_cap,
                                int32_t* perm_dest, int32_t* dest_offsets,
-                               int32_t* dest_expert_offsets, uint32_t* status, void* stream);
+                               int32_t* dest_expert_offsets, int32_t* row_dest, uint32_t* status,
+                               void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Receiver's grouping.  RU-B bullet 5, FR-B bullet 5: the copy that receives
+ * rows from every source runs the grouped GEMMs on dense per-expert blocks.
+ *
+ * src_expert_offsets [G][E+1] int32 device: row q is source q's
+ * dest_expert_offsets row for this receiver (as exchanged by an all-to-all);
+ * the received rows are source-major (source q's block after those of
+ * sources < q, expert e's rows at [T[q][e], T[q][e+1]) inside it).  Writes
+ * (device, int32):
+ *   order [rows_cap]  grouped position i holds received row order[i]; grouped
+ *                     order = experts ascending, then sources in rank order,
+ *                     then arrival order
+ *   inv [rows_cap]    its inverse: received row j sits at grouped position inv[j]
+ *   offsets [E+1]     the grouped blocks' offsets (the receiver's GEMM offsets)
+ * for the R = sum_q T[q][E] received rows (R <= rows_cap; more, or a
+ * decreasing row of T, sets LRMOE_ST_BAD_INDEX).  E*G*4 <= 200 KB.
+ * ------------------------------------------------------------------------- */
+int lrmoe_group_received(const int32_t* src_expert_offsets, int G, int E, int rows_cap,
+                         int32_t* order, int32_t* inv, int32_t* offsets, uint32_t* status,
+                         void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Exchange rows.  RU-B bullet 5: the retained rows move in compact blocks.  One
+ * wide row per retained pair holds all five operands the receiver needs side by
+ * side, [x_t | RNE(w_p dY_t) | a_p | g_p | u_p] (2H + 3I elements, the same
+ * values lrmoe_pack writes), so that a single all-to-all moves them.
+ *
+ * lrmoe_pack_wide: like lrmoe_pack with every output present, into
+ * rows [rows_cap][2H+3I] (usually in the order of lrmoe_split_by_destination).
+ * lrmoe_split_wide: the receiver's gather and split: for i < n, the five
+ * column blocks of rows[idx[i]] go to X_p[i], DY_p[i] [.][H] and A_p[i],
+ * G_p[i], U_p[i] [.][I] (dense blocks for the grouped GEMMs; idx = order of
+ * lrmoe_group_received).  idx outside [0, n_src) sets LRMOE_ST_BAD_INDEX and
+ * leaves that row unwritten; n = 0 is a no-op.
+ * ------------------------------------------------------------------------- */
+int lrmoe_pack_wide(const int32_t* perm, const int32_t* offsets, const float* topk_w, int T, int k,
+                    int E, const void* x, const void* dY, int H, const void* a, const void* g,
+                    const void* u, int I, lrmoe_dtype dt, void* rows, int rows_cap,
+                    uint32_t* status, void* stream);
+int lrmoe_split_wide(const void* rows, int n_src, const int32_t* idx, int n, int H, int I,
+                     lrmoe_dtype dt, void* Xp, void* DYp, void* Ap, void* Gp, void* Up,
+                     uint32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Row gather for the exchange of retained rows (RU-B bullet 5: rows move in

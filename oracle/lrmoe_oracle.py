@@ -45,6 +45,10 @@ redistribute     [RU-B] bullet 4 / [FR-B] bullet 4: the remaining pairs of each
                  GPU; no new copies appear (R11).
 split_by_destination  [RU-B] bullet 5: retained rows are grouped by receiver
                  and expert, so the all-to-all moves compact blocks.
+send_positions   where each local packed row sits in that send order (the map
+                 that puts returned rows back in the local packed layout).
+group_received   the receiver's side of [RU-B] bullet 5: rows that arrived from
+                 every source, regrouped into one dense block per expert.
 router_grad      the gradient of the routing weights, dL/dw_p = <dY_t, y_p>
                  with y_p = W_down[e] a_p the pair's expert output (the layer
                  output is sum_j w_tj y_tj); the pages do not treat it (R8).
@@ -331,6 +335,45 @@ def split_by_destination(perm, offsets, plan, global_start=None):
         dest_offsets.append(len(perm_dest))
     return (np.asarray(perm_dest, np.int32), np.asarray(dest_offsets, np.int32),
             dest_expert_offsets)
+
+
+def send_positions(perm, perm_dest, M: int):
+    """Slot of each local packed row r < M in the destination-major send order of
+    split_by_destination: the i with perm_dest[i] = perm[r] (a pair id occurs
+    once).  The returned rows come back in send order, and this map puts each
+    one back at its local packed row."""
+    where = {}
+    for i in range(M):
+        where[int(perm_dest[i])] = i
+    return np.asarray([where[int(perm[r])] for r in range(M)], np.int32)
+
+
+def group_received(src_expert_offsets):
+    """Regroup received rows expert-major ([RU-B] bullet 5: the receiving copy runs
+    the grouped GEMMs on dense per-expert blocks).
+
+    The received rows are source-major: source q's block follows the blocks of
+    sources 0..q-1 and holds its rows of expert e at [T[q][e], T[q][e+1]) inside
+    the block (T = src_expert_offsets [G][E+1], each source's dest_expert_offsets
+    row for this receiver).  Grouped order: experts ascending, inside an expert
+    the sources in rank order, inside a source the arrival order.  Returns order
+    (grouped position i holds received row order[i]), inv (its inverse) and the
+    grouped offsets [E+1]."""
+    tab = np.asarray(src_expert_offsets, np.int64)
+    G, E = tab.shape[0], tab.shape[1] - 1
+    base = [0]
+    for q in range(G):
+        base.append(base[-1] + int(tab[q, E]))
+    order, offsets = [], [0]
+    for e in range(E):
+        for q in range(G):
+            order.extend(range(base[q] + int(tab[q, e]), base[q] + int(tab[q, e + 1])))
+        offsets.append(len(order))
+    inv = [0] * len(order)
+    for i, j in enumerate(order):
+        inv[j] = i
+    return (np.asarray(order, np.int32), np.asarray(inv, np.int32),
+            np.asarray(offsets, np.int32))
 
 
 def quota_controller(topk_idx, E: int, cap: int, max_pairs: int):

@@ -176,7 +176,8 @@ int lrmoe_redistribute(const int64_t* m, const uint8_t* admissible, int E, int G
 int lrmoe_split_by_destination(const int32_t* perm, const int32_t* offsets, const int32_t* plan,
                                const int32_t* global_start, int E, int G, int rows_cap,
                                int32_t* perm_dest, int32_t* dest_offsets,
-                               int32_t* dest_expert_offsets, uint32_t* status, void* stream) {
+                               int32_t* dest_expert_offsets, int32_t* row_dest, uint32_t* status,
+                               void* stream) {
   g_last_error[0] = 0;
   REQUIRE(E > 0 && E <= kMaxGroupedExperts, "E=%d must be in [1, %d]", E, kMaxGroupedExperts);
   REQUIRE(G > 0 && (size_t)E * G * sizeof(int) <= 200 * 1024, "G=%d out of range for E=%d", G, E);
@@ -188,10 +189,72 @@ int lrmoe_split_by_destination(const int32_t* perm, const int32_t* offsets, cons
   REQUIRE_PTR(dest_offsets);
   REQUIRE_PTR(dest_expert_offsets);
   REQUIRE(global_start == nullptr || aligned16(global_start), "global_start is not 16-byte aligned");
+  REQUIRE(row_dest == nullptr || aligned16(row_dest), "row_dest is not 16-byte aligned");
   cudaError_t e = launch_split_by_destination(perm, offsets, plan, global_start, E, G, rows_cap,
-                                              perm_dest, dest_offsets, dest_expert_offsets, status,
-                                              static_cast<cudaStream_t>(stream));
+                                              perm_dest, dest_offsets, dest_expert_offsets,
+                                              row_dest, status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_split_by_destination launch");
+}
+
+int lrmoe_group_received(const int32_t* src_expert_offsets, int G, int E, int rows_cap,
+                         int32_t* order, int32_t* inv, int32_t* offsets, uint32_t* status,
+                         void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(E > 0 && E <= kMaxGroupedExperts, "E=%d must be in [1, %d]", E, kMaxGroupedExperts);
+  REQUIRE(G > 0 && (size_t)E * G * sizeof(int) <= 200 * 1024, "G=%d out of range for E=%d", G, E);
+  REQUIRE(rows_cap > 0, "rows_cap=%d must be positive", rows_cap);
+  REQUIRE_PTR(src_expert_offsets);
+  REQUIRE_PTR(order);
+  REQUIRE_PTR(inv);
+  REQUIRE_PTR(offsets);
+  cudaError_t e = launch_group_received(src_expert_offsets, G, E, rows_cap, order, inv, offsets,
+                                        status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_group_received launch");
+}
+
+int lrmoe_pack_wide(const int32_t* perm, const int32_t* offsets, const float* topk_w, int T, int k,
+                    int E, const void* x, const void* dY, int H, const void* a, const void* g,
+                    const void* u, int I, lrmoe_dtype dt, void* rows, int rows_cap,
+                    uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  if (int r = check_pairs(T, k, E)) return r;
+  if (int r = check_feature(H, dt, "H")) return r;
+  if (int r = check_feature(I, dt, "I")) return r;
+  REQUIRE(rows_cap > 0, "rows_cap must be positive");
+  REQUIRE_PTR(perm);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(topk_w);
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(dY);
+  REQUIRE_PTR(a);
+  REQUIRE_PTR(g);
+  REQUIRE_PTR(u);
+  REQUIRE_PTR(rows);
+  cudaError_t e = launch_pack_wide(perm, offsets, topk_w, T, k, E, x, dY, H, a, g, u, I, dt, rows,
+                                   rows_cap, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_pack_wide launch");
+}
+
+int lrmoe_split_wide(const void* rows, int n_src, const int32_t* idx, int n, int H, int I,
+                     lrmoe_dtype dt, void* Xp, void* DYp, void* Ap, void* Gp, void* Up,
+                     uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(valid_dtype(dt), "unknown dtype %d", (int)dt);
+  REQUIRE(n >= 0 && n_src > 0, "n=%d must be >= 0 and n_src=%d positive", n, n_src);
+  if (int r = check_feature(H, dt, "H")) return r;
+  if (int r = check_feature(I, dt, "I")) return r;
+  REQUIRE_PTR(rows);
+  REQUIRE_PTR(idx);
+  REQUIRE_PTR(Xp);
+  REQUIRE_PTR(DYp);
+  REQUIRE_PTR(Ap);
+  REQUIRE_PTR(Gp);
+  REQUIRE_PTR(Up);
+  if (n == 0) return LRMOE_OK;
+  cudaError_t e = launch_split_wide(rows, n_src, idx, n, H, I, dt, Xp, DYp, Ap, Gp, Up, status,
+                                    static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_split_wide launch");
 }
 
 size_t lrmoe_select_workspace_bytes(int T, int k, int E) {

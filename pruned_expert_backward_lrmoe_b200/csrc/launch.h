@@ -45,8 +45,18 @@ int redistribute_plan(const int64_t* m, const uint8_t* adm, int E, int G, int64_
 cudaError_t launch_split_by_destination(const int32_t* perm, const int32_t* offsets,
                                         const int32_t* plan, const int32_t* start, int E, int G,
                                         int rows_cap, int32_t* perm_dest, int32_t* dest_offsets,
-                                        int32_t* dest_expert_offsets, uint32_t* status,
-                                        cudaStream_t s);
+                                        int32_t* dest_expert_offsets, int32_t* row_dest,
+                                        uint32_t* status, cudaStream_t s);
+cudaError_t launch_group_received(const int32_t* tab, int G, int E, int rows_cap, int32_t* order,
+                                  int32_t* inv, int32_t* offsets, uint32_t* status,
+                                  cudaStream_t s);
+cudaError_t launch_pack_wide(const int32_t* perm, const int32_t* offsets, const float* w, int T,
+                             int k, int E, const void* x, const void* dY, int H, const void* a,
+                             const void* g, const void* u, int I, lrmoe_dtype dt, void* rows,
+                             int rows_cap, uint32_t* status, cudaStream_t s);
+cudaError_t launch_split_wide(const void* rows, int n_src, const int32_t* idx, int n, int H, int I,
+                              lrmoe_dtype dt, void* Xp, void* DYp, void* Ap, void* Gp, void* Up,
+                              uint32_t* status, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* src, int n_src, int row_bytes, const int32_t* idx,
                                int n, void* dst, uint32_t* status, cudaStream_t s);
 cudaError_t launch_row_sqnorm(const void* rows, int n, int D, lrmoe_dtype dt, float* out,
@@ -109,6 +119,14 @@ cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
 cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows_cap,
                             const int32_t* offsets, int E, int N1, int N2, float* dW,
                             int accumulate, uint32_t* status, cudaStream_t s, const char** why);
+// the same GEMMs with one MMA per pair of SMs (two-CTA clusters, 256 x 256 tiles)
+cudaError_t launch_dgrad_pair(const void* rows, int rows_cap, const void* W,
+                              const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
+                              const void* Gp, const void* Up, void* out, uint32_t* status,
+                              cudaStream_t s, const char** why, const int32_t* perm, int gu_rows);
+cudaError_t launch_wgrad_pair(const void* grad_rows, const void* in_rows, int rows_cap,
+                              const int32_t* offsets, int E, int N1, int N2, float* dW,
+                              int accumulate, uint32_t* status, cudaStream_t s, const char** why);
 cudaError_t launch_wgrad_gather_tc(const void* grad_rows, int rows_cap, const int32_t* perm,
                                    const void* src, int src_div, int perm_max,
                                    const int32_t* offsets, int E, int N1, int N2, float* dW,

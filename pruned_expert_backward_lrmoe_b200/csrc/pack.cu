@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(256) pack_kernel(
     const uint4* __restrict__ dY, int VH, const uint4* __restrict__ a,
     const uint4* __restrict__ g, const uint4* __restrict__ u, int VI, uint4* __restrict__ Xp,
     uint4* __restrict__ DYp, uint4* __restrict__ Ap, uint4* __restrict__ Gp,
-    uint4* __restrict__ Up, int rows_cap, uint32_t* __restrict__ status) {
+    uint4* __restrict__ Up, int ldH, int ldI, int rows_cap, uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   pdl_wait();
@@ -90,11 +90,13 @@ __global__ void __launch_bounds__(256) pack_kernel(
     const int t = p / k;
     const float wp = __ldg(w + p);
     const size_t rr = (size_t)r;
-    if (Xp) copy_row(Xp + rr * VH, x + (size_t)t * VH, VH, lane);  // X_p, A_p optional: the
-    scale_row<DT>(DYp + rr * VH, dY + (size_t)t * VH, VH, wp, lane);
-    if (Ap) copy_row(Ap + rr * VI, a + (size_t)p * VI, VI, lane);  // wgrad can gather them
-    if (Gp) copy_row(Gp + rr * VI, g + (size_t)p * VI, VI, lane);  // optional: the SwiGLU
-    if (Up) copy_row(Up + rr * VI, u + (size_t)p * VI, VI, lane);  // epilogue can gather g, u
+    // output row strides: ldH for X_p, DY_p and ldI for A_p, G_p, U_p (16-byte
+    // vectors); VH and VI for dense blocks, the wide-row width for exchange rows
+    if (Xp) copy_row(Xp + rr * ldH, x + (size_t)t * VH, VH, lane);  // X_p, A_p optional: the
+    scale_row<DT>(DYp + rr * ldH, dY + (size_t)t * VH, VH, wp, lane);
+    if (Ap) copy_row(Ap + rr * ldI, a + (size_t)p * VI, VI, lane);  // wgrad can gather them
+    if (Gp) copy_row(Gp + rr * ldI, g + (size_t)p * VI, VI, lane);  // optional: the SwiGLU
+    if (Up) copy_row(Up + rr * ldI, u + (size_t)p * VI, VI, lane);  // epilogue can gather g, u
   }
 }
 
@@ -254,8 +256,72 @@ cudaError_t launch_pack(const int32_t* perm, const int32_t* offsets, const float
   auto kern = dt == LRMOE_BF16 ? pack_kernel<LRMOE_BF16> : pack_kernel<LRMOE_F32>;
   return launch_pdl(kern, dim3(blocks), dim3(256), 0, s, perm, offsets, E, w, T * k, k, X, D, VH,
                     A, G, U, VI, static_cast<uint4*>(Xp), static_cast<uint4*>(DYp),
-                    static_cast<uint4*>(Ap), static_cast<uint4*>(Gp), static_cast<uint4*>(Up),
-                    rows_cap, status);
+                    static_cast<uint4*>(Ap), static_cast<uint4*>(Gp), static_cast<uint4*>(Up), VH,
+                    VI, rows_cap, status);
+}
+
+// Exchange rows: packed row r = [x_t | RNE(w_p dY_t) | a_p | g_p | u_p] side by side
+// (2H + 3I elements), so that one all-to-all moves every operand of a pair.
+cudaError_t launch_pack_wide(const int32_t* perm, const int32_t* offsets, const float* w, int T,
+                             int k, int E, const void* x, const void* dY, int H, const void* a,
+                             const void* g, const void* u, int I, lrmoe_dtype dt, void* rows,
+                             int rows_cap, uint32_t* status, cudaStream_t s) {
+  const int per = dt == LRMOE_BF16 ? 8 : 4;
+  const int VH = H / per, VI = I / per;
+  const int W = 2 * VH + 3 * VI;
+  uint4* base = static_cast<uint4*>(rows);
+  const int blocks = num_sms() * 8;
+  auto kern = dt == LRMOE_BF16 ? pack_kernel<LRMOE_BF16> : pack_kernel<LRMOE_F32>;
+  return launch_pdl(kern, dim3(blocks), dim3(256), 0, s, perm, offsets, E, w, T * k, k,
+                    static_cast<const uint4*>(x), static_cast<const uint4*>(dY), VH,
+                    static_cast<const uint4*>(a), static_cast<const uint4*>(g),
+                    static_cast<const uint4*>(u), VI, base, base + VH, base + 2 * VH,
+                    base + 2 * VH + VI, base + 2 * VH + 2 * VI, W, W, rows_cap, status);
+}
+
+// dst operand rows i = the column blocks of exchange row idx[i] (bad indices
+// flagged, row skipped).
+__global__ void __launch_bounds__(256) split_wide_kernel(const uint4* __restrict__ rows, int n_src,
+                                                         const int32_t* __restrict__ idx, int n,
+                                                         int VH, int VI, uint4* __restrict__ Xp,
+                                                         uint4* __restrict__ DYp,
+                                                         uint4* __restrict__ Ap,
+                                                         uint4* __restrict__ Gp,
+                                                         uint4* __restrict__ Up,
+                                                         uint32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  const int W = 2 * VH + 3 * VI;
+  pdl_wait();
+  pdl_trigger();
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n; i += gridDim.x * wpb) {
+    const int r = idx[i];
+    if (r < 0 || r >= n_src) {
+      if (lane == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
+      continue;
+    }
+    const uint4* src = rows + (size_t)r * W;
+    const size_t ii = (size_t)i;
+    copy_row(Xp + ii * VH, src, VH, lane);
+    copy_row(DYp + ii * VH, src + VH, VH, lane);
+    copy_row(Ap + ii * VI, src + 2 * VH, VI, lane);
+    copy_row(Gp + ii * VI, src + 2 * VH + VI, VI, lane);
+    copy_row(Up + ii * VI, src + 2 * VH + 2 * VI, VI, lane);
+  }
+}
+
+cudaError_t launch_split_wide(const void* rows, int n_src, const int32_t* idx, int n, int H, int I,
+                              lrmoe_dtype dt, void* Xp, void* DYp, void* Ap, void* Gp, void* Up,
+                              uint32_t* status, cudaStream_t s) {
+  const int per = dt == LRMOE_BF16 ? 8 : 4;
+  int blocks = (n + 7) / 8;
+  const int maxb = num_sms() * 8;
+  if (blocks > maxb) blocks = maxb;
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(split_wide_kernel, dim3(blocks), dim3(256), 0, s,
+                    static_cast<const uint4*>(rows), n_src, idx, n, H / per, I / per,
+                    static_cast<uint4*>(Xp), static_cast<uint4*>(DYp), static_cast<uint4*>(Ap),
+                    static_cast<uint4*>(Gp), static_cast<uint4*>(Up), status);
 }
 
 cudaError_t launch_unpack(const void* dXp, int rows_cap, const int32_t* pos, int T, int k, int H,

@@ -19,6 +19,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "grouped.cuh"
 #include "launch.h"
 
 namespace lrmoe {
@@ -150,7 +151,8 @@ __global__ void __launch_bounds__(256) dest_scatter_kernel(
     const int32_t* __restrict__ perm, const int32_t* __restrict__ offsets,
     const int32_t* __restrict__ plan, const int32_t* __restrict__ start, int E, int G,
     int rows_cap, const int32_t* __restrict__ dest_offsets,
-    const int32_t* __restrict__ dest_expert_offsets, int32_t* __restrict__ perm_dest) {
+    const int32_t* __restrict__ dest_expert_offsets, int32_t* __restrict__ perm_dest,
+    int32_t* __restrict__ row_dest) {
   pdl_wait();
   pdl_trigger();
   int M = offsets[E];
@@ -172,11 +174,79 @@ __global__ void __launch_bounds__(256) dest_scatter_kernel(
         const long long first = base > c ? base : c;
         const long long slot = dest_offsets[g] + dest_expert_offsets[(size_t)g * (E + 1) + e] +
                                (gi - first);
-        if (slot < rows_cap) perm_dest[slot] = perm[r];
+        if (slot < rows_cap) {
+          perm_dest[slot] = perm[r];
+          if (row_dest) row_dest[r] = (int32_t)slot;
+        }
         break;
       }
       c = next;
     }
+  }
+}
+
+// Received rows (source-major blocks) regrouped expert-major.  Every CTA builds
+// the start of each (expert, source) block in grouped order in shared memory
+// (E * G entries, one block-wide scan), then places its share of the rows.
+__global__ void __launch_bounds__(1024) group_received_kernel(
+    const int32_t* __restrict__ tab /* [G][E+1] */, int G, int E, int rows_cap,
+    int32_t* __restrict__ order, int32_t* __restrict__ inv, int32_t* __restrict__ offsets,
+    uint32_t* __restrict__ status) {
+  extern __shared__ int sm[];  // gstart [E*G] (expert-major), base [G+1], scan scratch [33]
+  int* gstart = sm;
+  int* base = sm + (size_t)E * G;
+  int* scratch = base + G + 1;
+  pdl_wait();
+  pdl_trigger();
+  for (int i = threadIdx.x; i < E * G; i += blockDim.x) {
+    const int e = i / G, q = i - e * G;
+    const int32_t* row = tab + (size_t)q * (E + 1);
+    const int c = row[e + 1] - row[e];
+    if (c < 0 && blockIdx.x == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
+    gstart[i] = c > 0 ? c : 0;
+  }
+  __syncthreads();
+  const int total = block_scan_inplace(gstart, E * G, scratch);
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int q = 0; q < G; ++q) {
+      base[q] = run;
+      run += tab[(size_t)q * (E + 1) + E];
+    }
+    base[G] = run;
+    if (run != total && blockIdx.x == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = gstart[e * G];
+    if (threadIdx.x == 0) offsets[E] = total;
+  }
+  int R = base[G];
+  if (R > rows_cap || R > total) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
+    R = min(min(R, rows_cap), total);
+  }
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < R; j += gridDim.x * blockDim.x) {
+    int lo = 0, hi = G - 1;  // source of row j: largest q with base[q] <= j
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (base[mid] <= j) lo = mid; else hi = mid - 1;
+    }
+    const int q = lo;
+    const int l = j - base[q];
+    const int32_t* row = tab + (size_t)q * (E + 1);
+    int a = 0, b = E - 1;  // expert: largest e with row[e] <= l
+    while (a < b) {
+      const int mid = (a + b + 1) >> 1;
+      if (row[mid] <= l) a = mid; else b = mid - 1;
+    }
+    const int i = gstart[a * G + q] + (l - row[a]);
+    if (i < 0 || i >= R) {
+      raise_status(status, LRMOE_ST_BAD_INDEX);
+      continue;
+    }
+    order[i] = j;
+    inv[j] = i;
   }
 }
 
@@ -214,8 +284,8 @@ int redistribute_plan(const int64_t* m, const uint8_t* adm, int E, int G, int64_
 cudaError_t launch_split_by_destination(const int32_t* perm, const int32_t* offsets,
                                         const int32_t* plan, const int32_t* start, int E, int G,
                                         int rows_cap, int32_t* perm_dest, int32_t* dest_offsets,
-                                        int32_t* dest_expert_offsets, uint32_t* status,
-                                        cudaStream_t s) {
+                                        int32_t* dest_expert_offsets, int32_t* row_dest,
+                                        uint32_t* status, cudaStream_t s) {
   const size_t smem = (size_t)E * G * sizeof(int);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(dest_plan_kernel,
@@ -228,7 +298,23 @@ cudaError_t launch_split_by_destination(const int32_t* perm, const int32_t* offs
   const int blocks = num_sms() * 4;
   return launch_pdl(dest_scatter_kernel, dim3(blocks), dim3(256), 0, s, perm, offsets, plan, start,
                     E, G, rows_cap, (const int32_t*)dest_offsets,
-                    (const int32_t*)dest_expert_offsets, perm_dest);
+                    (const int32_t*)dest_expert_offsets, perm_dest, row_dest);
+}
+
+cudaError_t launch_group_received(const int32_t* tab, int G, int E, int rows_cap, int32_t* order,
+                                  int32_t* inv, int32_t* offsets, uint32_t* status,
+                                  cudaStream_t s) {
+  const size_t smem = ((size_t)E * G + G + 1 + 33) * sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(group_received_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  int blocks = (rows_cap + 1023) / 1024;
+  if (blocks > num_sms()) blocks = num_sms();
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(group_received_kernel, dim3(blocks), dim3(1024), smem, s, tab, G, E, rows_cap,
+                    order, inv, offsets, status);
 }
 
 }  // namespace lrmoe

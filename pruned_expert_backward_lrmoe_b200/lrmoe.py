@@ -28,7 +28,8 @@ EXPORTS = ("lrmoe_version", "lrmoe_status_string", "lrmoe_last_error", "lrmoe_sc
            "lrmoe_select_quota_noalloc", "lrmoe_selftest_bounded_wait", "lrmoe_quota_controller",
            "lrmoe_row_sqnorm", "lrmoe_score_from_norms", "lrmoe_router_grad",
            "lrmoe_redistribute", "lrmoe_split_by_destination", "lrmoe_grouped_dgrad_wgrad",
-           "lrmoe_grouped_dgrad_swiglu_gather", "lrmoe_grouped_wgrad_gather", "lrmoe_gather_rows")
+           "lrmoe_grouped_dgrad_swiglu_gather", "lrmoe_grouped_wgrad_gather", "lrmoe_gather_rows",
+           "lrmoe_group_received", "lrmoe_pack_wide", "lrmoe_split_wide")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -67,7 +68,10 @@ def load() -> ctypes.CDLL:
     lib.lrmoe_row_sqnorm.argtypes = [P, I, I, I, P, P]
     lib.lrmoe_router_grad.argtypes = [P, I, I, I, P, I, P, I, P, P, P, P]
     lib.lrmoe_redistribute.argtypes = [P, P, I, I, P, P]
-    lib.lrmoe_split_by_destination.argtypes = [P, P, P, P, I, I, I, P, P, P, P, P]
+    lib.lrmoe_split_by_destination.argtypes = [P, P, P, P, I, I, I, P, P, P, P, P, P]
+    lib.lrmoe_group_received.argtypes = [P, I, I, I, P, P, P, P, P]
+    lib.lrmoe_pack_wide.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, I, I, P, I, P, P]
+    lib.lrmoe_split_wide.argtypes = [P, I, P, I, I, I, I, P, P, P, P, P, P, P]
     lib.lrmoe_score_from_norms.argtypes = [P, P, I, I, I, P, I, P, I, P, P, P]
     lib.lrmoe_select_workspace_bytes.argtypes = [I, I, I]
     lib.lrmoe_select_workspace_bytes.restype = Z
@@ -174,13 +178,43 @@ def lrmoe_redistribute(m, admissible):
 
 
 def lrmoe_split_by_destination(perm, offsets, plan, perm_dest, dest_offsets, dest_expert_offsets,
-                               global_start=None, status=None, stream=None) -> None:
+                               global_start=None, status=None, stream=None,
+                               row_dest=None) -> None:
     E, G = plan.shape
     _check(load().lrmoe_split_by_destination(_ptr(perm), _ptr(offsets), _ptr(plan),
                                              _ptr(global_start), E, G, perm.shape[0],
                                              _ptr(perm_dest), _ptr(dest_offsets),
-                                             _ptr(dest_expert_offsets), _ptr(status),
-                                             _stream(stream)))
+                                             _ptr(dest_expert_offsets), _ptr(row_dest),
+                                             _ptr(status), _stream(stream)))
+
+
+def lrmoe_group_received(src_expert_offsets, order, inv, offsets, status=None,
+                         stream=None) -> None:
+    """Received rows (source-major) regrouped expert-major: order, inv, offsets."""
+    G, E1 = src_expert_offsets.shape
+    _check(load().lrmoe_group_received(_ptr(src_expert_offsets), G, E1 - 1, order.numel(),
+                                       _ptr(order), _ptr(inv), _ptr(offsets), _ptr(status),
+                                       _stream(stream)))
+
+
+def lrmoe_pack_wide(perm, offsets, topk_w, x, dY, a, g, u, rows, status=None, stream=None) -> None:
+    """rows[r] = [x_t | RNE(w_p dY_t) | a_p | g_p | u_p] for packed rows r < offsets[-1]."""
+    T, k = topk_w.shape
+    E = offsets.numel() - 1
+    _check(load().lrmoe_pack_wide(_ptr(perm), _ptr(offsets), _ptr(topk_w), T, k, E, _ptr(x),
+                                  _ptr(dY), dY.shape[-1], _ptr(a), _ptr(g), _ptr(u), a.shape[-1],
+                                  _dt(dY), _ptr(rows), rows.shape[0], _ptr(status),
+                                  _stream(stream)))
+
+
+def lrmoe_split_wide(rows, idx, Xp, DYp, Ap, Gp, Up, status=None, stream=None) -> None:
+    """The five column blocks of rows[idx[i]] into X_p[i], DY_p[i], A_p[i], G_p[i], U_p[i]."""
+    n = idx.numel()
+    if n == 0:
+        return
+    _check(load().lrmoe_split_wide(_ptr(rows), rows.shape[0], _ptr(idx), n, Xp.shape[-1],
+                                   Ap.shape[-1], _dt(Xp), _ptr(Xp), _ptr(DYp), _ptr(Ap), _ptr(Gp),
+                                   _ptr(Up), _ptr(status), _stream(stream)))
 
 
 def lrmoe_select_quota(topk_idx, score, quota, counts, kept, offsets, perm, pos, workspace,

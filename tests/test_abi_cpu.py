@@ -94,7 +94,7 @@ def test_router_grad_rejects_bad_arguments(lib):
 
 def test_split_by_destination_rejects_bad_arguments(lib):
     f = lib.lrmoe_split_by_destination
-    args = [FAKE, FAKE, FAKE, NULL, 4, 2, 100, FAKE, FAKE, FAKE, NULL, NULL]
+    args = [FAKE, FAKE, FAKE, NULL, 4, 2, 100, FAKE, FAKE, FAKE, NULL, NULL, NULL]
     bad = list(args); bad[2] = NULL                       # plan
     assert f(*bad) == L.LRMOE_ERR_INVALID_ARG and b"plan" in lib.lrmoe_last_error()
     bad = list(args); bad[4] = 0                          # E
@@ -103,6 +103,44 @@ def test_split_by_destination_rejects_bad_arguments(lib):
     assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
     bad = list(args); bad[3] = ctypes.c_void_p(0x10004)   # misaligned global_start
     assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
+
+
+    bad = list(args); bad[10] = ctypes.c_void_p(0x10004)  # misaligned row_dest
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG and b"row_dest" in lib.lrmoe_last_error()
+
+
+def test_group_received_rejects_bad_arguments(lib):
+    f = lib.lrmoe_group_received
+    args = [FAKE, 2, 4, 100, FAKE, FAKE, FAKE, NULL, NULL]
+    bad = list(args); bad[0] = NULL
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG and b"src_expert_offsets" in lib.lrmoe_last_error()
+    bad = list(args); bad[2] = 0                          # E
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
+    bad = list(args); bad[1] = 100000                     # G too large for shared memory
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
+    bad = list(args); bad[3] = 0                          # rows_cap
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG
+    bad = list(args); bad[5] = NULL                       # inv
+    assert f(*bad) == L.LRMOE_ERR_INVALID_ARG and b"inv" in lib.lrmoe_last_error()
+
+
+def test_exchange_rows_reject_bad_arguments(lib):
+    p = lib.lrmoe_pack_wide
+    args = [FAKE, FAKE, FAKE, 4, 2, 3, FAKE, FAKE, 16, FAKE, FAKE, FAKE, 8, 1, FAKE, 8, NULL, NULL]
+    bad = list(args); bad[10] = NULL                      # g
+    assert p(*bad) == L.LRMOE_ERR_INVALID_ARG and b"g" in lib.lrmoe_last_error()
+    bad = list(args); bad[12] = 12                        # I not a multiple of 8 (bf16)
+    assert p(*bad) == L.LRMOE_ERR_INVALID_ARG
+    bad = list(args); bad[15] = 0                         # rows_cap
+    assert p(*bad) == L.LRMOE_ERR_INVALID_ARG
+    s = lib.lrmoe_split_wide
+    args = [FAKE, 10, FAKE, 4, 16, 8, 1, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, NULL]
+    bad = list(args); bad[11] = NULL                      # Up
+    assert s(*bad) == L.LRMOE_ERR_INVALID_ARG and b"Up" in lib.lrmoe_last_error()
+    bad = list(args); bad[1] = 0                          # n_src
+    assert s(*bad) == L.LRMOE_ERR_INVALID_ARG
+    bad = list(args); bad[3] = 0                          # nothing to do
+    assert s(*bad) == L.LRMOE_OK
 
 
 def test_fused_gemm_rejects_bad_arguments(lib):

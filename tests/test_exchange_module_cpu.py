@@ -1,8 +1,8 @@
 """exchange.redistributed_backward's own multi-rank code on 2 and 3 gloo ranks
 (CPU): every library device call is replaced by an oracle-backed CPU stand-in, so
 what runs is the module's bookkeeping (summed counts, plan, global starts, split,
-block sizes, the compact all-to-all, regrouping, dW reduction, the return and
-unpack of dX_p).  Each rank's dX and the summed dW must equal what each rank
+send slots, exchange rows, block sizes, the compact all-to-all, regrouping, one
+dW reduction, the return and unpack of dX_p).  Each rank's dX and the summed dW must equal what each rank
 computes from its own pairs alone."""
 import os
 import socket
@@ -42,21 +42,38 @@ def _install_cpu_stand_ins(L, O, dtype):
         perm[: len(p)] = torch.from_numpy(p.astype(np.int32))
         pos.copy_(torch.from_numpy(q.astype(np.int32)))
 
-    def split(perm, offsets, plan, pd, do, deo, global_start=None, status=None, stream=None):
+    def split(perm, offsets, plan, pd, do, deo, global_start=None, status=None, stream=None,
+              row_dest=None):
         start = None if global_start is None else np32(global_start)
         a, b, c = O.split_by_destination(np32(perm), np32(offsets), np32(plan), start)
         pd[: len(a)] = torch.from_numpy(a)
         do.copy_(torch.from_numpy(b))
         deo.copy_(torch.from_numpy(c))
+        if row_dest is not None:
+            M = int(offsets[-1])
+            row_dest[:M] = torch.from_numpy(O.send_positions(np32(perm), a, M))
 
-    def pack(perm, offsets, w, x, dY, a, g, u, Xp, DYp, Ap, Gp, Up, status=None, stream=None,
-             I=None):
+    def pack_wide(perm, offsets, w, x, dY, a, g, u, rows, status=None, stream=None):
         M = int(offsets[-1])
         k_ = w.shape[1]
-        rows = O.pack(np32(perm)[:M], np32(w), k_, np32(x), np32(dY), np32(a), np32(g), np32(u),
-                      dtype)
-        for dst, r in zip((Xp, DYp, Ap, Gp, Up), rows):
-            dst[:M] = torch.from_numpy(np.asarray(r, np.float32))
+        parts = O.pack(np32(perm)[:M], np32(w), k_, np32(x), np32(dY), np32(a), np32(g), np32(u),
+                       dtype)
+        rows[:M] = torch.from_numpy(np.concatenate([np.asarray(r, np.float32) for r in parts],
+                                                   axis=1))
+
+    def group_received(tab, order, inv, offsets, status=None, stream=None):
+        o, i, off = O.group_received(np32(tab))
+        order[: len(o)] = torch.from_numpy(o)
+        inv[: len(i)] = torch.from_numpy(i)
+        offsets.copy_(torch.from_numpy(off))
+
+    def split_wide(rows, idx, Xp, DYp, Ap, Gp, Up, status=None, stream=None):
+        n = idx.numel()
+        H_, I_ = Xp.shape[1], Ap.shape[1]
+        src = rows[idx.long()]
+        cols = np.cumsum([0, H_, H_, I_, I_, I_])
+        for j, dst in enumerate((Xp, DYp, Ap, Gp, Up)):
+            dst[:n] = src[:, cols[j]:cols[j + 1]]
 
     def gather(src, idx, dst, status=None, stream=None):
         if idx.numel():
@@ -89,7 +106,8 @@ def _install_cpu_stand_ins(L, O, dtype):
                                   .astype(np.float32)))
 
     L.lrmoe_score, L.lrmoe_select_quota = score, select
-    L.lrmoe_split_by_destination, L.lrmoe_pack, L.lrmoe_gather_rows = split, pack, gather
+    L.lrmoe_split_by_destination, L.lrmoe_pack_wide, L.lrmoe_gather_rows = split, pack_wide, gather
+    L.lrmoe_group_received, L.lrmoe_split_wide = group_received, split_wide
     L.lrmoe_grouped_dgrad, L.lrmoe_grouped_wgrad, L.lrmoe_unpack = dgrad, wgrad, unpack
 
 

@@ -623,6 +623,61 @@ def test_split_by_destination_covers_each_global_run_once():
             assert got[(g, e)] == plan[e, g]
 
 
+def test_send_positions_put_each_row_back():
+    """send_positions is the defining inverse of the split: the send slot of local
+    packed row r holds that row's pair, and every slot is used once."""
+    plan = np.array([[1, 3], [2, 0], [0, 4]])
+    mine = np.array([3, 2, 3])
+    offsets = np.concatenate([[0], np.cumsum(mine)])
+    perm = np.array([5, 9, 14, 2, 30, 7, 11, 40])               # arbitrary pair ids
+    start = np.array([1, 0, 1])
+    pd, do, _ = O.split_by_destination(perm, offsets, plan, start)
+    M = int(offsets[-1])
+    rd = O.send_positions(perm, pd, M)
+    assert sorted(rd.tolist()) == list(range(M))
+    assert all(pd[rd[r]] == perm[r] for r in range(M))
+    # one destination keeps the packed order: the map is the identity
+    pd1, _, _ = O.split_by_destination(perm, offsets, mine.reshape(-1, 1) + start.reshape(-1, 1) * 0,
+                                       None)
+    assert O.send_positions(perm, pd1, M).tolist() == list(range(M))
+
+
+def _group_by_sorting(tab):
+    """Brute force for group_received: tag every received row with (expert, source,
+    arrival index) and sort by that tag."""
+    tab = np.asarray(tab)
+    G, E = tab.shape[0], tab.shape[1] - 1
+    tags, j = [], 0
+    for q in range(G):
+        for e in range(E):
+            for i in range(tab[q, e], tab[q, e + 1]):
+                tags.append((e, q, i, j))
+                j += 1
+    tags.sort()
+    order = [t[3] for t in tags]
+    counts = np.bincount([t[0] for t in tags], minlength=E) if tags else np.zeros(E, int)
+    return order, np.concatenate([[0], np.cumsum(counts)])
+
+
+def test_group_received_against_sorting_and_closed_forms():
+    rng = np.random.default_rng(5)
+    for G, E in ((1, 4), (3, 5), (4, 2), (2, 7)):
+        cnt = rng.integers(0, 4, size=(G, E))
+        cnt[0, 0] = 0                                       # empty blocks occur
+        tab = np.concatenate([np.zeros((G, 1), int), np.cumsum(cnt, axis=1)], axis=1)
+        order, inv, offs = O.group_received(tab)
+        want_order, want_offs = _group_by_sorting(tab)
+        assert order.tolist() == want_order
+        assert offs.tolist() == list(want_offs)
+        assert np.array_equal(inv[order], np.arange(len(order)))
+        if G == 1:                                          # one source: already grouped
+            assert order.tolist() == list(range(len(order)))
+    # two sources, one expert each way: source 1's rows of expert 0 come before
+    # source 0's rows of expert 1
+    order, inv, offs = O.group_received([[0, 0, 2], [0, 1, 1]])
+    assert order.tolist() == [2, 0, 1] and offs.tolist() == [0, 1, 3]
+
+
 def test_pruned_backward_equals_torch_autograd_on_the_retained_pairs():
     """The pruned oracle equals torch autograd (fp64) of a forward that contains only
     the retained pairs: dropping a pair from the backward is the same as dropping
