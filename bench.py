@@ -132,7 +132,8 @@ def load_peaks():
 
 
 # the sources that define each kernel whose DRAM traffic is recorded
-_GEMM_SOURCES = ("gemm_tc.cu", "common.cuh", "grouped.cuh", "launch.h")
+_GEMM_SOURCES = ("gemm_tc.cu", "gemm_pair.cu", "gemm_common.cuh", "common.cuh", "grouped.cuh",
+                 "launch.h")
 KERNEL_SOURCES = {
     "score": ("score.cu", "rowreduce.cuh", "common.cuh"),
     "select": ("select.cu", "common.cuh"),

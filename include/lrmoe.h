@@ -508,6 +508,21 @@ int lrmoe_pruned_backward(const lrmoe_buffers* b, int T, int k, int E, int H, in
  * ------------------------------------------------------------------------- */
 int lrmoe_selftest_bounded_wait(uint32_t limit_us, uint32_t* status, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Diagnostic (no counterpart in the pages): the grouped dgrad (bf16, store
+ * epilogue; the same operands as lrmoe_grouped_dgrad with E, K, N) launched so
+ * that its producers withhold the first K block of their first tile, with every
+ * device-side wait limited to limit_us microseconds (1 .. 1 000 000).  The
+ * MMA issuer's wait for that block runs out, the kernel raises
+ * LRMOE_ST_TIMEOUT, lets the copies and tensor-core work already in flight
+ * finish, releases its tensor memory and returns; the output is then invalid,
+ * and the context stays usable.  two_sm selects the two-SM tiles (else the
+ * one-SM tiles).  status is required.
+ * ------------------------------------------------------------------------- */
+int lrmoe_selftest_gemm_stall(const void* rows, int rows_cap, const void* W,
+                              const int32_t* offsets, int E, int K, int N, void* out, int two_sm,
+                              uint32_t limit_us, uint32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -548,6 +548,29 @@ int lrmoe_selftest_bounded_wait(uint32_t limit_us, uint32_t* status, void* strea
   return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_selftest_bounded_wait launch");
 }
 
+int lrmoe_selftest_gemm_stall(const void* rows, int rows_cap, const void* W,
+                              const int32_t* offsets, int E, int K, int N, void* out, int two_sm,
+                              uint32_t limit_us, uint32_t* status, void* stream) {
+  g_last_error[0] = 0;
+  REQUIRE(status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u) == 0,
+          "status is null or misaligned");
+  REQUIRE(limit_us >= 1 && limit_us <= 1000000u, "limit_us=%u outside [1, 1000000]", limit_us);
+  REQUIRE(E > 0 && E <= kMaxGroupedExperts && rows_cap > 0, "E or rows_cap out of range");
+  if (int r = check_feature(K, LRMOE_BF16, "K")) return r;
+  if (int r = check_feature(N, LRMOE_BF16, "N")) return r;
+  REQUIRE_PTR(rows);
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(out);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned long long ns = 1000ull * limit_us;
+  cudaError_t e = two_sm ? launch_dgrad_stall_pair(rows, rows_cap, W, offsets, E, K, N, out, ns,
+                                                   status, s)
+                         : launch_dgrad_stall_tc(rows, rows_cap, W, offsets, E, K, N, out, ns,
+                                                 status, s);
+  return e == cudaSuccess ? LRMOE_OK : cuda_fail(e, "lrmoe_selftest_gemm_stall launch");
+}
+
 int lrmoe_pruned_backward(const lrmoe_buffers* b, int T, int k, int E, int H, int I,
                           int rows_cap, lrmoe_dtype dt, void* stream) {
   g_last_error[0] = 0;

@@ -351,6 +351,13 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
                : "memory");
 }
 
+// The same arrival without release semantics: for arrivals that only count
+// (the data they stand for is tracked by the barrier's transaction bytes).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr)
+               : "memory");
+}
+
 __device__ __forceinline__ void st_cluster_u32(uint32_t cl_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cl_addr), "r"(v) : "memory");
 }

@@ -84,6 +84,11 @@ struct GemmParams {
   int gdiv, gperm_max;
   uint32_t* status;
   int sched_slot;
+  // diagnostics (zero in normal launches): wait_ns > 0 replaces the limit of
+  // every bounded wait; stall != 0 makes the producers withhold the first K
+  // block of their first tile, so that the MMA issuer's wait runs out
+  unsigned long long wait_ns;
+  int stall;
 };
 
 template <int MODE>

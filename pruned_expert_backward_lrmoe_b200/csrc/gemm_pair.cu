@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
   using L = PairLayout<STAGES, OUTBUFS>;
   const int E = p.E;
   uint32_t* status = p.status;
+  const uint64_t wlim = p.wait_ns ? p.wait_ns : kWaitLimitNs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
     const int slot = it % kRing;
     const bool ok = __all_sync(kFull, mbar_wait_bounded<true>(&ring_full[slot],
                                                               (uint32_t)(it / kRing) & 1u,
-                                                              abort_flag, status));
+                                                              abort_flag, status, wlim));
     const int t = ok ? ring[slot] : -1;
     __syncwarp();
     if (lane == 0) mbar_arrive_cluster(lead_ring_empty + 8u * slot);
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
         if (lane == 0) {
           t = (int)next;
           if (!mbar_wait_bounded<true>(&ring_empty[slot], ((uint32_t)(it / kRing) & 1u) ^ 1u,
-                                       abort_flag, status) ||
+                                       abort_flag, status, wlim) ||
               t >= tc.total || *abort_flag)
             t = -1;
           ring[slot] = t;
@@ -252,10 +253,18 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
       if (leader && ti.nk == 0 && lane == 0) next = atomicAdd(&sched[0], 1u);
       bool ok = true;
       for (int kb = 0; kb < ti.nk; ++kb) {
-        if (!__all_sync(kFull, mbar_wait_bounded<true>(&empty[stage], phase ^ 1u, abort_flag,
-                                                       status))) {
+        if (!__all_sync(kFull, mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status,
+                                                 wlim))) {
           ok = false;
           break;
+        }
+        if (p.stall && it == 0 && kb == 0) {  // diagnostic: this block never arrives
+          if (leader && lane == 0 && kb == ti.nk - 1) next = atomicAdd(&sched[0], 1u);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          continue;
         }
         uint8_t* sa = smem + stage * kPairStage;
         uint8_t* sb = sa + kPairABytes;
@@ -295,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
               tma_load_3d_pair(sb, &tmB, fb, b_col, kb * BK, ti.e);
               tma_load_3d_pair(sb + 8192, &tmB, fb, b_col + 64, kb * BK, ti.e);
             }
-            mbar_arrive_cluster(fb);
+            mbar_arrive_cluster_relaxed(fb);  // the bytes themselves are counted by the barrier
           }
         } else {
           // peer, last K block of a wgrad tile: land it here, zero the rows past
@@ -355,15 +364,20 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
         const PairTile ti = decode_pair<WG>(t, p, offs_s, tab_d, tab_w, tc);
         if (ti.nk == 0) continue;
         const uint32_t b = acc_iter & 1u, bphase = (acc_iter >> 1) & 1u;
-        if (!__all_sync(kFull, mbar_wait_bounded<true>(&tempty[b], bphase ^ 1u, abort_flag,
-                                                       status)))
+        if (!__all_sync(kFull, mbar_wait_bounded(&tempty[b], bphase ^ 1u, abort_flag, status,
+                                                 wlim)))
           break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * BN;
         bool ok = true;
         for (int kb = 0; kb < ti.nk; ++kb) {
-          if (!__all_sync(kFull, mbar_wait_bounded<true>(&full[stage], phase, abort_flag,
-                                                         status))) {
+          // the K-tail block carries the peer's zeroed rows (generic writes released
+          // at cluster scope); every other block's data is counted in transaction bytes
+          const bool tail_blk = WG && ti.row_end - (ti.row0 + kb * BK) < BK;
+          const bool landed =
+              tail_blk ? mbar_wait_bounded<true>(&full[stage], phase, abort_flag, status, wlim)
+                       : mbar_wait_bounded(&full[stage], phase, abort_flag, status, wlim);
+          if (!__all_sync(kFull, landed)) {
             ok = false;
             break;
           }
@@ -444,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
       if (!zero_tile) {
         b = acc_iter & 1u;
         const uint32_t bphase = (acc_iter >> 1) & 1u;
-        if (!__all_sync(kFull, mbar_wait_bounded<true>(&tfull[b], bphase, abort_flag, status)))
+        if (!__all_sync(kFull, mbar_wait_bounded(&tfull[b], bphase, abort_flag, status, wlim)))
           break;
         tc_fence_after();
         tmem_ld_32x32b_x32(lane_base + b * BN + cbase * 32, ra);
@@ -609,6 +623,21 @@ cudaError_t launch_dgrad_pair(const void* rows, int rows_cap, const void* W,
       ((long long)rows_cap / kPairM + E) * ((N + kBNT - 1) / kBNT);
   if (epi == LRMOE_EPI_SWIGLU_BWD)
     return launch_pair_variant<kDgradSwiglu, 6, 0>(a, b, a, prm, s, tiles);
+  return launch_pair_variant<kDgradStore, 6, 0>(a, b, a, prm, s, tiles);
+}
+
+// Diagnostic: the dgrad (store epilogue) with the first K block withheld and every
+// wait limited to wait_ns; must end with LRMOE_ST_TIMEOUT and a usable context.
+cudaError_t launch_dgrad_stall_pair(const void* rows, int rows_cap, const void* W,
+                                    const int32_t* offsets, int E, int K, int N, void* out,
+                                    unsigned long long wait_ns, uint32_t* status, cudaStream_t s) {
+  CUtensorMap a, b;
+  if (!make_map_2d(&a, rows, (uint64_t)rows_cap, (uint64_t)K, 64, 128) ||
+      !make_map_3d(&b, W, (uint64_t)E, (uint64_t)K, (uint64_t)N))
+    return cudaErrorInvalidValue;
+  GemmParams prm{offsets, E, K, N, 0, 0, nullptr, nullptr, nullptr, 0, out, 0, nullptr, 1, 0,
+                 status, 0, wait_ns, 1};
+  const long long tiles = ((long long)rows_cap / kPairM + E) * ((N + kBNT - 1) / kBNT);
   return launch_pair_variant<kDgradStore, 6, 0>(a, b, a, prm, s, tiles);
 }
 

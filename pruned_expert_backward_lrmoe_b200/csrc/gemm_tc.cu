@@ -39,6 +39,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   using L = Layout<BN, STAGES, OUTBUFS>;
   const int E = p.E;
   uint32_t* status = p.status;
+  const uint64_t wlim = p.wait_ns ? p.wait_ns : kWaitLimitNs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   auto next_tile = [&](int it) -> int {
     const int slot = it % kRing;
     const bool ok = __all_sync(
-        kFull, mbar_wait_bounded(&ring_full[slot], (uint32_t)(it / kRing) & 1u, abort_flag, status));
+        kFull, mbar_wait_bounded(&ring_full[slot], (uint32_t)(it / kRing) & 1u, abort_flag, status, wlim));
     const int t = ok ? ring[slot] : -1;
     __syncwarp();
     if (lane == 0) mbar_arrive(&ring_empty[slot]);
@@ -146,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         if (lane == 0) {
           t = (int)next;
           if (!mbar_wait_bounded(&ring_empty[slot], ((uint32_t)(it / kRing) & 1u) ^ 1u,
-                                 abort_flag, status) ||
+                                 abort_flag, status, wlim) ||
               t >= tc.total || *abort_flag)
             t = -1;
           ring[slot] = t;
@@ -158,8 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         if (ti.nk == 0 && lane == 0) next = atomicAdd(&sched[0], 1u);
         bool ok = true;
         for (int kb = 0; kb < ti.nk; ++kb) {
-          if (!__all_sync(kFull, mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag,
-                                                   status))) {
+          if (!__all_sync(kFull, mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status, wlim))) {
             ok = false;
             break;
           }
@@ -226,8 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
       for (int it = 0;; ++it) {
         const int slot = it % kRing;
         int t = (int)next;
-        if (!mbar_wait_bounded(&ring_empty[slot], ((uint32_t)(it / kRing) & 1u) ^ 1u, abort_flag,
-                               status) ||
+        if (!mbar_wait_bounded(&ring_empty[slot], ((uint32_t)(it / kRing) & 1u) ^ 1u, abort_flag, status, wlim) ||
             t >= tc.total || *abort_flag)
           t = -1;
         ring[slot] = t;
@@ -236,10 +235,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
         const TileInfo ti = decode_tile<MODE>(t, p, offs_s, tab_d, tab_w, tc);
         if (ti.nk == 0) next = atomicAdd(&sched[0], 1u);
         for (int kb = 0; kb < ti.nk; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status)) break;
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status, wlim)) break;
           // claim the following tile only now, a few K blocks before this one ends,
           // so that no CTA sits on a tile it cannot start soon
           if (kb == ti.nk - 1) next = atomicAdd(&sched[0], 1u);
+          if (p.stall && it == 0 && kb == 0) {  // diagnostic: this block never arrives
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           uint8_t* sa = smem + stage * L::kStageBytes;
           uint8_t* sb = sa + L::kABytes;
           armed |= 1u << stage;
@@ -287,13 +293,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
       if (ti.nk == 0) continue;
       const bool wg = ti.kind == 1;
       const uint32_t b = acc_iter & 1u, bphase = (acc_iter >> 1) & 1u;
-      if (!__all_sync(kFull, mbar_wait_bounded(&tempty[b], bphase ^ 1u, abort_flag, status)))
+      if (!__all_sync(kFull, mbar_wait_bounded(&tempty[b], bphase ^ 1u, abort_flag, status, wlim)))
         break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + b * BN;
       bool ok = true;
       for (int kb = 0; kb < ti.nk; ++kb) {
-        if (!__all_sync(kFull, mbar_wait_bounded(&full[stage], phase, abort_flag, status))) {
+        if (!__all_sync(kFull, mbar_wait_bounded(&full[stage], phase, abort_flag, status, wlim))) {
           ok = false;
           break;
         }
@@ -382,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
       if (!zero_tile) {
         b = acc_iter & 1u;
         const uint32_t bphase = (acc_iter >> 1) & 1u;
-        if (!__all_sync(kFull, mbar_wait_bounded(&tfull[b], bphase, abort_flag, status))) break;
+        if (!__all_sync(kFull, mbar_wait_bounded(&tfull[b], bphase, abort_flag, status, wlim))) break;
         tc_fence_after();
         tmem_ld_32x32b_x32(lane_base + b * BN + cbase * 32, ra);
         tmem_wait_ld();
@@ -548,12 +554,13 @@ bool wgrad_maps(Maps* m, const void* grad_rows, const void* in_rows, int rows_ca
 
 }  // namespace
 
-// LRMOE_GEMM_ONE_SM=1 in the environment selects the one-SM tiles of this file
-// instead of the two-SM tiles of gemm_pair.cu (both compute the same result).
+// LRMOE_GEMM_TWO_SM=1 in the environment selects the two-SM tiles of
+// gemm_pair.cu instead of the one-SM tiles of this file (both compute the same
+// result, bit for bit).
 static bool one_sm_tiles() {
   static const bool v = [] {
-    const char* e = getenv("LRMOE_GEMM_ONE_SM");
-    return e != nullptr && e[0] == '1';
+    const char* e = getenv("LRMOE_GEMM_TWO_SM");
+    return !(e != nullptr && e[0] == '1');
   }();
   return v;
 }
@@ -574,6 +581,19 @@ cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
   GemmParams prm{offsets, E, K, N, 0, 0, static_cast<const uint16_t*>(Gp),
                  static_cast<const uint16_t*>(Up), perm, gu_rows, out, 0, nullptr, 1, 0, status, 0};
   if (epi == LRMOE_EPI_SWIGLU_BWD) return launch_mode<kDgradSwiglu>(m, prm, s, num_sms());
+  return launch_mode<kDgradStore>(m, prm, s, num_sms());
+}
+
+// Diagnostic: the one-SM dgrad (store epilogue) with the first K block withheld
+// and every wait limited to wait_ns.
+cudaError_t launch_dgrad_stall_tc(const void* rows, int rows_cap, const void* W,
+                                  const int32_t* offsets, int E, int K, int N, void* out,
+                                  unsigned long long wait_ns, uint32_t* status, cudaStream_t s) {
+  Maps m;
+  if (!dgrad_maps(&m, rows, rows_cap, W, E, K, N)) return cudaErrorInvalidValue;
+  m.aw = m.bw = m.out = m.ad;  // unused
+  GemmParams prm{offsets, E, K, N, 0, 0, nullptr, nullptr, nullptr, 0, out, 0, nullptr, 1, 0,
+                 status, 0, wait_ns, 1};
   return launch_mode<kDgradStore>(m, prm, s, num_sms());
 }
 

@@ -108,6 +108,13 @@ cudaError_t launch_quota(const int32_t* idx, int P, int E, int cap, long long bu
 
 // diagnostic: a bounded wait that must time out
 cudaError_t launch_selftest_wait(uint32_t limit_us, uint32_t* status, cudaStream_t s);
+// diagnostic: a grouped dgrad whose first K block never arrives (one-SM / two-SM tiles)
+cudaError_t launch_dgrad_stall_tc(const void* rows, int rows_cap, const void* W,
+                                  const int32_t* offsets, int E, int K, int N, void* out,
+                                  unsigned long long wait_ns, uint32_t* status, cudaStream_t s);
+cudaError_t launch_dgrad_stall_pair(const void* rows, int rows_cap, const void* W,
+                                    const int32_t* offsets, int E, int K, int N, void* out,
+                                    unsigned long long wait_ns, uint32_t* status, cudaStream_t s);
 
 // tcgen05 grouped GEMMs (bf16 storage)
 // perm != nullptr: the SwiGLU epilogue reads g, u ([gu_rows][N]) at row perm[r]

@@ -6,29 +6,29 @@
 // uint32 descending, then pair index ascending (scores are >= +0, so the bit
 // order is the numeric order; NaN sorts above +Inf).
 //
-// Four kernels, integer work only, deterministic (no order-dependent atomics):
+// Three kernels, integer work only, deterministic (no order-dependent atomics):
 //   1. chunk_count : per chunk of pairs, an expert histogram (+ pos = -1 for
 //                    empty/invalid slots)
-//   2. chunk_scan  : per expert, exclusive scan over chunks; counts, the
-//                    segment starts, m_e = min(max(q_e,0), c_e), offsets
-//   3. chunk_scatter: stable counting sort of the pairs by expert (ascending p
+//   2. chunk_scatter: per expert, the scan over chunks (counts, the segment
+//                    starts, m_e = min(max(q_e,0), c_e), offsets), then a stable
+//                    counting sort of the chunk's pairs by expert (ascending p
 //                    inside each expert) into seg_p / seg_key
-//   4. expert_topk : one CTA per expert: 4 x 8-bit radix select of the m_e-th
-//                    largest key, then an ordered compaction that keeps keys
-//                    above the threshold and the first (m_e - #above) equal
-//                    keys in ascending p; writes perm and pos.
+//   3. expert_topk : one CTA per expert: 3-pass (11, 11, 10-bit) radix select
+//                    of the m_e-th largest key, then an ordered compaction that
+//                    keeps keys above the threshold and the first (m_e - #above)
+//                    equal keys in ascending p; writes perm and pos.
 #include "common.cuh"
+#include "grouped.cuh"
 #include "launch.h"
 
 namespace lrmoe {
 namespace {
 
-constexpr int kScanThreads = 1024;
 constexpr int kCountThreads = 256;
 constexpr int kScatterWarps = 8;
 constexpr int kTopkThreads = 1024;
-constexpr int kScanSmemInts = 32768;  // E * nchunks kept in shared memory by chunk_scan
-constexpr int kTopkSmemKeys = 24576;  // segments up to this length are staged in smem
+constexpr int kScanSmemInts = 32768;  // bound on E * nchunks (every scatter CTA reads it all)
+constexpr int kTopkSmemKeys = 53248;  // segments up to this length are staged in smem (keys)
 
 __global__ void __launch_bounds__(kCountThreads) chunk_count(const int32_t* __restrict__ idx,
                                                               int P, int E, int chunk,
@@ -71,120 +71,24 @@ __global__ void __launch_bounds__(kCountThreads) chunk_count(const int32_t* __re
   for (int e = threadIdx.x; e < E; e += blockDim.x) cc[(size_t)e * nchunks + c] = hist[e];
 }
 
-// Exclusive scan of n ints held one per thread (n <= blockDim.x * items); returns
-// per-thread exclusive prefix of the thread's item sum, and the total.
-__device__ int block_excl_scan(int v, int* warp_sums, int* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int nw = blockDim.x >> 5;
-  const int incl = warp_incl_scan(v);
-  if (lane == 31) warp_sums[wid] = incl;
-  __syncthreads();
-  if (wid == 0) {
-    int s = lane < nw ? warp_sums[lane] : 0;
-    int si = warp_incl_scan(s);
-    if (lane < nw) warp_sums[lane] = si - s;
-    if (lane == 31) warp_sums[32] = si;
-  }
-  __syncthreads();
-  const int r = warp_sums[wid] + incl - v;
-  *total = warp_sums[32];
-  __syncthreads();
-  return r;
-}
-
-__global__ void __launch_bounds__(kScanThreads) chunk_scan(int32_t* __restrict__ cc, int E,
-                                                           int nchunks,
-                                                           const int32_t* __restrict__ quota,
-                                                           int32_t* __restrict__ counts,
-                                                           int32_t* __restrict__ kept,
-                                                           int32_t* __restrict__ offsets,
-                                                           int32_t* __restrict__ seg_start,
-                                                           uint32_t* __restrict__ status) {
-  extern __shared__ int sm[];  // [33] warp sums, then [E] counts, then cc copy if it fits
-  int* warp_sums = sm;
-  int* cnt = sm + 33;
-  int* ccs = cnt + E;
-  const bool in_smem = (size_t)E * nchunks <= (size_t)kScanSmemInts;
-  int* mat = in_smem ? ccs : cc;
-  const int n = E * nchunks;
-  pdl_wait();
-  pdl_trigger();
-  if (in_smem) {
-    // eight loads in flight per thread, then the stores
-    for (int i0 = 0; i0 < n; i0 += 8 * blockDim.x) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * blockDim.x + threadIdx.x;
-        v[u] = i < n ? __ldcg(cc + i) : 0;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * blockDim.x + threadIdx.x;
-        if (i < n) ccs[i] = v[u];
-      }
-    }
-  }
-  __syncthreads();
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int e = wid; e < E; e += nw) {
-    int carry = 0;
-    int* row = mat + (size_t)e * nchunks;
-    for (int c0 = 0; c0 < nchunks; c0 += 32) {
-      const int c = c0 + lane;
-      const int v = c < nchunks ? row[c] : 0;
-      const int incl = warp_incl_scan(v);
-      if (c < nchunks) row[c] = carry + incl - v;
-      carry += __shfl_sync(kFull, incl, 31);
-    }
-    if (lane == 0) cnt[e] = carry;
-  }
-  __syncthreads();
-  if (in_smem)
-    for (int i = threadIdx.x; i < n; i += blockDim.x) cc[i] = ccs[i];
-  // segment starts (exclusive scan of counts) and offsets (exclusive scan of kept)
-  const int per = (E + blockDim.x - 1) / blockDim.x;
-  const int e0 = threadIdx.x * per;
-  int csum = 0, ksum = 0;
-  bool badq = false;
-  for (int i = 0; i < per; ++i) {
-    const int e = e0 + i;
-    if (e < E) {
-      const int c = cnt[e];
-      const int q = quota[e];
-      badq |= q < 0;
-      csum += c;
-      ksum += min(max(q, 0), c);
-    }
-  }
-  if (__any_sync(kFull, badq) && lane == 0) raise_status(status, LRMOE_ST_BAD_QUOTA);
-  int ctot, ktot;
-  int cex = block_excl_scan(csum, warp_sums, &ctot);
-  int kex = block_excl_scan(ksum, warp_sums, &ktot);
-  for (int i = 0; i < per; ++i) {
-    const int e = e0 + i;
-    if (e < E) {
-      const int c = cnt[e];
-      const int m = min(max(quota[e], 0), c);
-      counts[e] = c;
-      kept[e] = m;
-      seg_start[e] = cex;
-      offsets[e] = kex;
-      cex += c;
-      kex += m;
-    }
-  }
-  if (threadIdx.x == 0) {
-    seg_start[E] = ctot;
-    offsets[E] = ktot;
-  }
-}
-
+// Stable counting sort of the pairs by expert, with the scan over chunks folded
+// in.  CTA c handles chunk c.  First every CTA reads the whole per-(expert,
+// chunk) count matrix (one warp per expert, 32 chunks per load): the expert's
+// total and the count of the chunks before c.  An exclusive scan of the totals
+// gives the segment starts; CTA 0 also writes counts, kept (m_e = min(max(q_e,
+// 0), c_e)), offsets (scan of kept) and seg_start.  Then the chunk's pairs are
+// placed in ascending pair order (per-warp ranks by match_any).
 __global__ void __launch_bounds__(kScatterWarps * 32) chunk_scatter(
     const int32_t* __restrict__ idx, const uint32_t* __restrict__ score_bits, int P, int E,
-    int chunk, int nchunks, const int32_t* __restrict__ cc, const int32_t* __restrict__ seg_start,
-    int32_t* __restrict__ seg_p, uint32_t* __restrict__ seg_key) {
-  extern __shared__ int wbase[];  // [kScatterWarps][E]
+    int chunk, int nchunks, const int32_t* __restrict__ cc, const int32_t* __restrict__ quota,
+    int32_t* __restrict__ counts, int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ seg_start, int32_t* __restrict__ seg_p, uint32_t* __restrict__ seg_key,
+    uint32_t* __restrict__ status) {
+  extern __shared__ int sm_sc[];  // wbase [kScatterWarps][E], tot [E], pre [E], scratch [33]
+  int* wbase = sm_sc;
+  int* tot = wbase + kScatterWarps * E;
+  int* pre = tot + E;
+  int* scratch = pre + E;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int c = blockIdx.x;
   const int begin = c * chunk;
@@ -196,6 +100,47 @@ __global__ void __launch_bounds__(kScatterWarps * 32) chunk_scatter(
   __syncthreads();
   pdl_wait();
   pdl_trigger();
+  // per expert: total over chunks and the part before this chunk
+  for (int e = wid; e < E; e += kScatterWarps) {
+    const int32_t* row = cc + (size_t)e * nchunks;
+    int t_all = 0, t_pre = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 64) {
+      const int i0 = c0 + lane, i1 = c0 + 32 + lane;
+      const int v0 = i0 < nchunks ? __ldcg(row + i0) : 0;
+      const int v1 = i1 < nchunks ? __ldcg(row + i1) : 0;
+      t_all += __reduce_add_sync(kFull, v0 + v1);
+      t_pre += __reduce_add_sync(kFull, (i0 < c ? v0 : 0) + (i1 < c ? v1 : 0));
+    }
+    if (lane == 0) {
+      tot[e] = t_all;
+      pre[e] = t_pre;
+    }
+  }
+  __syncthreads();
+  if (c == 0) {
+    bool badq = false;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      const int q = quota[e];
+      badq |= q < 0;
+      const int m = min(max(q, 0), tot[e]);
+      counts[e] = tot[e];
+      kept[e] = m;
+      wbase[e] = m;  // scratch for the scan of kept (wbase is rebuilt below)
+    }
+    if (__any_sync(kFull, badq) && lane == 0) raise_status(status, LRMOE_ST_BAD_QUOTA);
+    __syncthreads();
+    const int ktot = block_scan_inplace(wbase, E, scratch);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = wbase[e];
+    if (threadIdx.x == 0) offsets[E] = ktot;
+    __syncthreads();
+    for (int i = threadIdx.x; i < E; i += blockDim.x) wbase[i] = 0;
+  }
+  // segment starts: exclusive scan of the totals (tot becomes the start)
+  const int ctot = block_scan_inplace(tot, E, scratch);
+  if (c == 0) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) seg_start[e] = tot[e];
+    if (threadIdx.x == 0) seg_start[E] = ctot;
+  }
   int* mine = wbase + wid * E;
   constexpr int kSteps = 4;  // 32-pair steps whose loads are in flight together
   for (int q0 = wbeg; q0 < wend; q0 += 32 * kSteps) {
@@ -211,7 +156,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) chunk_scatter(
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = seg_start[e] + cc[(size_t)e * nchunks + c];
+    int run = tot[e] + pre[e];
 #pragma unroll
     for (int w = 0; w < kScatterWarps; ++w) {
       const int v = wbase[w * E + e];
@@ -250,46 +195,25 @@ __global__ void __launch_bounds__(kScatterWarps * 32) chunk_scatter(
   }
 }
 
-// Block-wide exclusive scan of 64-bit values (two 32-bit counters packed in one
-// word, low and high halves); returns the total too.  blockDim.x <= 1024.
-__device__ __forceinline__ unsigned long long block_excl_scan_u64(unsigned long long v,
-                                                                  unsigned long long* ws,
-                                                                  unsigned long long* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  unsigned long long incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long n = __shfl_up_sync(kFull, incl, o);
-    if (lane >= o) incl += n;
-  }
-  if (lane == 31) ws[wid] = incl;
-  __syncthreads();
-  if (wid == 0) {
-    const unsigned long long x = lane < nw ? ws[lane] : 0ull;
-    unsigned long long xi = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned long long n = __shfl_up_sync(kFull, xi, o);
-      if (lane >= o) xi += n;
-    }
-    if (lane < nw) ws[lane] = xi - x;
-    if (lane == 31) ws[32] = xi;
-  }
-  __syncthreads();
-  const unsigned long long r = ws[wid] + incl - v;
-  *total = ws[32];
-  __syncthreads();
-  return r;
-}
+// Digits of the radix select, most significant first: 11 + 11 + 10 bits.
+__device__ __forceinline__ int digit_shift(int d) { return d == 0 ? 21 : (d == 1 ? 10 : 0); }
+__device__ __forceinline__ int digit_bins(int d) { return d == 2 ? 1024 : 2048; }
 
+// One CTA per expert.  The expert's keys (its segment of seg_key, pairs in
+// ascending p) are staged in shared memory when they fit.  A 3-pass radix
+// select (11, 11, 10 bits) finds tau, the m-th largest key, and how many keys
+// equal to tau stay (the first ones in segment order, i.e. ascending p).  The
+// compaction is warp-contiguous: warp w owns a contiguous run of the segment,
+// walked 32 keys at a time; ballots give each kept key its rank inside the step,
+// one block scan of the warps' (above, equal) counts gives each warp's start.
 __global__ void __launch_bounds__(kTopkThreads) expert_topk(
     const int32_t* __restrict__ counts, const int32_t* __restrict__ kept,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ seg_start,
     const int32_t* __restrict__ seg_p, const uint32_t* __restrict__ seg_key,
     int32_t* __restrict__ perm, int32_t* __restrict__ pos) {
-  extern __shared__ uint32_t sm_keys[];  // [kTopkSmemKeys] keys, then [kTopkSmemKeys] pairs
-  __shared__ int hist[256];
-  __shared__ unsigned long long scan_ws[33];
+  extern __shared__ uint32_t sm_keys[];  // [kTopkSmemKeys]
+  __shared__ int hist[2048];
+  __shared__ int warp_gt[kTopkThreads / 32], warp_eq[kTopkThreads / 32];
   __shared__ int found_bin, found_above;
   pdl_wait();
   pdl_trigger();
@@ -299,7 +223,7 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
   const int s0 = seg_start[e];
   const int out0 = offsets[e];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int nt = blockDim.x;
+  const int nt = blockDim.x, nw = nt >> 5;
   const int32_t* sp = seg_p + s0;
   const uint32_t* sk = seg_key + s0;
 
@@ -316,52 +240,40 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
     return;
   }
 
-  // stage the segment in shared memory (four loads in flight per thread)
+  // stage the keys (eight loads in flight per thread)
   const bool in_smem = c <= kTopkSmemKeys;
   const uint32_t* K = sk;
-  const int32_t* PP = sp;
   if (in_smem) {
-    uint32_t* ks = sm_keys;
-    int32_t* ps = reinterpret_cast<int32_t*>(sm_keys + kTopkSmemKeys);
-    for (int i0 = 0; i0 < c; i0 += 4 * nt) {
-      uint32_t kv[4];
-      int pv[4];
+    for (int i0 = 0; i0 < c; i0 += 8 * nt) {
+      uint32_t kv[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int i = i0 + u * nt + tid;
-        if (i < c) {
-          kv[u] = sk[i];
-          pv[u] = sp[i];
-        }
+        kv[u] = i < c ? __ldcg(sk + i) : 0u;
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int i = i0 + u * nt + tid;
-        if (i < c) {
-          ks[i] = kv[u];
-          ps[i] = pv[u];
-        }
+        if (i < c) sm_keys[i] = kv[u];
       }
     }
-    K = ks;
-    PP = ps;
+    K = sm_keys;
   }
   __syncthreads();
 
-  // radix select of the m-th largest key, most significant byte first
-  uint32_t prefix = 0;
+  // radix select of the m-th largest key
+  uint32_t prefix = 0, pmask = 0;
   int need = m;
-  for (int d = 3; d >= 0; --d) {
-    const int shift = 8 * d;
-    const uint32_t hmask = d == 3 ? 0u : (0xffffffffu << (shift + 8));
-    for (int i = tid; i < 256; i += nt) hist[i] = 0;
+  for (int d = 0; d < 3; ++d) {
+    const int shift = digit_shift(d), nb = digit_bins(d);
+    for (int i = tid; i < nb; i += nt) hist[i] = 0;
     __syncthreads();
     for (int i0 = 0; i0 < c; i0 += nt) {
       const int i = i0 + tid;
       int digit = -1;
       if (i < c) {
         const uint32_t key = K[i];
-        if ((key & hmask) == prefix) digit = (int)((key >> shift) & 255u);
+        if ((key & pmask) == prefix) digit = (int)((key >> shift) & (uint32_t)(nb - 1));
       }
       if (__any_sync(kFull, digit >= 0)) {  // later passes: most warps hold no candidate
         const unsigned grp = __match_any_sync(kFull, digit);
@@ -370,63 +282,78 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
     }
     __syncthreads();
     if (wid == 0) {
-      // lane l owns bins 255-8l down to 248-8l (descending key order)
-      int cnt8[8];
+      // lane l owns the nb/32 bins below nb - 1 - l*nb/32 (descending key order)
+      const int per = nb >> 5;
+      const int top = nb - 1 - lane * per;
       int lsum = 0;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        cnt8[b] = hist[255 - 8 * lane - b];
-        lsum += cnt8[b];
-      }
+      for (int b = 0; b < per; ++b) lsum += hist[top - b];
       const int incl = warp_incl_scan(lsum);
       const int excl = incl - lsum;
       if (excl < need && need <= incl) {
         int cum = excl;
-#pragma unroll
-        for (int b = 0; b < 8; ++b) {
-          if (cum + cnt8[b] >= need) {
-            found_bin = 255 - 8 * lane - b;
+        for (int b = 0; b < per; ++b) {
+          const int v = hist[top - b];
+          if (cum + v >= need) {
+            found_bin = top - b;
             found_above = cum;
             break;
           }
-          cum += cnt8[b];
+          cum += v;
         }
       }
     }
     __syncthreads();
     prefix |= (uint32_t)found_bin << shift;
+    pmask |= (uint32_t)(nb - 1) << shift;
     need -= found_above;
     __syncthreads();
   }
   const uint32_t tau = prefix;
-  const unsigned long long need_eq = (unsigned long long)need;  // equal keys kept, in ascending p
+  const int need_eq = need;  // keys equal to tau that stay, first ones in ascending p
 
-  // ordered compaction: thread t owns the contiguous run [t*R, t*R + R); one scan
-  // of (above, equal) counts gives every run its starting row.
-  const int R = (c + nt - 1) / nt;
-  const int b0 = min(c, tid * R), b1 = min(c, b0 + R);
-  unsigned long long ngt = 0, neq = 0;
-  for (int i = b0; i < b1; ++i) {
+  // warp-contiguous compaction
+  const int run = ((c + nw - 1) / nw + 31) & ~31;  // keys per warp, whole steps
+  const int w0 = min(c, wid * run), w1 = min(c, w0 + run);
+  int ngt = 0, neq = 0;
+  for (int i = w0 + lane; i < w1; i += 32) {
     const uint32_t key = K[i];
     ngt += key > tau;
     neq += key == tau;
   }
-  unsigned long long tot;
-  const unsigned long long ex = block_excl_scan_u64(ngt | (neq << 32), scan_ws, &tot);
-  unsigned long long gt_before = ex & 0xffffffffull, eq_before = ex >> 32;
-  for (int i = b0; i < b1; ++i) {
-    const uint32_t key = K[i];
-    const int p = PP[i];
-    const bool gt = key > tau, eq = key == tau;
-    if (gt || (eq && eq_before < need_eq)) {
-      const int row = out0 + (int)(gt_before + (eq_before < need_eq ? eq_before : need_eq));
+  ngt = __reduce_add_sync(kFull, ngt);
+  neq = __reduce_add_sync(kFull, neq);
+  if (lane == 0) {
+    warp_gt[wid] = ngt;
+    warp_eq[wid] = neq;
+  }
+  __syncthreads();
+  int gt_before = 0, eq_before = 0;  // exclusive prefix over the warps before this one
+  {
+    const int g = lane < nw && lane < wid ? warp_gt[lane] : 0;
+    const int q = lane < nw && lane < wid ? warp_eq[lane] : 0;
+    gt_before = __reduce_add_sync(kFull, g);
+    eq_before = __reduce_add_sync(kFull, q);
+  }
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i0 = w0; i0 < w1; i0 += 32) {
+    const int i = i0 + lane;
+    const bool in = i < w1;
+    const uint32_t key = in ? K[i] : 0u;
+    const int p = in ? __ldg(sp + i) : 0;
+    const bool gt = in && key > tau, eq = in && key == tau;
+    const unsigned mgt = __ballot_sync(kFull, gt), meq = __ballot_sync(kFull, eq);
+    const int eq_rank = eq_before + __popc(meq & lt);
+    const bool keep = gt || (eq && eq_rank < need_eq);
+    if (keep) {
+      const int kept_eq_before = min(eq_rank, need_eq);
+      const int row = out0 + gt_before + __popc(mgt & lt) + kept_eq_before;
       perm[row] = p;
       pos[p] = row;
-    } else {
+    } else if (in) {
       pos[p] = -1;
     }
-    gt_before += gt;
-    eq_before += eq;
+    gt_before += __popc(mgt);
+    eq_before += __popc(meq);
   }
 }
 
@@ -452,29 +379,22 @@ static cudaError_t enqueue_select(const SelectWs& L, const int32_t* idx, const f
   // Shared-memory limits are set on every call (host-side calls, no device
   // work), so that they hold in whatever context is current, also after a
   // context reset, and no host-side flag is shared between threads.
-  cudaError_t e = cudaFuncSetAttribute(chunk_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (33 + 4096 + kScanSmemInts) * 4);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(chunk_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kScatterWarps * 4096 * 4);
+  const size_t scatter_smem = ((size_t)kScatterWarps * E + 2 * (size_t)E + 33) * 4;
+  cudaError_t e = cudaFuncSetAttribute(chunk_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)((kScatterWarps + 2) * 4096 + 33) * 4);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(expert_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kTopkSmemKeys * 8);
+                             kTopkSmemKeys * 4);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(chunk_count, dim3(L.nchunks), dim3(kCountThreads), (size_t)E * 4, s,
-                             idx, P, E, L.chunk, L.nchunks, cc, pos, status);
+  e = launch_pdl(chunk_count, dim3(L.nchunks), dim3(kCountThreads), (size_t)E * 4, s, idx, P, E,
+                 L.chunk, L.nchunks, cc, pos, status);
   if (e != cudaSuccess) return e;
-  const bool fits = (size_t)E * L.nchunks <= (size_t)kScanSmemInts;
-  const size_t scan_smem = (33 + (size_t)E + (fits ? (size_t)E * L.nchunks : 0)) * 4;
-  e = launch_pdl(chunk_scan, dim3(1), dim3(kScanThreads), scan_smem, s, cc, E, L.nchunks, quota,
-                 counts, kept, offsets, seg_start, status);
+  e = launch_pdl(chunk_scatter, dim3(L.nchunks), dim3(kScatterWarps * 32), scatter_smem, s, idx,
+                 reinterpret_cast<const uint32_t*>(score), P, E, L.chunk, L.nchunks,
+                 static_cast<const int32_t*>(cc), quota, counts, kept, offsets, seg_start, seg_p,
+                 seg_key, status);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(chunk_scatter, dim3(L.nchunks), dim3(kScatterWarps * 32),
-                 (size_t)kScatterWarps * E * 4, s, idx, reinterpret_cast<const uint32_t*>(score),
-                 P, E, L.chunk, L.nchunks, static_cast<const int32_t*>(cc),
-                 static_cast<const int32_t*>(seg_start), seg_p, seg_key);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(expert_topk, dim3(E), dim3(kTopkThreads), (size_t)kTopkSmemKeys * 8, s,
+  return launch_pdl(expert_topk, dim3(E), dim3(kTopkThreads), (size_t)kTopkSmemKeys * 4, s,
                     static_cast<const int32_t*>(counts), static_cast<const int32_t*>(kept),
                     static_cast<const int32_t*>(offsets), static_cast<const int32_t*>(seg_start),
                     static_cast<const int32_t*>(seg_p), static_cast<const uint32_t*>(seg_key),

@@ -29,7 +29,8 @@ EXPORTS = ("lrmoe_version", "lrmoe_status_string", "lrmoe_last_error", "lrmoe_sc
            "lrmoe_row_sqnorm", "lrmoe_score_from_norms", "lrmoe_router_grad",
            "lrmoe_redistribute", "lrmoe_split_by_destination", "lrmoe_grouped_dgrad_wgrad",
            "lrmoe_grouped_dgrad_swiglu_gather", "lrmoe_grouped_wgrad_gather", "lrmoe_gather_rows",
-           "lrmoe_group_received", "lrmoe_pack_wide", "lrmoe_split_wide")
+           "lrmoe_group_received", "lrmoe_pack_wide", "lrmoe_split_wide",
+           "lrmoe_selftest_gemm_stall")
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -78,6 +79,7 @@ def load() -> ctypes.CDLL:
     lib.lrmoe_select_quota.argtypes = [P, P, I, I, I, P, P, P, P, P, P, P, Z, P, P]
     lib.lrmoe_select_quota_noalloc.argtypes = [P, P, I, I, I, P, P, P, P, P, P, P, P]
     lib.lrmoe_selftest_bounded_wait.argtypes = [U32, P, P]
+    lib.lrmoe_selftest_gemm_stall.argtypes = [P, I, P, P, I, I, I, P, I, U32, P, P]
     lib.lrmoe_quota_controller.argtypes = [P, I, I, I, ctypes.c_int32, ctypes.c_int64, P, P, P, P]
     lib.lrmoe_pack.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, I, I, P, P, P, P, P, I, P, P]
     lib.lrmoe_grouped_dgrad.argtypes = [P, I, P, P, I, I, I, I, I, P, P, P, P, P]
@@ -325,6 +327,15 @@ def lrmoe_grouped_dgrad_wgrad(grad_rows, W, offsets, epilogue: int, out, in_rows
 def lrmoe_unpack(dXp, pos, T: int, k: int, dX, status=None, stream=None) -> None:
     _check(load().lrmoe_unpack(_ptr(dXp), dXp.shape[0], _ptr(pos), T, k, dXp.shape[-1], _dt(dXp),
                                _ptr(dX), _ptr(status), _stream(stream)))
+
+
+def lrmoe_selftest_gemm_stall(rows, W, offsets, out, two_sm: bool, limit_us: int, status,
+                              stream=None) -> None:
+    """The grouped dgrad with its first K block withheld; must set ST_TIMEOUT."""
+    E, K, N = W.shape
+    _check(load().lrmoe_selftest_gemm_stall(_ptr(rows), rows.shape[0], _ptr(W), _ptr(offsets), E,
+                                            K, N, _ptr(out), int(bool(two_sm)), int(limit_us),
+                                            _ptr(status), _stream(stream)))
 
 
 def lrmoe_selftest_bounded_wait(limit_us: int, status, stream=None) -> None:

@@ -203,6 +203,12 @@ def test_full_size_parity(name):
     want = O.unpack_tokens(tokens, dxp, pos, s.k, s.H)
     got = out["dX"][tokens].float().cpu().numpy()
     assert PT.rel_fro(got, want) <= tol
+    # the same bound on every sampled token alone, so that one wrong row cannot
+    # hide in the pooled norm
+    per_token = [PT.rel_fro(got[i], want[i]) for i in range(len(tokens)) if np.any(want[i])]
+    worst = max(per_token) if per_token else 0.0
+    print(f"{name}: dX pooled rel err {PT.rel_fro(got, want):.3e}, worst token {worst:.3e}")
+    assert worst <= tol, worst
     none = [i for i, t in enumerate(tokens) if (pos.reshape(-1, s.k)[t] < 0).all()]
     assert not got[none].any()
     # invariant that holds at any size: every retained row belongs to its block's expert
