@@ -545,7 +545,8 @@ def make_runner(layer, dev):
         names = CALL_NAMES if not fused else CALL_NAMES[:3] + FUSED_NAMES + CALL_NAMES[-1:]
         for i, c in enumerate(calls):
             if waits and i in waits:
-                stream.wait_event(waits[i])
+                for ev_ in waits[i]:
+                    stream.wait_event(ev_)
             if ev is not None:
                 ev[i].record(stream)
             nvtx.range_push(names[i])   # one NVTX range per C-ABI call
@@ -817,8 +818,9 @@ def run_e2e(layer, res, dev, args, dist):
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(n_e2e)]
     # The compute stream waits only where it needs each group (score and select:
-    # routing, dY, a; pack: x; the SwiGLU dgrad: g, u).
-    copy_stream = torch.cuda.Stream(dev)
+    # routing, dY, a; pack: x; the SwiGLU dgrad: g, u).  Each group's tensors are
+    # split over two copy streams (two DMA queues in flight at once).
+    copy_streams = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
     groups = (("topk_idx", "topk_w", "quota", "dY", "a"), ("x",), ("g", "u"))
     need_at = (0, 2, 3)   # step call index before which each group must have landed
     for i in range(n_e2e + 2):
@@ -826,15 +828,22 @@ def run_e2e(layer, res, dev, args, dist):
         flush_l2()
         if timed:
             e2e_ev[i - 2][0].record(stream)
-        copy_stream.wait_stream(stream)   # the previous step is done with its inputs
+        for cs in copy_streams:
+            cs.wait_stream(stream)   # the previous step is done with its inputs
         landed = []
-        with torch.cuda.stream(copy_stream):
-            for grp in groups:
-                for k_ in grp:
-                    inp[k_].copy_(pin[k_], non_blocking=True)
-                ev_ = torch.cuda.Event()
-                ev_.record(copy_stream)
-                landed.append(ev_)
+        for grp in groups:
+            evs_ = []
+            for j, cs in enumerate(copy_streams):
+                with torch.cuda.stream(cs):
+                    for k_ in grp:
+                        half = pin[k_].shape[0] // 2
+                        rows = slice(0, half) if j == 0 else slice(half, None)
+                        if pin[k_][rows].numel():
+                            inp[k_][rows].copy_(pin[k_][rows], non_blocking=True)
+                    ev_ = torch.cuda.Event()
+                    ev_.record(cs)
+                    evs_.append(ev_)
+            landed.append(evs_)
         step(waits=dict(zip(need_at, landed)))
         dX_host.copy_(out["dX"], non_blocking=True)
         st_host.copy_(out["status"], non_blocking=True)

@@ -351,6 +351,13 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
                : "memory");
 }
 
+// Remote arrival with release at CTA scope (the arriving thread's own earlier
+// accesses are ordered before it; no cluster-wide fence).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cl_addr)
+               : "memory");
+}
+
 // The same arrival without release semantics: for arrivals that only count
 // (the data they stand for is tracked by the barrier's transaction bytes).
 __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cl_addr) {

@@ -43,7 +43,9 @@ constexpr int kHalfN = kBNT / 2;             // B columns loaded by each CTA
 constexpr int kPairABytes = BM * BK * 2;     // 16 KB: this CTA's 128 A rows of a K block
 constexpr int kPairBBytes = kHalfN * BK * 2; // 16 KB: this CTA's 128 B columns
 constexpr int kPairStage = kPairABytes + kPairBBytes;
-constexpr int kPairConsumers = 2 * (1 + kEpiWarps);  // warps that read a tile-ring slot
+// warps that read a tile-ring slot: leader MMA + epilogue, peer producer +
+// epilogue, and (wgrad) the peer's K-tail warp
+__host__ __device__ constexpr int pair_consumers(bool wg) { return 2 * (1 + kEpiWarps) + (wg ? 1 : 0); }
 
 // Launch counter of the pair kernels (picks the scheduling slot).
 std::atomic<unsigned int> g_launches{0};
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
     mbar_init(mma_done, 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&ring_full[i], 1);
-      mbar_init(&ring_empty[i], kPairConsumers);
+      mbar_init(&ring_empty[i], pair_consumers(WG));
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -210,12 +212,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
   // Tile of the it-th round for this CTA's consumer warps (-1: no more tiles).
   auto next_tile = [&](int it) -> int {
     const int slot = it % kRing;
-    const bool ok = __all_sync(kFull, mbar_wait_bounded<true>(&ring_full[slot],
-                                                              (uint32_t)(it / kRing) & 1u,
-                                                              abort_flag, status, wlim));
+    // the leader's ring is written by its own producer (CTA scope); the peer's by
+    // the leader's producer across the cluster
+    const uint32_t par = (uint32_t)(it / kRing) & 1u;
+    const bool ok = __all_sync(
+        kFull, leader ? mbar_wait_bounded(&ring_full[slot], par, abort_flag, status, wlim)
+                      : mbar_wait_bounded<true>(&ring_full[slot], par, abort_flag, status, wlim));
     const int t = ok ? ring[slot] : -1;
     __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(lead_ring_empty + 8u * slot);
+    if (lane == 0) mbar_arrive_remote(lead_ring_empty + 8u * slot);
     return t;
   };
 
@@ -224,25 +229,33 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
     int stage = 0;
     uint32_t phase = 0;
     uint32_t armed = 0, armed_par = 0;  // leader: stages with loads issued, and their phase
-    uint32_t tail_par = 0;              // peer: phase of each stage's tail barrier
-    unsigned int next = 0;
-    if (leader && lane == 0) next = atomicAdd(&sched[0], 1u);
+    uint32_t tail_used = 0, tail_next = 0;  // peer: stages with a tail load issued; next phase
     const uint32_t peer_ring = cluster_addr((const void*)ring, 1);
     const uint32_t peer_ring_full = cluster_addr(ring_full, 1);
+    // Leader: claim a tile and hand it to both CTAs' consumers in ring slot it2 % kRing
+    // (lane 0).  Tiles are claimed and published one ahead of the loads, so that the
+    // peer knows its next tile before it finishes the current one.
+    auto publish = [&](int it2) -> int {
+      const int slot2 = it2 % kRing;
+      int t2 = (int)atomicAdd(&sched[0], 1u);
+      if (!mbar_wait_bounded<true>(&ring_empty[slot2], ((uint32_t)(it2 / kRing) & 1u) ^ 1u,
+                                   abort_flag, status, wlim) ||
+          t2 >= tc.total || *abort_flag)
+        t2 = -1;
+      ring[slot2] = t2;
+      st_cluster_u32(peer_ring + 4u * slot2, (uint32_t)t2);
+      mbar_arrive(&ring_full[slot2]);
+      mbar_arrive_cluster(peer_ring_full + 8u * slot2);
+      return t2;
+    };
+    int ahead = -1;  // leader: the tile published for the next round
+    if (leader && lane == 0) ahead = publish(0);
     for (int it = 0;; ++it) {
-      const int slot = it % kRing;
       int t = -1;
       if (leader) {
         if (lane == 0) {
-          t = (int)next;
-          if (!mbar_wait_bounded<true>(&ring_empty[slot], ((uint32_t)(it / kRing) & 1u) ^ 1u,
-                                       abort_flag, status, wlim) ||
-              t >= tc.total || *abort_flag)
-            t = -1;
-          ring[slot] = t;
-          st_cluster_u32(peer_ring + 4u * slot, (uint32_t)t);
-          mbar_arrive(&ring_full[slot]);
-          mbar_arrive_cluster(peer_ring_full + 8u * slot);
+          t = ahead;
+          if (t >= 0) ahead = publish(it + 1);
         }
         t = __shfl_sync(kFull, t, 0);
       } else {
@@ -250,7 +263,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
       }
       if (t < 0) break;
       const PairTile ti = decode_pair<WG>(t, p, offs_s, tab_d, tab_w, tc);
-      if (leader && ti.nk == 0 && lane == 0) next = atomicAdd(&sched[0], 1u);
       bool ok = true;
       for (int kb = 0; kb < ti.nk; ++kb) {
         if (!__all_sync(kFull, mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status,
@@ -259,7 +271,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
           break;
         }
         if (p.stall && it == 0 && kb == 0) {  // diagnostic: this block never arrives
-          if (leader && lane == 0 && kb == ti.nk - 1) next = atomicAdd(&sched[0], 1u);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -276,7 +287,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
         const int b_col = ti.n0 + (int)rank * kHalfN;
         if (leader) {
           if (lane == 0) {
-            if (kb == ti.nk - 1) next = atomicAdd(&sched[0], 1u);
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
             mbar_arrive_expect_tx(&full[stage], kPairStage + (tail ? 0 : kPairStage));
@@ -307,32 +317,19 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
             mbar_arrive_cluster_relaxed(fb);  // the bytes themselves are counted by the barrier
           }
         } else {
-          // peer, last K block of a wgrad tile: land it here, zero the rows past
-          // the expert's end, then let the leader's MMAs read it
+          // peer, last K block of a wgrad tile: land it on this CTA's tail barrier;
+          // warp 1 zeroes the rows past the expert's end and then lets the
+          // leader's MMAs read it (this warp goes on with the next loads)
           if constexpr (WG) {
             if (lane == 0) {
+              tail_used |= 1u << stage;
+              tail_next ^= 1u << stage;
               mbar_arrive_expect_tx(&tailb[stage], kPairStage);
               tma_load_2d(sa, &tmA, &tailb[stage], a_c0, a_c1);
               tma_load_2d(sa + 8192, &tmA, &tailb[stage], a_c0 + 64, a_c1);
               tma_load_2d(sb, &tmB, &tailb[stage], b_col, r);
               tma_load_2d(sb + 8192, &tmB, &tailb[stage], b_col + 64, r);
             }
-            const bool landed = __all_sync(kFull, mbar_wait_drain(&tailb[stage],
-                                                                  (tail_par >> stage) & 1u));
-            tail_par ^= 1u << stage;
-            if (!landed) {
-              if (lane == 0) {
-                *abort_flag = 1;
-                raise_status(status, LRMOE_ST_TIMEOUT);
-              }
-              ok = false;
-              break;
-            }
-            const int nkk = (valid + UK - 1) / UK;
-            zero_tail_rows(sa, sb, valid, nkk * UK - valid, lane);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(lead_full + 8u * stage);
           }
         }
         if (++stage == STAGES) {
@@ -348,7 +345,47 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
     if (leader && lane == 0)
       for (int i = 0; i < STAGES; ++i)
         if ((armed >> i) & 1u) mbar_wait_drain<true>(&full[i], (armed_par >> i) & 1u);
+    if (!leader && lane == 0)
+      for (int i = 0; i < STAGES; ++i)
+        if ((tail_used >> i) & 1u) mbar_wait_drain(&tailb[i], ((tail_next >> i) & 1u) ^ 1u);
     __syncwarp();
+  } else if (warp == 1 && !leader) {
+    // ---------------- peer: K-tail blocks (wgrad) ----------------
+    // Follows the producer's tile and stage sequence; for each tile's last K
+    // block waits for its own copy to land, zeroes the rows past the expert's
+    // end and arrives on the leader's stage barrier.
+    if constexpr (WG) {
+      int stage = 0;
+      uint32_t tail_par = 0;  // phase of each stage's tail barrier
+      for (int it = 0;; ++it) {
+        const int t = next_tile(it);
+        if (t < 0) break;
+        const PairTile ti = decode_pair<WG>(t, p, offs_s, tab_d, tab_w, tc);
+        bool ok = true;
+        for (int kb = 0; kb < ti.nk; ++kb) {
+          const int valid = ti.row_end - (ti.row0 + kb * BK);
+          if (valid < BK && !(p.stall && it == 0 && kb == 0)) {
+            uint8_t* sa = smem + stage * kPairStage;
+            uint8_t* sb = sa + kPairABytes;
+            const bool landed = __all_sync(
+                kFull, mbar_wait_bounded(&tailb[stage], (tail_par >> stage) & 1u, abort_flag,
+                                         status, wlim));
+            tail_par ^= 1u << stage;
+            if (!landed) {
+              ok = false;
+              break;
+            }
+            const int nkk = (valid + UK - 1) / UK;
+            zero_tail_rows(sa, sb, valid, nkk * UK - valid, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lead_full + 8u * stage);
+          }
+          if (++stage == STAGES) stage = 0;
+        }
+        if (!ok) break;
+      }
+    }
   } else if (warp == 1) {
     if (leader) {
       // ---------------- MMA issuer (leader only) ----------------
@@ -446,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
     auto release_acc = [&](uint32_t b) {
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead_tempty + 8u * b);
+      if (lane == 0) mbar_arrive_remote(lead_tempty + 8u * b);
     };
     for (int it = 0;; ++it) {
       const int t = next_tile(it);

@@ -554,13 +554,15 @@ bool wgrad_maps(Maps* m, const void* grad_rows, const void* in_rows, int rows_ca
 
 }  // namespace
 
-// LRMOE_GEMM_TWO_SM=1 in the environment selects the two-SM tiles of
-// gemm_pair.cu instead of the one-SM tiles of this file (both compute the same
-// result, bit for bit).
+// The grouped dgrad and wgrad run on the two-SM tiles of gemm_pair.cu (a pair of
+// SMs per 256 x 256 output tile).  LRMOE_GEMM_ONE_SM=1 in the environment selects
+// the one-SM tiles of this file instead (128 x 256 per SM; faster for the dgrads
+// of layers whose experts keep fewer than about 128 rows, where a 256-row tile
+// is mostly empty).  Both compute the same result, bit for bit.
 static bool one_sm_tiles() {
   static const bool v = [] {
-    const char* e = getenv("LRMOE_GEMM_TWO_SM");
-    return !(e != nullptr && e[0] == '1');
+    const char* e = getenv("LRMOE_GEMM_ONE_SM");
+    return e != nullptr && e[0] == '1';
   }();
   return v;
 }

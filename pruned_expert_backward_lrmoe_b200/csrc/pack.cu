@@ -10,6 +10,7 @@
 // on the device (offsets[E]) and is never read back by the host.
 #include "common.cuh"
 #include "launch.h"
+#include "rowreduce.cuh"
 
 namespace lrmoe {
 namespace {
@@ -145,9 +146,17 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ d
   const int wpb = blockDim.x >> 5;
   pdl_wait();
   pdl_trigger();
-  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+  const int stride = gridDim.x * wpb;
+  int t = blockIdx.x * wpb + (threadIdx.x >> 5);
+  // the next token's slots are loaded while this token's rows are in flight
+  int r_next = (t < T && lane < k) ? __ldg(pos + (size_t)t * k + lane) : -1;
+  for (; t < T; t += stride) {
     // retained rows of this token, in ascending slot order (k <= 32)
-    int r = lane < k ? pos[(size_t)t * k + lane] : -1;
+    int r = r_next;
+    {
+      const int tn = t + stride;
+      r_next = (tn < T && lane < k) ? __ldg(pos + (size_t)tn * k + lane) : -1;
+    }
     if (r >= rows_cap) {
       raise_status(status, LRMOE_ST_BAD_INDEX);
       r = -1;
@@ -247,12 +256,14 @@ cudaError_t launch_pack(const int32_t* perm, const int32_t* offsets, const float
                         cudaStream_t s) {
   const int per = dt == LRMOE_BF16 ? 8 : 4;
   const int VH = H / per, VI = I / per;
-  const int blocks = num_sms() * 8;
   auto X = static_cast<const uint4*>(x);
   auto D = static_cast<const uint4*>(dY);
   auto A = static_cast<const uint4*>(a);
   auto G = static_cast<const uint4*>(g);
   auto U = static_cast<const uint4*>(u);
+  // one resident wave (the row count lives on the device; a grid-stride loop)
+  const int blocks = dt == LRMOE_BF16 ? rowred::grid_for<pack_kernel<LRMOE_BF16>>(rows_cap)
+                                      : rowred::grid_for<pack_kernel<LRMOE_F32>>(rows_cap);
   auto kern = dt == LRMOE_BF16 ? pack_kernel<LRMOE_BF16> : pack_kernel<LRMOE_F32>;
   return launch_pdl(kern, dim3(blocks), dim3(256), 0, s, perm, offsets, E, w, T * k, k, X, D, VH,
                     A, G, U, VI, static_cast<uint4*>(Xp), static_cast<uint4*>(DYp),
@@ -270,7 +281,8 @@ cudaError_t launch_pack_wide(const int32_t* perm, const int32_t* offsets, const 
   const int VH = H / per, VI = I / per;
   const int W = 2 * VH + 3 * VI;
   uint4* base = static_cast<uint4*>(rows);
-  const int blocks = num_sms() * 8;
+  const int blocks = dt == LRMOE_BF16 ? rowred::grid_for<pack_kernel<LRMOE_BF16>>(rows_cap)
+                                      : rowred::grid_for<pack_kernel<LRMOE_F32>>(rows_cap);
   auto kern = dt == LRMOE_BF16 ? pack_kernel<LRMOE_BF16> : pack_kernel<LRMOE_F32>;
   return launch_pdl(kern, dim3(blocks), dim3(256), 0, s, perm, offsets, E, w, T * k, k,
                     static_cast<const uint4*>(x), static_cast<const uint4*>(dY), VH,
@@ -328,6 +340,8 @@ cudaError_t launch_unpack(const void* dXp, int rows_cap, const int32_t* pos, int
                           lrmoe_dtype dt, void* dX, uint32_t* status, cudaStream_t s) {
   const int per = dt == LRMOE_BF16 ? 8 : 4;
   const int VH = H / per;
+  // a warp per token (up to eight blocks per SM, then a grid-stride loop); one
+  // resident wave with two tokens per warp measured slower
   const int wpb = 8;
   int blocks = (T + wpb - 1) / wpb;
   const int maxb = num_sms() * 8;

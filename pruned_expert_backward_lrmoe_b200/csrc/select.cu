@@ -100,20 +100,35 @@ __global__ void __launch_bounds__(kScatterWarps * 32) chunk_scatter(
   __syncthreads();
   pdl_wait();
   pdl_trigger();
-  // per expert: total over chunks and the part before this chunk
-  for (int e = wid; e < E; e += kScatterWarps) {
-    const int32_t* row = cc + (size_t)e * nchunks;
-    int t_all = 0, t_pre = 0;
-    for (int c0 = 0; c0 < nchunks; c0 += 64) {
-      const int i0 = c0 + lane, i1 = c0 + 32 + lane;
-      const int v0 = i0 < nchunks ? __ldcg(row + i0) : 0;
-      const int v1 = i1 < nchunks ? __ldcg(row + i1) : 0;
-      t_all += __reduce_add_sync(kFull, v0 + v1);
-      t_pre += __reduce_add_sync(kFull, (i0 < c ? v0 : 0) + (i1 < c ? v1 : 0));
+  // per expert: total over chunks and the part before this chunk.  A warp takes
+  // kExpertsInFlight experts at a time with all their loads in flight (one
+  // round trip per group instead of one per expert).
+  constexpr int kExpertsInFlight = 8;
+  for (int e0 = wid * kExpertsInFlight; e0 < E; e0 += kScatterWarps * kExpertsInFlight) {
+    int t_all[kExpertsInFlight], t_pre[kExpertsInFlight];
+#pragma unroll
+    for (int u = 0; u < kExpertsInFlight; ++u) t_all[u] = t_pre[u] = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 32) {
+      const int ci = c0 + lane;
+      int v[kExpertsInFlight];
+#pragma unroll
+      for (int u = 0; u < kExpertsInFlight; ++u) {
+        const int e = e0 + u;
+        v[u] = (e < E && ci < nchunks) ? __ldcg(cc + (size_t)e * nchunks + ci) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < kExpertsInFlight; ++u) {
+        t_all[u] += __reduce_add_sync(kFull, v[u]);
+        t_pre[u] += __reduce_add_sync(kFull, ci < c ? v[u] : 0);
+      }
     }
     if (lane == 0) {
-      tot[e] = t_all;
-      pre[e] = t_pre;
+#pragma unroll
+      for (int u = 0; u < kExpertsInFlight; ++u)
+        if (e0 + u < E) {
+          tot[e0 + u] = t_all[u];
+          pre[e0 + u] = t_pre[u];
+        }
     }
   }
   __syncthreads();
@@ -214,6 +229,7 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
   extern __shared__ uint32_t sm_keys[];  // [kTopkSmemKeys]
   __shared__ int hist[2048];
   __shared__ int warp_gt[kTopkThreads / 32], warp_eq[kTopkThreads / 32];
+  __shared__ int warp_sum[kTopkThreads / 32];
   __shared__ int found_bin, found_above;
   pdl_wait();
   pdl_trigger();
@@ -281,13 +297,23 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
       }
     }
     __syncthreads();
-    if (wid == 0) {
-      // lane l owns the nb/32 bins below nb - 1 - l*nb/32 (descending key order)
-      const int per = nb >> 5;
-      const int top = nb - 1 - lane * per;
+    {
+      // thread t owns the nb/1024 bins just below nb - 1 - t*nb/1024 (descending
+      // key order); one block-wide scan of the per-thread sums finds the bin
+      const int per = nb / kTopkThreads;
+      const int top = nb - 1 - tid * per;
       int lsum = 0;
       for (int b = 0; b < per; ++b) lsum += hist[top - b];
-      const int incl = warp_incl_scan(lsum);
+      const int incl_w = warp_incl_scan(lsum);
+      if (lane == 31) warp_sum[wid] = incl_w;
+      __syncthreads();
+      if (wid == 0) {
+        const int x = lane < nw ? warp_sum[lane] : 0;
+        const int xi = warp_incl_scan(x);
+        if (lane < nw) warp_sum[lane] = xi - x;
+      }
+      __syncthreads();
+      const int incl = warp_sum[wid] + incl_w;
       const int excl = incl - lsum;
       if (excl < need && need <= incl) {
         int cum = excl;
