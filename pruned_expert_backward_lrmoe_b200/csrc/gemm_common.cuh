@@ -89,6 +89,9 @@ struct GemmParams {
   // block of their first tile, so that the MMA issuer's wait runs out
   unsigned long long wait_ns;
   int stall;
+  int part;             // dgrad: which row tiles of each expert (RowPart)
+  int late_wait;        // launched after another dgrad over other rows of the same
+                        // output: run first, wait for the preceding kernel at the end
 };
 
 template <int MODE>
@@ -150,7 +153,7 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     ti.e = e;
     ti.m0 = 0;
     ti.n0 = (local % tc.nt_d) * kBNT;
-    ti.row0 = offs[e] + (local / tc.nt_d) * BM;
+    ti.row0 = dgrad_tile_row0(offs[e], offs[e + 1] - offs[e], BM, p.part, local / tc.nt_d);
     ti.row_end = offs[e + 1];
     ti.nk = (p.Kd + BK - 1) / BK;
   }

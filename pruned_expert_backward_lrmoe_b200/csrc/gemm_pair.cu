@@ -96,7 +96,7 @@ __device__ __forceinline__ PairTile decode_pair(int t, const GemmParams& p, cons
     ti.e = e;
     ti.m0 = 0;
     ti.n0 = (local % tc.nt_d) * kBNT;
-    ti.row0 = offs[e] + (local / tc.nt_d) * kPairM;
+    ti.row0 = dgrad_tile_row0(offs[e], offs[e + 1] - offs[e], kPairM, p.part, local / tc.nt_d);
     ti.row_end = offs[e + 1];
     ti.nk = (p.Kd + BK - 1) / BK;
   }
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
     tc.tw = E * tc.mt_w * tc.nt_w;
   } else {
     tc.nt_d = (p.Nd + BN - 1) / BN;
-    tc.td = build_dgrad_tiles(p.offsets, E, kPairM, tc.nt_d, tab_d, scratch);
+    tc.td = build_dgrad_tiles(p.offsets, E, kPairM, tc.nt_d, tab_d, scratch, p.part);
   }
   tc.total = tc.td + tc.tw;
   for (int i = threadIdx.x; i <= E; i += blockDim.x) offs_s[i] = p.offsets[i];
@@ -646,7 +646,7 @@ cudaError_t launch_dgrad_pair(const void* rows, int rows_cap, const void* W,
                               const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
                               const void* Gp, const void* Up, void* out, uint32_t* status,
                               cudaStream_t s, const char** why, const int32_t* perm,
-                              int gu_rows) {
+                              int gu_rows, int part) {
   CUtensorMap a, b;
   if (!make_map_2d(&a, rows, (uint64_t)rows_cap, (uint64_t)K, 64, 128) ||
       !make_map_3d(&b, W, (uint64_t)E, (uint64_t)K, (uint64_t)N)) {
@@ -654,7 +654,8 @@ cudaError_t launch_dgrad_pair(const void* rows, int rows_cap, const void* W,
     return cudaErrorInvalidValue;
   }
   GemmParams prm{offsets, E, K, N, 0, 0, static_cast<const uint16_t*>(Gp),
-                 static_cast<const uint16_t*>(Up), perm, gu_rows, out, 0, nullptr, 1, 0, status, 0};
+                 static_cast<const uint16_t*>(Up), perm, gu_rows, out, 0, nullptr, 1, 0, status, 0,
+                 0, 0, part, 0};
   // an upper bound of the tile count (the real one is built on the device)
   const long long tiles =
       ((long long)rows_cap / kPairM + E) * ((N + kBNT - 1) / kBNT);

@@ -97,8 +97,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
     tmem_relinquish();
   }
   // everything above touches no global memory; from here on, earlier kernels' outputs
-  pdl_wait();
-  pdl_trigger();
+  // (a late-wait launch reads only outputs that were complete when it started, see
+  // GemmParams::late_wait, and waits for its predecessor at the end instead)
+  if (!p.late_wait) {
+    pdl_wait();
+    pdl_trigger();
+  }
   // tile tables
   TileCounts tc{0, 0, 0, 0, 0, 0};
   if constexpr (Tr::kHasW) {
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   }
   if constexpr (Tr::kHasD) {
     tc.nt_d = (p.Nd + BN - 1) / BN;
-    tc.td = build_dgrad_tiles(p.offsets, E, BM, tc.nt_d, tab_d, scratch);
+    tc.td = build_dgrad_tiles(p.offsets, E, BM, tc.nt_d, tab_d, scratch, p.part);
   }
   tc.total = tc.td + tc.tw;
   for (int i = threadIdx.x; i <= E; i += blockDim.x) offs_s[i] = p.offsets[i];
@@ -498,6 +502,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
       __threadfence();
     }
   }
+  if (p.late_wait) {
+    // this grid completes only after the kernel before it, so the next kernel in
+    // the stream sees both kernels' rows
+    pdl_wait();
+    pdl_trigger();
+  }
 }
 
 
@@ -567,13 +577,19 @@ static bool one_sm_tiles() {
   return v;
 }
 
+// Default: each expert's rows in 256-row tiles on pairs of SMs (gemm_pair.cu), and
+// a last tile of at most 128 rows on one SM in a second launch that runs as the
+// first drains (a 256-row tile would leave half of its pair idle there).
 cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
                             const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
                             const void* Gp, const void* Up, void* out, uint32_t* status,
                             cudaStream_t s, const char** why, const int32_t* perm, int gu_rows) {
-  if (!one_sm_tiles())
-    return launch_dgrad_pair(rows, rows_cap, W, offsets, E, K, N, epi, Gp, Up, out, status, s, why,
-                             perm, gu_rows);
+  const bool split = !one_sm_tiles();
+  if (split) {
+    const cudaError_t e = launch_dgrad_pair(rows, rows_cap, W, offsets, E, K, N, epi, Gp, Up, out,
+                                            status, s, why, perm, gu_rows, kRowsPairs);
+    if (e != cudaSuccess) return e;
+  }
   Maps m;
   if (!dgrad_maps(&m, rows, rows_cap, W, E, K, N)) {
     *why = "cuTensorMapEncodeTiled failed for a dgrad operand";
@@ -581,7 +597,8 @@ cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
   }
   m.aw = m.bw = m.out = m.ad;  // unused
   GemmParams prm{offsets, E, K, N, 0, 0, static_cast<const uint16_t*>(Gp),
-                 static_cast<const uint16_t*>(Up), perm, gu_rows, out, 0, nullptr, 1, 0, status, 0};
+                 static_cast<const uint16_t*>(Up), perm, gu_rows, out, 0, nullptr, 1, 0, status, 0,
+                 0, 0, split ? kRowsTails : kRowsAll, split ? 1 : 0};
   if (epi == LRMOE_EPI_SWIGLU_BWD) return launch_mode<kDgradSwiglu>(m, prm, s, num_sms());
   return launch_mode<kDgradStore>(m, prm, s, num_sms());
 }

@@ -43,14 +43,36 @@ __device__ __forceinline__ int block_scan_inplace(int* v, int n, int* scratch /*
   return total;
 }
 
-// dgrad (variable M): tiles of expert e = ceil(m_e / BM) * n_tiles, experts in order.
+// Which rows of each expert a dgrad launch covers (variable M).
+//   kRowsAll   : every row, in tiles of BM rows
+//   kRowsPairs : the 256-row tiles of a two-SM launch, without a last tile of at
+//                most 128 rows (m_e / 256 tiles, plus one if m_e % 256 > 128)
+//   kRowsTails : that last tile of at most 128 rows (m_e % 256 in (0, 128]), for a
+//                one-SM launch of 128-row tiles
+enum RowPart : int { kRowsAll = 0, kRowsPairs = 1, kRowsTails = 2 };
+
+__device__ __forceinline__ int dgrad_row_tiles(int m, int BM, int part) {
+  if (m <= 0) return 0;
+  if (part == kRowsPairs) return m / 256 + (m % 256 > 128 ? 1 : 0);
+  if (part == kRowsTails) return (m % 256 > 0 && m % 256 <= 128) ? 1 : 0;
+  return (m + BM - 1) / BM;
+}
+
+// First packed row of row tile j of expert e (rows [first, first + BM) clipped
+// to the expert's end).
+__device__ __forceinline__ int dgrad_tile_row0(int e_first, int m, int BM, int part, int j) {
+  if (part == kRowsTails) return e_first + m - m % 256;
+  return e_first + j * BM;
+}
+
+// dgrad (variable M): tiles of expert e = row tiles(m_e) * n_tiles, experts in order.
 // tstart[0..E] receives the exclusive prefix; returns the total tile count.
 __device__ __forceinline__ int build_dgrad_tiles(const int32_t* __restrict__ offsets, int E,
                                                  int BM, int n_tiles, int* tstart,
-                                                 int* scratch) {
+                                                 int* scratch, int part = kRowsAll) {
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int m = offsets[e + 1] - offsets[e];
-    tstart[e] = m > 0 ? ((m + BM - 1) / BM) * n_tiles : 0;
+    tstart[e] = dgrad_row_tiles(m, BM, part) * n_tiles;
   }
   __syncthreads();
   const int total = block_scan_inplace(tstart, E, scratch);

@@ -130,7 +130,8 @@ cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows
 cudaError_t launch_dgrad_pair(const void* rows, int rows_cap, const void* W,
                               const int32_t* offsets, int E, int K, int N, lrmoe_epilogue epi,
                               const void* Gp, const void* Up, void* out, uint32_t* status,
-                              cudaStream_t s, const char** why, const int32_t* perm, int gu_rows);
+                              cudaStream_t s, const char** why, const int32_t* perm, int gu_rows,
+                              int part);
 cudaError_t launch_wgrad_pair(const void* grad_rows, const void* in_rows, int rows_cap,
                               const int32_t* offsets, int E, int N1, int N2, float* dW,
                               int accumulate, uint32_t* status, cudaStream_t s, const char** why);
