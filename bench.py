@@ -47,8 +47,10 @@ UNIT = "retained pairs/s"
 DEFAULT_CONFIG = "sweep100"
 OTHER_CONFIGS = ("qwen", "glm", "skew")
 KERNELS = ("score", "select", "pack", "dgrad_swiglu", "wgrad_down", "wgrad_gu", "dgrad_x", "unpack")
-KERNEL_LAUNCHES = {"score": 1, "select": 4, "pack": 1, "dgrad_swiglu": 1, "wgrad_down": 1,
-                   "wgrad_gu": 1, "dgrad_x": 1, "unpack": 1}
+# kernel launches per call: selection is three kernels; each grouped dgrad is a
+# two-SM launch for the 256-row tiles plus a one-SM launch for experts' last tiles
+KERNEL_LAUNCHES = {"score": 1, "select": 3, "pack": 1, "dgrad_swiglu": 2, "wgrad_down": 1,
+                   "wgrad_gu": 1, "dgrad_x": 2, "unpack": 1}
 # C-ABI call of each step position (NVTX range names)
 CALL_NAMES = ("lrmoe_score", "lrmoe_select_quota", "lrmoe_pack", "lrmoe_grouped_dgrad[swiglu]",
               "lrmoe_grouped_wgrad[down]", "lrmoe_grouped_wgrad[gate|up]",
