@@ -138,7 +138,7 @@ _GEMM_SOURCES = ("gemm_tc.cu", "gemm_pair.cu", "gemm_common.cuh", "common.cuh", 
                  "launch.h")
 KERNEL_SOURCES = {
     "score": ("score.cu", "rowreduce.cuh", "common.cuh"),
-    "select": ("select.cu", "common.cuh"),
+    "select": ("select.cu", "grouped.cuh", "common.cuh"),
     "pack": ("pack.cu", "common.cuh"),
     "unpack": ("pack.cu", "common.cuh"),
     "dgrad_swiglu": _GEMM_SOURCES, "wgrad_down": _GEMM_SOURCES,

@@ -74,6 +74,7 @@ struct PairTile {
   int row_end;  // end of the expert's rows
   int m0, n0;   // wgrad: first output row (feature) of the pair tile; both: first column
   int nk;       // K blocks
+  int narrow;   // at most 128 output columns left: an N = 128 MMA, 64 B columns per CTA
 };
 
 template <bool WG>
@@ -90,6 +91,7 @@ __device__ __forceinline__ PairTile decode_pair(int t, const GemmParams& p, cons
     ti.row0 = offs[ti.e];
     ti.row_end = offs[ti.e + 1];
     ti.nk = (ti.row_end - ti.row0 + BK - 1) / BK;
+    ti.narrow = p.N2 - ti.n0 <= kHalfN;
   } else {
     const int e = find_group(tab_d, p.E, t);
     const int local = t - tab_d[e];
@@ -99,6 +101,7 @@ __device__ __forceinline__ PairTile decode_pair(int t, const GemmParams& p, cons
     ti.row0 = dgrad_tile_row0(offs[e], offs[e + 1] - offs[e], kPairM, p.part, local / tc.nt_d);
     ti.row_end = offs[e + 1];
     ti.nk = (p.Kd + BK - 1) / BK;
+    ti.narrow = p.Nd - ti.n0 <= kHalfN;
   }
   return ti;
 }
@@ -284,21 +287,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
         const bool tail = WG && valid < BK;
         const int a_c0 = WG ? ti.m0 + (int)rank * BM : kb * BK;  // A coordinates of this CTA
         const int a_c1 = WG ? r : ti.row0 + (int)rank * BM;
-        const int b_col = ti.n0 + (int)rank * kHalfN;
+        // B columns of this CTA: 128 (two 64-column boxes), or 64 on a narrow tile
+        const int b_col = ti.n0 + (int)rank * (ti.narrow ? 64 : kHalfN);
+        const uint32_t cta_bytes = kPairABytes + (ti.narrow ? kPairBBytes / 2 : kPairBBytes);
         if (leader) {
           if (lane == 0) {
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-            mbar_arrive_expect_tx(&full[stage], kPairStage + (tail ? 0 : kPairStage));
+            mbar_arrive_expect_tx(&full[stage], cta_bytes + (tail ? 0u : cta_bytes));
             if constexpr (WG) {
               tma_load_2d(sa, &tmA, &full[stage], a_c0, a_c1);
               tma_load_2d(sa + 8192, &tmA, &full[stage], a_c0 + 64, a_c1);
               tma_load_2d(sb, &tmB, &full[stage], b_col, r);
-              tma_load_2d(sb + 8192, &tmB, &full[stage], b_col + 64, r);
+              if (!ti.narrow) tma_load_2d(sb + 8192, &tmB, &full[stage], b_col + 64, r);
             } else {
               tma_load_2d(sa, &tmA, &full[stage], a_c0, a_c1);
               tma_load_3d(sb, &tmB, &full[stage], b_col, kb * BK, ti.e);
-              tma_load_3d(sb + 8192, &tmB, &full[stage], b_col + 64, kb * BK, ti.e);
+              if (!ti.narrow) tma_load_3d(sb + 8192, &tmB, &full[stage], b_col + 64, kb * BK, ti.e);
             }
           }
         } else if (!tail) {
@@ -308,11 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
               tma_load_2d_pair(sa, &tmA, fb, a_c0, a_c1);
               tma_load_2d_pair(sa + 8192, &tmA, fb, a_c0 + 64, a_c1);
               tma_load_2d_pair(sb, &tmB, fb, b_col, r);
-              tma_load_2d_pair(sb + 8192, &tmB, fb, b_col + 64, r);
+              if (!ti.narrow) tma_load_2d_pair(sb + 8192, &tmB, fb, b_col + 64, r);
             } else {
               tma_load_2d_pair(sa, &tmA, fb, a_c0, a_c1);
               tma_load_3d_pair(sb, &tmB, fb, b_col, kb * BK, ti.e);
-              tma_load_3d_pair(sb + 8192, &tmB, fb, b_col + 64, kb * BK, ti.e);
+              if (!ti.narrow) tma_load_3d_pair(sb + 8192, &tmB, fb, b_col + 64, kb * BK, ti.e);
             }
             mbar_arrive_cluster_relaxed(fb);  // the bytes themselves are counted by the barrier
           }
@@ -324,11 +329,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
             if (lane == 0) {
               tail_used |= 1u << stage;
               tail_next ^= 1u << stage;
-              mbar_arrive_expect_tx(&tailb[stage], kPairStage);
+              mbar_arrive_expect_tx(&tailb[stage], cta_bytes);
               tma_load_2d(sa, &tmA, &tailb[stage], a_c0, a_c1);
               tma_load_2d(sa + 8192, &tmA, &tailb[stage], a_c0 + 64, a_c1);
               tma_load_2d(sb, &tmB, &tailb[stage], b_col, r);
-              tma_load_2d(sb + 8192, &tmB, &tailb[stage], b_col + 64, r);
+              if (!ti.narrow) tma_load_2d(sb + 8192, &tmB, &tailb[stage], b_col + 64, r);
             }
           }
         }
@@ -389,7 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
   } else if (warp == 1) {
     if (leader) {
       // ---------------- MMA issuer (leader only) ----------------
-      constexpr uint32_t idesc = idesc_bf16_f32(kPairM, BN, WG, true);
+      constexpr uint32_t idesc_full = idesc_bf16_f32(kPairM, BN, WG, true);
+      constexpr uint32_t idesc_narrow = idesc_bf16_f32(kPairM, kHalfN, WG, true);
       const uint32_t peer_empty = cluster_addr(empty, 1);
       const uint32_t peer_tfull = cluster_addr(tfull, 1);
       int stage = 0;
@@ -442,7 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
               const uint64_t adesc = WG ? smem_desc_sw128(a_addr + kk * 2048, 8192, 1024)
                                         : smem_desc_sw128(a_addr + kk * 32, 16, 1024);
               const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, 8192, 1024);
-              tc_mma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_f16_pair(d_tmem, adesc, bdesc, ti.narrow ? idesc_narrow : idesc_full,
+                              (kb | kk) != 0 ? 1u : 0u);
             }
             // the stage is free in both CTAs once these MMAs have read it
             tc_commit_pair(smem_u32(&empty[stage]));

@@ -65,38 +65,8 @@ __device__ __forceinline__ void scale_row(uint4* __restrict__ dst, const uint4* 
   for (; c < V; c += 32) dst[c] = scale_vec<DT>(__ldg(src + c), w);
 }
 
-// X_p row = x row and DY_p row = RNE(w * dY row) (X_p optional), four vectors of
-// each in flight per lane and round trip.
 template <lrmoe_dtype DT>
-__device__ __forceinline__ void copy_scale_rows(uint4* __restrict__ xdst,
-                                                const uint4* __restrict__ xsrc,
-                                                uint4* __restrict__ ddst,
-                                                const uint4* __restrict__ dsrc, int V, float w,
-                                                int lane) {
-  constexpr int U = 4;
-  for (int c0 = lane; c0 < V; c0 += 32 * U) {
-    uint4 xv[U], dv[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = c0 + 32 * u;
-      if (c < V) {
-        if (xdst) xv[u] = __ldg(xsrc + c);
-        dv[u] = __ldg(dsrc + c);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c = c0 + 32 * u;
-      if (c < V) {
-        if (xdst) xdst[c] = xv[u];
-        ddst[c] = scale_vec<DT>(dv[u], w);
-      }
-    }
-  }
-}
-
-template <lrmoe_dtype DT>
-__global__ void __launch_bounds__(256, 4) pack_kernel(
+__global__ void __launch_bounds__(256) pack_kernel(
     const int32_t* __restrict__ perm, const int32_t* __restrict__ offsets, int E,
     const float* __restrict__ w, int P, int k, const uint4* __restrict__ x,
     const uint4* __restrict__ dY, int VH, const uint4* __restrict__ a,
@@ -112,13 +82,8 @@ __global__ void __launch_bounds__(256, 4) pack_kernel(
     if (blockIdx.x == 0 && threadIdx.x == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
     M = rows_cap;
   }
-  const int stride = gridDim.x * wpb;
-  int r = blockIdx.x * wpb + (threadIdx.x >> 5);
-  // the next row's pair id is loaded while this row's data is in flight
-  int p_next = r < M ? __ldg(perm + r) : 0;
-  for (; r < M; r += stride) {
-    const int p = p_next;
-    p_next = r + stride < M ? __ldg(perm + r + stride) : 0;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < M; r += gridDim.x * wpb) {
+    const int p = perm[r];
     if (p < 0 || p >= P) {
       if (lane == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
       continue;
@@ -127,11 +92,10 @@ __global__ void __launch_bounds__(256, 4) pack_kernel(
     const float wp = __ldg(w + p);
     const size_t rr = (size_t)r;
     // output row strides: ldH for X_p, DY_p and ldI for A_p, G_p, U_p (16-byte
-    // vectors); VH and VI for dense blocks, the wide-row width for exchange rows.
-    // X_p, A_p are optional (the gathering wgrad can read x, a in place).
-    copy_scale_rows<DT>(Xp ? Xp + rr * ldH : nullptr, x + (size_t)t * VH, DYp + rr * ldH,
-                        dY + (size_t)t * VH, VH, wp, lane);
-    if (Ap) copy_row(Ap + rr * ldI, a + (size_t)p * VI, VI, lane);
+    // vectors); VH and VI for dense blocks, the wide-row width for exchange rows
+    if (Xp) copy_row(Xp + rr * ldH, x + (size_t)t * VH, VH, lane);  // X_p, A_p optional: the
+    scale_row<DT>(DYp + rr * ldH, dY + (size_t)t * VH, VH, wp, lane);
+    if (Ap) copy_row(Ap + rr * ldI, a + (size_t)p * VI, VI, lane);  // wgrad can gather them
     if (Gp) copy_row(Gp + rr * ldI, g + (size_t)p * VI, VI, lane);  // optional: the SwiGLU
     if (Up) copy_row(Up + rr * ldI, u + (size_t)p * VI, VI, lane);  // epilogue can gather g, u
   }
@@ -168,35 +132,30 @@ __device__ __forceinline__ uint4 to_vec(const float (&acc)[DT == LRMOE_BF16 ? 8 
 }
 
 // dX[t] = sum over retained slots j (ascending) of dXp[pos[t*k+j]], fp32, rounded once.
-// Work unit = (token, column slice): a token's 32-vector column chunks are split
-// into S slices handled by S warps.  A unit's loads form one list, chunk by chunk,
+// A token's loads form one list, column chunk by column chunk (32 vectors each),
 // retained rows in ascending slot order inside a chunk; the warp issues
-// kUnpackLoads of them at once, so a unit with n retained rows and C chunks needs
-// about ceil(n * C / kUnpackLoads) memory round trips, plus one for the slots,
-// which are loaded one unit ahead.
+// kUnpackLoads of them at once, so a token with n retained rows needs about
+// ceil(n * chunks / kUnpackLoads) memory round trips rather than one per chunk.
 template <lrmoe_dtype DT>
 __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ dXp, int rows_cap,
                                                      const int32_t* __restrict__ pos, int T,
-                                                     int k, int VH, int S,
-                                                     uint4* __restrict__ dX,
+                                                     int k, int VH, uint4* __restrict__ dX,
                                                      uint32_t* __restrict__ status) {
   constexpr int PER = DT == LRMOE_BF16 ? 8 : 4;
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   pdl_wait();
   pdl_trigger();
-  const int nch = (VH + 31) >> 5;
-  const long long units = (long long)T * S;
   const int stride = gridDim.x * wpb;
-  long long u = (long long)blockIdx.x * wpb + (threadIdx.x >> 5);
-  int r_next = (u < units && lane < k) ? __ldg(pos + (size_t)(u / S) * k + lane) : -1;
-  for (; u < units; u += stride) {
-    const int t = (int)(u / S), h = (int)(u - (long long)t * S);
+  int t = blockIdx.x * wpb + (threadIdx.x >> 5);
+  // the next token's slots are loaded while this token's rows are in flight
+  int r_next = (t < T && lane < k) ? __ldg(pos + (size_t)t * k + lane) : -1;
+  for (; t < T; t += stride) {
     // retained rows of this token, in ascending slot order (k <= 32)
     int r = r_next;
     {
-      const long long un = u + stride;
-      r_next = (un < units && lane < k) ? __ldg(pos + (size_t)(un / S) * k + lane) : -1;
+      const int tn = t + stride;
+      r_next = (tn < T && lane < k) ? __ldg(pos + (size_t)tn * k + lane) : -1;
     }
     if (r >= rows_cap) {
       raise_status(status, LRMOE_ST_BAD_INDEX);
@@ -213,19 +172,17 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint4* __restrict__ d
         todo &= todo - 1;
       }
     }
-    const int ch_lo = h * nch / S, ch_hi = (h + 1) * nch / S;  // this slice's chunks
     uint4* __restrict__ out = dX + (size_t)t * VH;
     if (nrows == 0) {
-      for (int c = (ch_lo << 5) + lane; c < VH && c < (ch_hi << 5); c += 32)
-        out[c] = make_uint4(0, 0, 0, 0);
+      for (int c = lane; c < VH; c += 32) out[c] = make_uint4(0, 0, 0, 0);
       continue;
     }
-    // item i = (chunk ch_lo + i / nrows, row i % nrows); warp-uniform bookkeeping
-    const int items = (ch_hi - ch_lo) * nrows;
+    // item i = (chunk i / nrows, row i % nrows); nrows, items, ch and ri are warp-uniform
+    const int items = ((VH + 31) >> 5) * nrows;
     float acc[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
-    int ch = ch_lo, ri = 0;  // chunk and row of item i0
+    int ch = 0, ri = 0;  // chunk and row of item i0
     for (int i0 = 0; i0 < items; i0 += kUnpackLoads) {
       uint4 v[kUnpackLoads];
       {
@@ -383,16 +340,15 @@ cudaError_t launch_unpack(const void* dXp, int rows_cap, const int32_t* pos, int
                           lrmoe_dtype dt, void* dX, uint32_t* status, cudaStream_t s) {
   const int per = dt == LRMOE_BF16 ? 8 : 4;
   const int VH = H / per;
-  // two warps per token (column halves) once a row has four or more 32-vector
-  // chunks; up to eight blocks per SM, then a grid-stride loop
-  const int S = ((VH + 31) / 32) >= 4 ? 2 : 1;
+  // a warp per token (up to eight blocks per SM, then a grid-stride loop); one
+  // resident wave with two tokens per warp measured slower
   const int wpb = 8;
-  long long blocks = ((long long)T * S + wpb - 1) / wpb;
+  int blocks = (T + wpb - 1) / wpb;
   const int maxb = num_sms() * 8;
   if (blocks > maxb) blocks = maxb;
   auto kern = dt == LRMOE_BF16 ? unpack_kernel<LRMOE_BF16> : unpack_kernel<LRMOE_F32>;
-  return launch_pdl(kern, dim3((unsigned)blocks), dim3(256), 0, s, static_cast<const uint4*>(dXp),
-                    rows_cap, pos, T, k, VH, S, static_cast<uint4*>(dX), status);
+  return launch_pdl(kern, dim3(blocks), dim3(256), 0, s, static_cast<const uint4*>(dXp), rows_cap,
+                    pos, T, k, VH, static_cast<uint4*>(dX), status);
 }
 
 }  // namespace lrmoe
