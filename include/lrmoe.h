@@ -40,6 +40,12 @@
  *   - topk_idx < 0 marks an empty slot (no pair).
  *   - Feature sizes H, I (and the GEMM sizes K, N, N1, N2) are multiples of 8
  *     elements for bf16 and of 4 for fp32.
+ *   - Checked-index debug build (liblrmoe_checked.so, the same ABI compiled
+ *     with -DLRMOE_CHECKED): indices the kernels derive from their inputs or
+ *     from their own scans are also bounds-checked before use, including the
+ *     grouped GEMMs' offsets (offsets[0] >= 0, rising, offsets[E] <= rows_cap;
+ *     otherwise the launch computes nothing).  A failed check skips the access
+ *     and sets LRMOE_ST_BAD_INDEX.  The normal build trusts those contracts.
  */
 #ifndef LRMOE_H
 #define LRMOE_H
@@ -74,7 +80,7 @@ typedef enum {
 #define LRMOE_ST_BAD_QUOTA  2u /* some quota < 0 (treated as 0) */
 #define LRMOE_ST_NONFINITE  4u /* some score was +Inf or NaN */
 #define LRMOE_ST_TIMEOUT    8u /* a bounded device-side wait gave up; outputs invalid */
-#define LRMOE_ST_BAD_INDEX 16u /* a perm/pos entry was out of range and was skipped */
+#define LRMOE_ST_BAD_INDEX 16u /* an index (perm/pos entry; checked build: any) was out of range; skipped */
 
 /* Library version, (major << 16) | minor. */
 int lrmoe_version(void);

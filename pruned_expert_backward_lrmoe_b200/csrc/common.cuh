@@ -19,6 +19,23 @@ __device__ __forceinline__ void raise_status(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);
 }
 
+// Checked-index build (compiled with -DLRMOE_CHECKED, library liblrmoe_checked.so):
+// an index that a kernel takes from its inputs or from one of its own scans is
+// compared with the extent of the buffer it addresses before the access; outside
+// it, the access is skipped and LRMOE_ST_BAD_INDEX is raised.  The normal build
+// compiles the check away (the index is trusted, as the header's contracts say).
+#ifdef LRMOE_CHECKED
+constexpr bool kChecked = true;
+__device__ __forceinline__ bool idx_ok(long long i, long long n, uint32_t* status) {
+  if (i >= 0 && i < n) return true;
+  raise_status(status, LRMOE_ST_BAD_INDEX);
+  return false;
+}
+#else
+constexpr bool kChecked = false;
+__device__ __forceinline__ bool idx_ok(long long, long long, uint32_t*) { return true; }
+#endif
+
 // ---------------------------------------------------------------------------
 // storage types
 // ---------------------------------------------------------------------------

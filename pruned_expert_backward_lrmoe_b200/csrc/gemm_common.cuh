@@ -92,6 +92,7 @@ struct GemmParams {
   int part;             // dgrad: which row tiles of each expert (RowPart)
   int late_wait;        // launched after another dgrad over other rows of the same
                         // output: run first, wait for the preceding kernel at the end
+  int rows_cap;         // rows of the packed operands (the tensor maps' row extent)
 };
 
 template <int MODE>

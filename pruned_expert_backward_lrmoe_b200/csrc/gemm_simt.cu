@@ -21,7 +21,8 @@ __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf
 __global__ void __launch_bounds__(NT) dgrad_simt_kernel(
     const float* __restrict__ rows, const float* __restrict__ W,
     const int32_t* __restrict__ offsets, int E, int K, int N, int epi,
-    const float* __restrict__ Gp, const float* __restrict__ Up, float* __restrict__ out) {
+    const float* __restrict__ Gp, const float* __restrict__ Up, float* __restrict__ out,
+    int rows_cap, uint32_t* __restrict__ status) {
   __shared__ int tstart[kMaxExperts + 1];
   __shared__ int scratch[33];
   __shared__ float As[BK][BM + 4];
@@ -29,7 +30,8 @@ __global__ void __launch_bounds__(NT) dgrad_simt_kernel(
   pdl_wait();
   pdl_trigger();
   const int n_tiles = (N + BN - 1) / BN;
-  const int total = build_dgrad_tiles(offsets, E, BM, n_tiles, tstart, scratch);
+  const int total = offsets_invalid(offsets, E, rows_cap, status)
+                        ? 0 : build_dgrad_tiles(offsets, E, BM, n_tiles, tstart, scratch);
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   for (int t = blockIdx.x; t < total; t += gridDim.x) {
     const int e = find_group(tstart, E, t);
@@ -98,14 +100,14 @@ __global__ void __launch_bounds__(NT) dgrad_simt_kernel(
 __global__ void __launch_bounds__(NT) wgrad_simt_kernel(
     const float* __restrict__ grad, const float* __restrict__ in,
     const int32_t* __restrict__ offsets, int E, int N1, int N2, float* __restrict__ dW,
-    int accumulate) {
+    int accumulate, int rows_cap, uint32_t* __restrict__ status) {
   __shared__ float As[BK][BM];
   __shared__ float Bs[BK][BN];
   pdl_wait();
   pdl_trigger();
   const int m_tiles = (N1 + BM - 1) / BM, n_tiles = (N2 + BN - 1) / BN;
   const int per_e = m_tiles * n_tiles;
-  const int total = per_e * E;
+  const int total = offsets_invalid(offsets, E, rows_cap, status) ? 0 : per_e * E;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   for (int t = blockIdx.x; t < total; t += gridDim.x) {
     const int e = t / per_e;
@@ -159,24 +161,20 @@ cudaError_t launch_dgrad_simt(const void* rows, int rows_cap, const void* W,
                               const int32_t* offsets, int E, int K, int N, lrmoe_dtype dt,
                               lrmoe_epilogue epi, const void* Gp, const void* Up, void* out,
                               uint32_t* status, cudaStream_t s) {
-  (void)rows_cap;
   (void)dt;
-  (void)status;
   return launch_pdl(dgrad_simt_kernel, dim3(num_sms() * 4), dim3(NT), 0, s,
                     static_cast<const float*>(rows), static_cast<const float*>(W), offsets, E, K,
                     N, (int)epi, static_cast<const float*>(Gp), static_cast<const float*>(Up),
-                    static_cast<float*>(out));
+                    static_cast<float*>(out), rows_cap, status);
 }
 
 cudaError_t launch_wgrad_simt(const void* grad_rows, const void* in_rows, int rows_cap,
                               const int32_t* offsets, int E, int N1, int N2, lrmoe_dtype dt,
                               float* dW, int accumulate, uint32_t* status, cudaStream_t s) {
-  (void)rows_cap;
   (void)dt;
-  (void)status;
   return launch_pdl(wgrad_simt_kernel, dim3(num_sms() * 4), dim3(NT), 0, s,
                     static_cast<const float*>(grad_rows), static_cast<const float*>(in_rows),
-                    offsets, E, N1, N2, dW, accumulate);
+                    offsets, E, N1, N2, dW, accumulate, rows_cap, status);
 }
 
 }  // namespace lrmoe

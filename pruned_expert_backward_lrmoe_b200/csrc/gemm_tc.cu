@@ -120,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_tc(
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (offsets_invalid(offs_s, E, p.rows_cap, status)) tc.total = tc.td = tc.tw = 0;
   const uint32_t tmem_base = *tmem_slot;
 
   // Tile of the it-th round for the MMA and epilogue warps (-1: no more tiles).
@@ -599,6 +600,7 @@ cudaError_t launch_dgrad_tc(const void* rows, int rows_cap, const void* W,
   GemmParams prm{offsets, E, K, N, 0, 0, static_cast<const uint16_t*>(Gp),
                  static_cast<const uint16_t*>(Up), perm, gu_rows, out, 0, nullptr, 1, 0, status, 0,
                  0, 0, split ? kRowsTails : kRowsAll, split ? 1 : 0};
+  prm.rows_cap = rows_cap;
   if (epi == LRMOE_EPI_SWIGLU_BWD) return launch_mode<kDgradSwiglu>(m, prm, s, num_sms());
   return launch_mode<kDgradStore>(m, prm, s, num_sms());
 }
@@ -613,6 +615,7 @@ cudaError_t launch_dgrad_stall_tc(const void* rows, int rows_cap, const void* W,
   m.aw = m.bw = m.out = m.ad;  // unused
   GemmParams prm{offsets, E, K, N, 0, 0, nullptr, nullptr, nullptr, 0, out, 0, nullptr, 1, 0,
                  status, 0, wait_ns, 1};
+  prm.rows_cap = rows_cap;
   return launch_mode<kDgradStore>(m, prm, s, num_sms());
 }
 
@@ -633,6 +636,7 @@ cudaError_t launch_wgrad_tc(const void* grad_rows, const void* in_rows, int rows
   if (total < grid) grid = (int)total;
   GemmParams prm{offsets, E, 0, 0, N1, N2, nullptr, nullptr, nullptr, 0, nullptr, accumulate,
                  nullptr, 1, 0, status, 0};
+  prm.rows_cap = rows_cap;
   return launch_mode<kWgrad>(m, prm, s, grid);
 }
 
@@ -653,6 +657,7 @@ cudaError_t launch_wgrad_gather_tc(const void* grad_rows, int rows_cap, const in
   if (total < grid) grid = (int)total;
   GemmParams prm{offsets, E, 0, 0, N1, N2, nullptr, nullptr, perm, 0, nullptr, accumulate,
                  static_cast<const uint16_t*>(src), src_div, perm_max, status, 0};
+  prm.rows_cap = rows_cap;
   return launch_mode<kWgradGather>(m, prm, s, grid);
 }
 
@@ -670,6 +675,7 @@ cudaError_t launch_dgrad_wgrad_tc(const void* grad_rows, int rows_cap, const voi
   GemmParams prm{offsets, E, K, N, K, N2, static_cast<const uint16_t*>(Gp),
                  static_cast<const uint16_t*>(Up), nullptr, 0, out, accumulate, nullptr, 1, 0,
                  status, 0};
+  prm.rows_cap = rows_cap;
   if (epi == LRMOE_EPI_SWIGLU_BWD) return launch_mode<kFusedSwiglu>(m, prm, s, num_sms());
   return launch_mode<kFusedStore>(m, prm, s, num_sms());
 }

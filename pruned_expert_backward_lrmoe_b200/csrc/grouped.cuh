@@ -43,6 +43,23 @@ __device__ __forceinline__ int block_scan_inplace(int* v, int n, int* scratch /*
   return total;
 }
 
+// Checked-index build: offsets must rise from offsets[0] >= 0 to offsets[E] <=
+// rows_cap.  Block-wide; true (and LRMOE_ST_BAD_INDEX raised) when they do not,
+// in which case the launch computes no tile.  Always false in the normal build.
+__device__ __forceinline__ bool offsets_invalid(const int32_t* offs, int E, int rows_cap,
+                                                uint32_t* status) {
+  if constexpr (!kChecked) {
+    return false;
+  } else {
+    bool bad = false;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) bad |= offs[i] > offs[i + 1];
+    if (threadIdx.x == 0) bad |= offs[0] < 0 || offs[E] > rows_cap;
+    const bool any = __syncthreads_or(bad);
+    if (any && blockIdx.x == 0 && threadIdx.x == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
+    return any;
+  }
+}
+
 // Which rows of each expert a dgrad launch covers (variable M).
 //   kRowsAll   : every row, in tiles of BM rows
 //   kRowsPairs : the 256-row tiles of a two-SM launch, without a last tile of at

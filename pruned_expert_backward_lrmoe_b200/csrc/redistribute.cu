@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(256) dest_scatter_kernel(
     const int32_t* __restrict__ plan, const int32_t* __restrict__ start, int E, int G,
     int rows_cap, const int32_t* __restrict__ dest_offsets,
     const int32_t* __restrict__ dest_expert_offsets, int32_t* __restrict__ perm_dest,
-    int32_t* __restrict__ row_dest) {
+    int32_t* __restrict__ row_dest, uint32_t* __restrict__ status) {
   pdl_wait();
   pdl_trigger();
   int M = offsets[E];
@@ -174,9 +174,11 @@ __global__ void __launch_bounds__(256) dest_scatter_kernel(
         const long long first = base > c ? base : c;
         const long long slot = dest_offsets[g] + dest_expert_offsets[(size_t)g * (E + 1) + e] +
                                (gi - first);
-        if (slot < rows_cap) {
+        if (slot >= 0 && slot < rows_cap) {
           perm_dest[slot] = perm[r];
           if (row_dest) row_dest[r] = (int32_t)slot;
+        } else if (kChecked) {
+          raise_status(status, LRMOE_ST_BAD_INDEX);
         }
         break;
       }
@@ -298,7 +300,7 @@ cudaError_t launch_split_by_destination(const int32_t* perm, const int32_t* offs
   const int blocks = num_sms() * 4;
   return launch_pdl(dest_scatter_kernel, dim3(blocks), dim3(256), 0, s, perm, offsets, plan, start,
                     E, G, rows_cap, (const int32_t*)dest_offsets,
-                    (const int32_t*)dest_expert_offsets, perm_dest, row_dest);
+                    (const int32_t*)dest_expert_offsets, perm_dest, row_dest, status);
 }
 
 cudaError_t launch_group_received(const int32_t* tab, int G, int E, int rows_cap, int32_t* order,

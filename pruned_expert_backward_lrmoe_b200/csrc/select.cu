@@ -200,8 +200,10 @@ __global__ void __launch_bounds__(kScatterWarps * 32) chunk_scatter(
       if (valid) {
         base = mine[e];
         const int dst = base + __popc(m & lt);
-        seg_p[dst] = p;
-        seg_key[dst] = sv[s];
+        if (idx_ok(dst, P, status)) {
+          seg_p[dst] = p;
+          seg_key[dst] = sv[s];
+        }
       }
       __syncwarp();
       if (valid && lane == __ffs(m) - 1) mine[e] = base + __popc(m);
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
     const int32_t* __restrict__ counts, const int32_t* __restrict__ kept,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ seg_start,
     const int32_t* __restrict__ seg_p, const uint32_t* __restrict__ seg_key,
-    int32_t* __restrict__ perm, int32_t* __restrict__ pos) {
+    int32_t* __restrict__ perm, int32_t* __restrict__ pos, int P, uint32_t* __restrict__ status) {
   extern __shared__ uint32_t sm_keys[];  // [kTopkSmemKeys]
   __shared__ int hist[2048];
   __shared__ int warp_gt[kTopkThreads / 32], warp_eq[kTopkThreads / 32];
@@ -242,17 +244,23 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
   const int nt = blockDim.x, nw = nt >> 5;
   const int32_t* sp = seg_p + s0;
   const uint32_t* sk = seg_key + s0;
+  if (kChecked && !(c >= 0 && m >= 0 && m <= c && idx_ok(s0, P - c + 1, status) &&
+                    idx_ok(out0, P - m + 1, status))) {
+    if (tid == 0) raise_status(status, LRMOE_ST_BAD_INDEX);
+    return;
+  }
 
   if (m == c) {  // everything stays, already in ascending p
     for (int i = tid; i < c; i += nt) {
       const int p = sp[i];
       perm[out0 + i] = p;
-      pos[p] = out0 + i;
+      if (idx_ok(p, P, status)) pos[p] = out0 + i;
     }
     return;
   }
   if (m == 0) {
-    for (int i = tid; i < c; i += nt) pos[sp[i]] = -1;
+    for (int i = tid; i < c; i += nt)
+      if (idx_ok(sp[i], P, status)) pos[sp[i]] = -1;
     return;
   }
 
@@ -374,8 +382,8 @@ __global__ void __launch_bounds__(kTopkThreads) expert_topk(
       const int kept_eq_before = min(eq_rank, need_eq);
       const int row = out0 + gt_before + __popc(mgt & lt) + kept_eq_before;
       perm[row] = p;
-      pos[p] = row;
-    } else if (in) {
+      if (idx_ok(p, P, status)) pos[p] = row;
+    } else if (in && idx_ok(p, P, status)) {
       pos[p] = -1;
     }
     gt_before += __popc(mgt);
@@ -424,7 +432,7 @@ static cudaError_t enqueue_select(const SelectWs& L, const int32_t* idx, const f
                     static_cast<const int32_t*>(counts), static_cast<const int32_t*>(kept),
                     static_cast<const int32_t*>(offsets), static_cast<const int32_t*>(seg_start),
                     static_cast<const int32_t*>(seg_p), static_cast<const uint32_t*>(seg_key),
-                    perm, pos);
+                    perm, pos, P, status);
 }
 
 SelectWs select_ws_layout(int T, int k, int E) {

@@ -14,7 +14,9 @@ from typing import Dict, Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblrmoe.so")
+# LRMOE_CHECKED=1 selects the checked-index debug build (see build.py --checked)
+LIB_PATH = os.path.join(_HERE, "liblrmoe_checked.so" if os.environ.get("LRMOE_CHECKED") == "1"
+                        else "liblrmoe.so")
 
 LRMOE_OK, LRMOE_ERR_INVALID_ARG, LRMOE_ERR_UNSUPPORTED, LRMOE_ERR_CUDA, LRMOE_ERR_WORKSPACE = range(5)
 LRMOE_F32, LRMOE_BF16 = 0, 1
@@ -58,7 +60,8 @@ def load() -> ctypes.CDLL:
         return _lib
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(f"{LIB_PATH} is missing: build it with "
-                           "`python -m pruned_expert_backward_lrmoe_b200.build`")
+                           "`python -m pruned_expert_backward_lrmoe_b200.build`"
+                           + (" --checked" if LIB_PATH.endswith("_checked.so") else ""))
     lib = ctypes.CDLL(LIB_PATH)
     P, I, Z, U32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint32
     lib.lrmoe_version.restype = I

@@ -46,12 +46,14 @@ def device_inputs(layer, device="cuda"):
     }
 
 
-def run_steps(layer, inp=None, poison=True):
-    """Run a1..a5 one entry point at a time; returns the device buffers."""
+def run_steps(layer, inp=None, poison=True, out=None):
+    """Run a1..a5 one entry point at a time; returns the device buffers (`out`:
+    buffers laid out like alloc_buffers' to use instead of fresh ones)."""
     s = layer.spec
     tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
     inp = inp or device_inputs(layer)
-    out = L.alloc_buffers(s.T, s.k, s.E, s.H, s.I, tdt)
+    if out is None:
+        out = L.alloc_buffers(s.T, s.k, s.E, s.H, s.I, tdt)
     if poison:  # unwritten memory must not leak into results
         for k_, v in out.items():
             if k_ in ("status",):
@@ -80,11 +82,12 @@ def run_steps(layer, inp=None, poison=True):
     return out
 
 
-def run_chain(layer, inp=None):
+def run_chain(layer, inp=None, out=None):
     s = layer.spec
     tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
     inp = inp or device_inputs(layer)
-    out = L.alloc_buffers(s.T, s.k, s.E, s.H, s.I, tdt)
+    if out is None:
+        out = L.alloc_buffers(s.T, s.k, s.E, s.H, s.I, tdt)
     out["status"].zero_()
     L.lrmoe_pruned_backward(inp, out)
     torch.cuda.synchronize()

@@ -32,6 +32,17 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) <= set(L.EXPORTS)
 
 
+def test_checked_build_exports_the_same_symbols():
+    """The checked-index debug library (-DLRMOE_CHECKED) builds and exports the
+    same ABI; the binding selects it with LRMOE_CHECKED=1."""
+    path = B.build(checked=True)
+    assert path.endswith("liblrmoe_checked.so") and os.path.exists(path)
+    chk = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(chk, n), n
+    assert chk.lrmoe_version() == L.load().lrmoe_version()
+
+
 def test_version_and_strings(lib):
     assert lib.lrmoe_version() >> 16 == 1
     assert lib.lrmoe_status_string(0) == b"ok"
