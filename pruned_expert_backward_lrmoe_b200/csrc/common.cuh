@@ -386,6 +386,18 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t cl_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cl_addr), "r"(v) : "memory");
 }
 
+// 16 zero bytes at a cluster shared-memory address (16-byte aligned).
+__device__ __forceinline__ void st_cluster_zero16(uint32_t cl_addr) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(cl_addr), "r"(0u)
+               : "memory");
+}
+
+// Generic-proxy writes to shared memory of any CTA of the cluster become visible to
+// the async proxy (TMA, tensor cores) of later operations.
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+
 // Every thread of both CTAs of the cluster.
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::

@@ -270,6 +270,26 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-window map over a [rows][cols] bf16 matrix, for K-tail blocks that must end at
+// an arbitrary row: dims (cols, 64, rows - 63) with both outer dims stepping one row
+// (the same stride).  A 64 x 64 box loaded at coordinates (c, 64 - v, e - 64) holds
+// rows e-v .. e-1 of columns c .. c+63 and then 64 - v rows of zeros: element i of
+// the box sits at window coordinate 64 - v + i, past the window's extent for i >= v.
+// Needs e >= 64 (a smaller end is a negative, out-of-range coordinate: zeros only);
+// an element inside all extents is row (64 - v + i) + (e - 64) <= rows - 1, so
+// nothing outside the matrix is read.  128-B swizzle, like the 2D maps.
+bool make_map_rows_window(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, 64, rows > 64 ? rows - 63 : 1};
+  cuuint64_t strides[2] = {cols * 2, cols * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3D bf16 map over [E][K][N], box = 64 (N) x 64 (K) x 1, 128-B swizzle.
 bool make_map_3d(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t N) {
   EncodeTiledFn fn = encode_fn();

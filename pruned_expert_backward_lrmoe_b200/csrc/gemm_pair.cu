@@ -45,7 +45,8 @@ constexpr int kPairBBytes = kHalfN * BK * 2; // 16 KB: this CTA's 128 B columns
 constexpr int kPairStage = kPairABytes + kPairBBytes;
 // warps that read a tile-ring slot: leader MMA + epilogue, peer producer +
 // epilogue, and (wgrad) the peer's K-tail warp
-__host__ __device__ constexpr int pair_consumers(bool wg) { return 2 * (1 + kEpiWarps) + (wg ? 1 : 0); }
+// tile-ring consumers: per CTA the MMA warp (leader) or producer (peer), and the epilogue warps
+__host__ __device__ constexpr int pair_consumers() { return 2 * (1 + kEpiWarps); }
 
 // Launch counter of the pair kernels (picks the scheduling slot).
 std::atomic<unsigned int> g_launches{0};
@@ -57,9 +58,9 @@ struct PairLayout {
   static constexpr int kOutOff = kTilesBytes;
   static constexpr int kOutBytes = kEpiWarps * OUTBUFS * kOutBufBytes;
   static constexpr int kBarOff = kOutOff + kOutBytes;
-  // per stage: full (leader), empty, tail (peer: its K-tail block landed);
-  // tfull[2], tempty[2], mma_done; per ring slot: full, empty
-  static constexpr int kNumBars = 3 * STAGES + 5 + 2 * kRing;
+  // per stage: full (leader), empty; tfull[2], tempty[2], mma_done; per ring
+  // slot: full, empty
+  static constexpr int kNumBars = 2 * STAGES + 5 + 2 * kRing;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag, tile ring
   static constexpr int kTableOff = kMiscOff + 16 + 4 * kRing;
   __host__ __device__ static constexpr int table_ints(int E) { return 3 * (E + 1) + 33; }
@@ -110,18 +111,17 @@ __device__ __forceinline__ PairTile decode_pair(int t, const GemmParams& p, cons
   return ti;
 }
 
-// Zero rows [valid, valid + rows_bad) of every 64-wide column chunk of this CTA's
-// stage (A: two chunks, B: two chunks; 128-byte rows), one warp.
-__device__ __forceinline__ void zero_tail_rows(uint8_t* sa, uint8_t* sb, int valid, int rows_bad,
-                                               int lane) {
-  constexpr int nchunk = 4;
+// Zero rows [valid, valid + rows_bad) of the four 64-column chunks (A: two, B: two;
+// 128-byte rows) of one stage in both CTAs of the pair, through cluster addresses
+// (own: rank 0, peer: rank 1).  One warp.
+__device__ __forceinline__ void zero_rows_both(uint32_t own, uint32_t peer, int valid,
+                                               int rows_bad, int lane) {
   const int per_chunk = rows_bad * 8;  // 16-byte pieces per chunk
-  for (int i = lane; i < nchunk * per_chunk; i += 32) {
-    const int ch = i / per_chunk;
-    const int rem = i - ch * per_chunk;
-    uint8_t* base = ch < 2 ? sa + ch * 8192 : sb + (ch - 2) * 8192;
-    *reinterpret_cast<uint4*>(base + (valid + (rem >> 3)) * 128 + (rem & 7) * 16) =
-        make_uint4(0, 0, 0, 0);
+  for (int i = lane; i < 8 * per_chunk; i += 32) {
+    const int c = i / per_chunk, rem = i - c * per_chunk;  // c: CTA * 4 + chunk
+    const uint32_t off =
+        (uint32_t)((c & 3) * 8192 + (valid + (rem >> 3)) * 128 + (rem & 7) * 16);
+    st_cluster_zero16((c < 4 ? own : peer) + off);
   }
 }
 
@@ -132,6 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
     const __grid_constant__ CUtensorMap tmA /* dgrad rows (K-major) / wgrad grad rows */,
     const __grid_constant__ CUtensorMap tmB /* dgrad W [E][K][N] / wgrad in rows */,
     const __grid_constant__ CUtensorMap tmOut /* wgrad dW [E][N1][N2] fp32 */,
+    const __grid_constant__ CUtensorMap tmTA /* wgrad K-tail row windows over tmA's rows */,
+    const __grid_constant__ CUtensorMap tmTB /* the same over tmB's rows */,
     const GemmParams p) {
   constexpr bool WG = MODE == kWgrad;
   constexpr bool SWIGLU = MODE == kDgradSwiglu;
@@ -146,12 +148,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
-  uint64_t* tailb = bars + 2 * STAGES;
-  uint64_t* tfull = bars + 3 * STAGES;       // [2]
-  uint64_t* tempty = bars + 3 * STAGES + 2;  // [2]
-  uint64_t* mma_done = bars + 3 * STAGES + 4;
-  uint64_t* ring_full = bars + 3 * STAGES + 5;           // [kRing]
-  uint64_t* ring_empty = bars + 3 * STAGES + 5 + kRing;  // [kRing]
+  uint64_t* tfull = bars + 2 * STAGES;       // [2]
+  uint64_t* tempty = bars + 2 * STAGES + 2;  // [2]
+  uint64_t* mma_done = bars + 2 * STAGES + 4;
+  uint64_t* ring_full = bars + 2 * STAGES + 5;           // [kRing]
+  uint64_t* ring_empty = bars + 2 * STAGES + 5 + kRing;  // [kRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   volatile int* ring = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 16);  // [kRing]
@@ -169,7 +170,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&full[i], 2);  // leader's arrive.expect_tx + one arrival of the peer
       mbar_init(&empty[i], 1);
-      mbar_init(&tailb[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
     mbar_init(mma_done, 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&ring_full[i], 1);
-      mbar_init(&ring_empty[i], pair_consumers(WG));
+      mbar_init(&ring_empty[i], pair_consumers());
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -186,6 +186,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if constexpr (WG) {
+      tma_prefetch_desc(&tmTA);
+      tma_prefetch_desc(&tmTB);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 2 * BN);
@@ -237,7 +241,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
     int stage = 0;
     uint32_t phase = 0;
     uint32_t armed = 0, armed_par = 0;  // leader: stages with loads issued, and their phase
-    uint32_t tail_used = 0, tail_next = 0;  // peer: stages with a tail load issued; next phase
     const uint32_t peer_ring = cluster_addr((const void*)ring, 1);
     const uint32_t peer_ring_full = cluster_addr(ring_full, 1);
     // Leader: claim a tile and hand it to both CTAs' consumers in ring slot it2 % kRing
@@ -289,7 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
         uint8_t* sb = sa + kPairABytes;
         const int r = ti.row0 + kb * BK;
         const int valid = ti.row_end - r;
-        const bool tail = WG && valid < BK;
+        // wgrad K-tail block (fewer than 64 of the expert's rows left): loaded through
+        // the row-window maps, whose window ends at the expert's last row, so that
+        // the rows past it land as zeros.  An expert that ends before packed row 64
+        // has no such window: its tail block is loaded plainly and the MMA warp
+        // zeroes the rows past the end (rare: only the first rows of the buffer).
+        const bool win = WG && valid < BK && ti.row_end >= BK;
+        const int tw = BK - valid, te = ti.row_end - BK;  // window coordinates
         const int a_c0 = WG ? ti.m0 + (int)rank * BM : kb * BK;  // A coordinates of this CTA
         const int a_c1 = WG ? r : ti.row0 + (int)rank * BM;
         // B columns of this CTA: 128 (two 64-column boxes), or 64 on a narrow tile
@@ -299,47 +308,46 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
           if (lane == 0) {
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-            mbar_arrive_expect_tx(&full[stage], cta_bytes + (tail ? 0u : cta_bytes));
+            mbar_arrive_expect_tx(&full[stage], 2 * cta_bytes);
             if constexpr (WG) {
-              tma_load_2d(sa, &tmA, &full[stage], a_c0, a_c1);
-              tma_load_2d(sa + 8192, &tmA, &full[stage], a_c0 + 64, a_c1);
-              tma_load_2d(sb, &tmB, &full[stage], b_col, r);
-              if (!ti.narrow) tma_load_2d(sb + 8192, &tmB, &full[stage], b_col + 64, r);
+              if (win) {
+                tma_load_3d(sa, &tmTA, &full[stage], a_c0, tw, te);
+                tma_load_3d(sa + 8192, &tmTA, &full[stage], a_c0 + 64, tw, te);
+                tma_load_3d(sb, &tmTB, &full[stage], b_col, tw, te);
+                if (!ti.narrow) tma_load_3d(sb + 8192, &tmTB, &full[stage], b_col + 64, tw, te);
+              } else {
+                tma_load_2d(sa, &tmA, &full[stage], a_c0, a_c1);
+                tma_load_2d(sa + 8192, &tmA, &full[stage], a_c0 + 64, a_c1);
+                tma_load_2d(sb, &tmB, &full[stage], b_col, r);
+                if (!ti.narrow) tma_load_2d(sb + 8192, &tmB, &full[stage], b_col + 64, r);
+              }
             } else {
               tma_load_2d(sa, &tmA, &full[stage], a_c0, a_c1);
               tma_load_3d(sb, &tmB, &full[stage], b_col, kb * BK, ti.e);
               if (!ti.narrow) tma_load_3d(sb + 8192, &tmB, &full[stage], b_col + 64, kb * BK, ti.e);
             }
           }
-        } else if (!tail) {
+        } else {
           if (lane == 0) {
             const uint32_t fb = lead_full + 8u * stage;
             if constexpr (WG) {
-              tma_load_2d_pair(sa, &tmA, fb, a_c0, a_c1);
-              tma_load_2d_pair(sa + 8192, &tmA, fb, a_c0 + 64, a_c1);
-              tma_load_2d_pair(sb, &tmB, fb, b_col, r);
-              if (!ti.narrow) tma_load_2d_pair(sb + 8192, &tmB, fb, b_col + 64, r);
+              if (win) {
+                tma_load_3d_pair(sa, &tmTA, fb, a_c0, tw, te);
+                tma_load_3d_pair(sa + 8192, &tmTA, fb, a_c0 + 64, tw, te);
+                tma_load_3d_pair(sb, &tmTB, fb, b_col, tw, te);
+                if (!ti.narrow) tma_load_3d_pair(sb + 8192, &tmTB, fb, b_col + 64, tw, te);
+              } else {
+                tma_load_2d_pair(sa, &tmA, fb, a_c0, a_c1);
+                tma_load_2d_pair(sa + 8192, &tmA, fb, a_c0 + 64, a_c1);
+                tma_load_2d_pair(sb, &tmB, fb, b_col, r);
+                if (!ti.narrow) tma_load_2d_pair(sb + 8192, &tmB, fb, b_col + 64, r);
+              }
             } else {
               tma_load_2d_pair(sa, &tmA, fb, a_c0, a_c1);
               tma_load_3d_pair(sb, &tmB, fb, b_col, kb * BK, ti.e);
               if (!ti.narrow) tma_load_3d_pair(sb + 8192, &tmB, fb, b_col + 64, kb * BK, ti.e);
             }
             mbar_arrive_cluster_relaxed(fb);  // the bytes themselves are counted by the barrier
-          }
-        } else {
-          // peer, last K block of a wgrad tile: land it on this CTA's tail barrier;
-          // warp 1 zeroes the rows past the expert's end and then lets the
-          // leader's MMAs read it (this warp goes on with the next loads)
-          if constexpr (WG) {
-            if (lane == 0) {
-              tail_used |= 1u << stage;
-              tail_next ^= 1u << stage;
-              mbar_arrive_expect_tx(&tailb[stage], cta_bytes);
-              tma_load_2d(sa, &tmA, &tailb[stage], a_c0, a_c1);
-              tma_load_2d(sa + 8192, &tmA, &tailb[stage], a_c0 + 64, a_c1);
-              tma_load_2d(sb, &tmB, &tailb[stage], b_col, r);
-              if (!ti.narrow) tma_load_2d(sb + 8192, &tmB, &tailb[stage], b_col + 64, r);
-            }
           }
         }
         if (++stage == STAGES) {
@@ -350,52 +358,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
       if (!ok) break;
     }
     // Let every load this pair started land before shared memory is released:
-    // the leader's stage barriers count the peer's bytes too (the peer's own
-    // tail loads were waited for above).
+    // the leader's stage barriers count the peer's bytes too.
     if (leader && lane == 0)
       for (int i = 0; i < STAGES; ++i)
         if ((armed >> i) & 1u) mbar_wait_drain<true>(&full[i], (armed_par >> i) & 1u);
-    if (!leader && lane == 0)
-      for (int i = 0; i < STAGES; ++i)
-        if ((tail_used >> i) & 1u) mbar_wait_drain(&tailb[i], ((tail_next >> i) & 1u) ^ 1u);
     __syncwarp();
-  } else if (warp == 1 && !leader) {
-    // ---------------- peer: K-tail blocks (wgrad) ----------------
-    // Follows the producer's tile and stage sequence; for each tile's last K
-    // block waits for its own copy to land, zeroes the rows past the expert's
-    // end and arrives on the leader's stage barrier.
-    if constexpr (WG) {
-      int stage = 0;
-      uint32_t tail_par = 0;  // phase of each stage's tail barrier
-      for (int it = 0;; ++it) {
-        const int t = next_tile(it);
-        if (t < 0) break;
-        const PairTile ti = decode_pair<WG>(t, p, offs_s, tab_d, tab_w, tc);
-        bool ok = true;
-        for (int kb = 0; kb < ti.nk; ++kb) {
-          const int valid = ti.row_end - (ti.row0 + kb * BK);
-          if (valid < BK && !(p.stall && it == 0 && kb == 0)) {
-            uint8_t* sa = smem + stage * kPairStage;
-            uint8_t* sb = sa + kPairABytes;
-            const bool landed = __all_sync(
-                kFull, mbar_wait_bounded(&tailb[stage], (tail_par >> stage) & 1u, abort_flag,
-                                         status, wlim));
-            tail_par ^= 1u << stage;
-            if (!landed) {
-              ok = false;
-              break;
-            }
-            const int nkk = (valid + UK - 1) / UK;
-            zero_tail_rows(sa, sb, valid, nkk * UK - valid, lane);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(lead_full + 8u * stage);
-          }
-          if (++stage == STAGES) stage = 0;
-        }
-        if (!ok) break;
-      }
-    }
   } else if (warp == 1) {
     if (leader) {
       // ---------------- MMA issuer (leader only) ----------------
@@ -419,12 +386,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
         const uint32_t d_tmem = tmem_base + b * BN;
         bool ok = true;
         for (int kb = 0; kb < ti.nk; ++kb) {
-          // the K-tail block carries the peer's zeroed rows (generic writes released
-          // at cluster scope); every other block's data is counted in transaction bytes
-          const bool tail_blk = WG && ti.row_end - (ti.row0 + kb * BK) < BK;
+          // every block's data (both CTAs' halves) is counted in transaction bytes; an
+          // early K-tail block (see the producer) is zeroed here, after a wait at
+          // cluster scope so that the peer's copy is ordered before those stores
+          const int valid = ti.row_end - (ti.row0 + kb * BK);
+          const bool early = WG && valid < BK && ti.row_end < BK;
           const bool landed =
-              tail_blk ? mbar_wait_bounded<true>(&full[stage], phase, abort_flag, status, wlim)
-                       : mbar_wait_bounded(&full[stage], phase, abort_flag, status, wlim);
+              early ? mbar_wait_bounded<true>(&full[stage], phase, abort_flag, status, wlim)
+                    : mbar_wait_bounded(&full[stage], phase, abort_flag, status, wlim);
           if (!__all_sync(kFull, landed)) {
             ok = false;
             break;
@@ -434,15 +403,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
           uint8_t* sb = sa + kPairABytes;
           int nkk = BK / UK;
           if constexpr (WG) {
-            const int valid = ti.row_end - (ti.row0 + kb * BK);
-            if (valid < BK) {
-              nkk = (valid + UK - 1) / UK;
-              const int rows_bad = nkk * UK - valid;
-              if (rows_bad > 0) {
-                zero_tail_rows(sa, sb, valid, rows_bad, lane);
-                fence_proxy_async_smem();
-                __syncwarp();
-              }
+            // K-tail block: only the 16-row steps that hold the expert's rows (the
+            // rest of the last step is zero)
+            if (valid < BK) nkk = (valid + UK - 1) / UK;
+            if (early && nkk * UK > valid) {
+              zero_rows_both(cluster_addr(sa, 0), cluster_addr(sa, 1), valid, nkk * UK - valid,
+                             lane);
+              fence_proxy_async_cluster();
+              __syncwarp();
             }
           }
           if (lane == 0) {
@@ -613,7 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
 
 template <int MODE, int S, int OB>
 cudaError_t launch_pair_variant(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& out,
-                                GemmParams prm, cudaStream_t s, long long tiles) {
+                                const CUtensorMap& ta, const CUtensorMap& tb, GemmParams prm,
+                                cudaStream_t s, long long tiles) {
   using L = PairLayout<S, OB>;
   const int smem = L::alloc(prm.E);
   if (smem > kSmemLimit) return cudaErrorInvalidConfiguration;
@@ -647,7 +616,7 @@ cudaError_t launch_pair_variant(const CUtensorMap& a, const CUtensorMap& b, cons
   cfg.gridDim = dim3(2 * clusters);
   cfg.numAttrs = 2;
   prm.sched_slot = (int)(g_launches.fetch_add(1u) % kSchedSlots);
-  return cudaLaunchKernelEx(&cfg, kern, a, b, out, prm);
+  return cudaLaunchKernelEx(&cfg, kern, a, b, out, ta, tb, prm);
 }
 
 }  // namespace
@@ -673,8 +642,8 @@ cudaError_t launch_dgrad_pair(const void* rows, int rows_cap, const void* W,
   const long long tiles =
       ((long long)rows_cap / kPairM + E) * ((N + kBNT - 1) / kBNT);
   if (epi == LRMOE_EPI_SWIGLU_BWD)
-    return launch_pair_variant<kDgradSwiglu, 6, 0>(a, b, a, prm, s, tiles);
-  return launch_pair_variant<kDgradStore, 6, 0>(a, b, a, prm, s, tiles);
+    return launch_pair_variant<kDgradSwiglu, 6, 0>(a, b, a, a, a, prm, s, tiles);
+  return launch_pair_variant<kDgradStore, 6, 0>(a, b, a, a, a, prm, s, tiles);
 }
 
 // Diagnostic: the dgrad (store epilogue) with the first K block withheld and every
@@ -690,7 +659,7 @@ cudaError_t launch_dgrad_stall_pair(const void* rows, int rows_cap, const void* 
                  status, 0, wait_ns, 1};
   prm.rows_cap = rows_cap;
   const long long tiles = ((long long)rows_cap / kPairM + E) * ((N + kBNT - 1) / kBNT);
-  return launch_pair_variant<kDgradStore, 6, 0>(a, b, a, prm, s, tiles);
+  return launch_pair_variant<kDgradStore, 6, 0>(a, b, a, a, a, prm, s, tiles);
 }
 
 // wgrad on pairs of SMs: dW[e] = grad[R_e]^T . in[R_e] (fp32 out, stored or added).
@@ -698,9 +667,11 @@ cudaError_t launch_wgrad_pair(const void* grad_rows, const void* in_rows, int ro
                               const int32_t* offsets, int E, int N1, int N2, float* dW,
                               int accumulate, uint32_t* status, cudaStream_t s,
                               const char** why) {
-  CUtensorMap a, b, out;
+  CUtensorMap a, b, out, ta, tb;
   if (!make_map_2d(&a, grad_rows, (uint64_t)rows_cap, (uint64_t)N1, 64, 64) ||
       !make_map_2d(&b, in_rows, (uint64_t)rows_cap, (uint64_t)N2, 64, 64) ||
+      !make_map_rows_window(&ta, grad_rows, (uint64_t)rows_cap, (uint64_t)N1) ||
+      !make_map_rows_window(&tb, in_rows, (uint64_t)rows_cap, (uint64_t)N2) ||
       !make_map_out_f32(&out, dW, (uint64_t)E, (uint64_t)N1, (uint64_t)N2)) {
     *why = "cuTensorMapEncodeTiled failed for a wgrad operand";
     return cudaErrorInvalidValue;
@@ -710,8 +681,8 @@ cudaError_t launch_wgrad_pair(const void* grad_rows, const void* in_rows, int ro
   prm.rows_cap = rows_cap;
   const long long tiles = (long long)E * ((N1 + kPairM - 1) / kPairM) * ((N2 + kBNT - 1) / kBNT);
   if (PairLayout<5, 1>::alloc(E) <= kSmemLimit)
-    return launch_pair_variant<kWgrad, 5, 1>(a, b, out, prm, s, tiles);
-  return launch_pair_variant<kWgrad, 4, 1>(a, b, out, prm, s, tiles);
+    return launch_pair_variant<kWgrad, 5, 1>(a, b, out, ta, tb, prm, s, tiles);
+  return launch_pair_variant<kWgrad, 4, 1>(a, b, out, ta, tb, prm, s, tiles);
 }
 
 }  // namespace lrmoe
