@@ -33,6 +33,8 @@
 // issues).  Every wait is bounded (LRMOE_ST_TIMEOUT, then a clean exit through
 // a cluster barrier, so that neither CTA leaves while the other can still
 // touch its shared memory).  No TMA multicast.
+#include <type_traits>
+
 #include "gemm_common.cuh"
 
 namespace lrmoe {
@@ -274,31 +276,37 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
       }
       if (t < 0) break;
       const PairTile ti = decode_pair<WG>(t, p, offs_s, tab_d, tab_w, tc);
-      bool ok = true;
-      for (int kb = 0; kb < ti.nk; ++kb) {
+      // one K block: wait for its stage, then both CTAs' copies; the last block of a
+      // wgrad tile may be a K tail (the loop over the other blocks carries no tail
+      // logic at all)
+      auto load_block = [&](int kb, auto last_c) -> bool {
+        constexpr bool kLast = decltype(last_c)::value && WG;
         if (!__all_sync(kFull, mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status,
-                                                 wlim))) {
-          ok = false;
-          break;
-        }
+                                                 wlim)))
+          return false;
         if (p.stall && it == 0 && kb == 0) {  // diagnostic: this block never arrives
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
-          continue;
+          return true;
         }
         uint8_t* sa = smem + stage * kPairStage;
         uint8_t* sb = sa + kPairABytes;
         const int r = ti.row0 + kb * BK;
-        const int valid = ti.row_end - r;
         // wgrad K-tail block (fewer than 64 of the expert's rows left): loaded through
         // the row-window maps, whose window ends at the expert's last row, so that
         // the rows past it land as zeros.  An expert that ends before packed row 64
         // has no such window: its tail block is loaded plainly and the MMA warp
         // zeroes the rows past the end (rare: only the first rows of the buffer).
-        const bool win = WG && valid < BK && ti.row_end >= BK;
-        const int tw = BK - valid, te = ti.row_end - BK;  // window coordinates
+        bool win = false;
+        int tw = 0, te = 0;  // window coordinates
+        if constexpr (kLast) {
+          const int valid = ti.row_end - r;
+          win = valid < BK && ti.row_end >= BK;
+          tw = BK - valid;
+          te = ti.row_end - BK;
+        }
         const int a_c0 = WG ? ti.m0 + (int)rank * BM : kb * BK;  // A coordinates of this CTA
         const int a_c1 = WG ? r : ti.row0 + (int)rank * BM;
         // B columns of this CTA: 128 (two 64-column boxes), or 64 on a narrow tile
@@ -354,6 +362,58 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
           stage = 0;
           phase ^= 1u;
         }
+        return true;
+      };
+      bool ok = true;
+      if constexpr (WG) {  // the last block peeled off
+        for (int kb = 0; kb + 1 < ti.nk; ++kb)
+          if (!(ok = load_block(kb, std::false_type{}))) break;
+        if (ok && ti.nk > 0) ok = load_block(ti.nk - 1, std::true_type{});
+      } else {
+        // dgrad: the same steps written inline in one loop (measured faster than the
+        // block function for these instantiations)
+        for (int kb = 0; kb < ti.nk; ++kb) {
+          if (!__all_sync(kFull, mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, status,
+                                                   wlim))) {
+            ok = false;
+            break;
+          }
+          if (p.stall && it == 0 && kb == 0) {  // diagnostic: this block never arrives
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
+          uint8_t* sa = smem + stage * kPairStage;
+          uint8_t* sb = sa + kPairABytes;
+          const int a_c1 = ti.row0 + (int)rank * BM;  // A rows of this CTA
+          // B columns of this CTA: 128 (two 64-column boxes), or 64 on a narrow tile
+          const int b_col = ti.n0 + (int)rank * (ti.narrow ? 64 : kHalfN);
+          const uint32_t cta_bytes = kPairABytes + (ti.narrow ? kPairBBytes / 2 : kPairBBytes);
+          if (leader) {
+            if (lane == 0) {
+              armed |= 1u << stage;
+              armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+              mbar_arrive_expect_tx(&full[stage], 2 * cta_bytes);
+              tma_load_2d(sa, &tmA, &full[stage], kb * BK, a_c1);
+              tma_load_3d(sb, &tmB, &full[stage], b_col, kb * BK, ti.e);
+              if (!ti.narrow) tma_load_3d(sb + 8192, &tmB, &full[stage], b_col + 64, kb * BK, ti.e);
+            }
+          } else {
+            if (lane == 0) {
+              const uint32_t fb = lead_full + 8u * stage;
+              tma_load_2d_pair(sa, &tmA, fb, kb * BK, a_c1);
+              tma_load_3d_pair(sb, &tmB, fb, b_col, kb * BK, ti.e);
+              if (!ti.narrow) tma_load_3d_pair(sb + 8192, &tmB, fb, b_col + 64, kb * BK, ti.e);
+              mbar_arrive_cluster_relaxed(fb);  // the bytes themselves are counted by the barrier
+            }
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
       }
       if (!ok) break;
     }
@@ -384,25 +444,28 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
           break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * BN;
-        bool ok = true;
-        for (int kb = 0; kb < ti.nk; ++kb) {
-          // every block's data (both CTAs' halves) is counted in transaction bytes; an
-          // early K-tail block (see the producer) is zeroed here, after a wait at
-          // cluster scope so that the peer's copy is ordered before those stores
-          const int valid = ti.row_end - (ti.row0 + kb * BK);
-          const bool early = WG && valid < BK && ti.row_end < BK;
+        // one K block: wait for both CTAs' copies and issue its MMAs; the last block of
+        // a wgrad tile may be a K tail (the loop over the other blocks carries no tail
+        // logic at all).  Every block's data is counted in transaction bytes; an early
+        // K-tail block (see the producer) is zeroed here, after a wait at cluster scope
+        // so that the peer's copy is ordered before those stores.
+        auto mma_block = [&](int kb, auto last_c) -> bool {
+          constexpr bool kLast = decltype(last_c)::value && WG;
+          int valid = BK;
+          bool early = false;
+          if constexpr (kLast) {
+            valid = ti.row_end - (ti.row0 + kb * BK);
+            early = valid < BK && ti.row_end < BK;
+          }
           const bool landed =
               early ? mbar_wait_bounded<true>(&full[stage], phase, abort_flag, status, wlim)
                     : mbar_wait_bounded(&full[stage], phase, abort_flag, status, wlim);
-          if (!__all_sync(kFull, landed)) {
-            ok = false;
-            break;
-          }
+          if (!__all_sync(kFull, landed)) return false;
           tc_fence_after();
           uint8_t* sa = smem + stage * kPairStage;
           uint8_t* sb = sa + kPairABytes;
           int nkk = BK / UK;
-          if constexpr (WG) {
+          if constexpr (kLast) {
             // K-tail block: only the 16-row steps that hold the expert's rows (the
             // rest of the last step is zero)
             if (valid < BK) nkk = (valid + UK - 1) / UK;
@@ -415,14 +478,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
           }
           if (lane == 0) {
             const uint32_t a_addr = smem_u32(sa), b_addr = smem_u32(sb);
+            const uint32_t idesc = ti.narrow ? idesc_narrow : idesc_full;
 #pragma unroll
             for (int kk = 0; kk < BK / UK; ++kk) {
-              if (kk >= nkk) break;
+              if (kLast && kk >= nkk) break;
               const uint64_t adesc = WG ? smem_desc_sw128(a_addr + kk * 2048, 8192, 1024)
                                         : smem_desc_sw128(a_addr + kk * 32, 16, 1024);
               const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, 8192, 1024);
-              tc_mma_f16_pair(d_tmem, adesc, bdesc, ti.narrow ? idesc_narrow : idesc_full,
-                              (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
             }
             // the stage is free in both CTAs once these MMAs have read it
             tc_commit_pair(smem_u32(&empty[stage]));
@@ -432,6 +495,45 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_pair(
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
+          }
+          return true;
+        };
+        bool ok = true;
+        if constexpr (WG) {  // the last block peeled off
+          for (int kb = 0; kb + 1 < ti.nk; ++kb)
+            if (!(ok = mma_block(kb, std::false_type{}))) break;
+          if (ok) ok = mma_block(ti.nk - 1, std::true_type{});
+        } else {
+          // dgrad: the same steps written inline in one loop (measured faster than the
+          // block function for these instantiations)
+          for (int kb = 0; kb < ti.nk; ++kb) {
+            // every block's data (both CTAs' halves) is counted in transaction bytes
+            if (!__all_sync(kFull,
+                            mbar_wait_bounded(&full[stage], phase, abort_flag, status, wlim))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            uint8_t* sa = smem + stage * kPairStage;
+            uint8_t* sb = sa + kPairABytes;
+            if (lane == 0) {
+              const uint32_t a_addr = smem_u32(sa), b_addr = smem_u32(sb);
+#pragma unroll
+              for (int kk = 0; kk < BK / UK; ++kk) {
+                const uint64_t adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+                const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, 8192, 1024);
+                tc_mma_f16_pair(d_tmem, adesc, bdesc, ti.narrow ? idesc_narrow : idesc_full,
+                                (kb | kk) != 0 ? 1u : 0u);
+              }
+              // the stage is free in both CTAs once these MMAs have read it
+              tc_commit_pair(smem_u32(&empty[stage]));
+              tc_commit_pair(peer_empty + 8u * stage);
+            }
+            __syncwarp();
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
         if (!ok) break;
