@@ -31,6 +31,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -147,14 +148,22 @@ KERNEL_SOURCES = {
 GEMM_SOURCES = _GEMM_SOURCES
 
 
+def _code_only(text: str) -> str:
+    """C++/CUDA source without comments and with whitespace runs collapsed, so that an
+    edit of comments alone does not count as a change of the kernel."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_sha1(kernel: str = "wgrad_gu") -> str:
-    """sha1 over the source files that define `kernel` (name and bytes of each)."""
+    """sha1 over the code (comments dropped) of the source files that define `kernel`."""
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "pruned_expert_backward_lrmoe_b200", "csrc")
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 

@@ -27,10 +27,11 @@
 //            Peer: only allocates and frees its half of the tensor memory.
 //   warps 2-9  epilogue in both CTAs, each on its own 128 rows; the leader may
 //            reuse an accumulator once all 16 epilogue warps have drained it.
-// Variable K (wgrad): the last K block of an expert may reach into the next
-// expert's rows.  Each CTA zeroes those rows of its own halves (the peer's
-// producer before it signals the leader, the leader's MMA warp before it
-// issues).  Every wait is bounded (LRMOE_ST_TIMEOUT, then a clean exit through
+// Variable K (wgrad): the last K block of an expert would reach into the next
+// expert's rows.  It is loaded through row-window tensor maps whose window ends
+// at the expert's last row, so the rows past it arrive as zeros; only an expert
+// that ends before packed row 64 (no window fits) is zeroed by the leader's MMA
+// warp in both CTAs' shared memory.  Every wait is bounded (LRMOE_ST_TIMEOUT, then a clean exit through
 // a cluster barrier, so that neither CTA leaves while the other can still
 // touch its shared memory).  No TMA multicast.
 #include <type_traits>
@@ -45,9 +46,8 @@ constexpr int kHalfN = kBNT / 2;             // B columns loaded by each CTA
 constexpr int kPairABytes = BM * BK * 2;     // 16 KB: this CTA's 128 A rows of a K block
 constexpr int kPairBBytes = kHalfN * BK * 2; // 16 KB: this CTA's 128 B columns
 constexpr int kPairStage = kPairABytes + kPairBBytes;
-// warps that read a tile-ring slot: leader MMA + epilogue, peer producer +
-// epilogue, and (wgrad) the peer's K-tail warp
-// tile-ring consumers: per CTA the MMA warp (leader) or producer (peer), and the epilogue warps
+// warps that read a tile-ring slot: the leader's MMA warp, the peer's producer, and
+// the epilogue warps of both CTAs
 __host__ __device__ constexpr int pair_consumers() { return 2 * (1 + kEpiWarps); }
 
 // Launch counter of the pair kernels (picks the scheduling slot).
