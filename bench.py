@@ -808,6 +808,21 @@ def run_extras(layer, res, dev, args, dist, peaks):
     }
     if int(st.item()) != 0:
         raise SystemExit(f"device status {int(st.item())} after the destination split")
+
+    # ---------------- the redistributed backward at world size 1 ----------------
+    # exchange.redistributed_backward on this layer with one rank: the same GEMMs as
+    # the step plus the exchange bookkeeping (split by receiver, wide exchange rows,
+    # grouping of the received rows, their split, the return gathers) and its two
+    # host synchronisations; the all-to-alls are local copies at this size.
+    from pruned_expert_backward_lrmoe_b200 import exchange as X
+    ones = np.ones((s.E, 1), bool)
+    ex_st = {}
+    ex_ms = timed(lambda: ex_st.update(X.redistributed_backward(inp, ones)), n=5, warm=2)
+    x["exchange_world1"] = {"ms": ex_ms, "step_ms": res["ms_per_step"],
+                            "value": M_all / (ex_ms * 1e-3),
+                            "unit": UNIT, "status": int(ex_st["status"].item())}
+    del ex_st
+    torch.cuda.empty_cache()
     return x
 
 
