@@ -494,61 +494,63 @@ def make_runner(layer, dev):
         flush.sum()
     st = out["status"]
 
-    def step(ev=None, a_sqnorm=None, fused=False, wgrad_gather=False, waits=None):
+    def step(ev=None, a_sqnorm=None, fused=False, wgrad_gather=False, waits=None, src=None):
         """One pass of the path; with a_sqnorm (||a_p||^2 saved by the forward) the
-        score reads dY and the saved norms instead of a."""
+        score reads dY and the saved norms instead of a; `src` replaces the device
+        inputs (a second set, for uploads that overlap the previous step)."""
+        inp_ = inp if src is None else src
         gather = s.dtype == "bf16" and not fused   # the path's g, u handling
         score_call = (
-            (lambda: L.lrmoe_score(inp["topk_idx"], inp["topk_w"], inp["dY"], inp["a"], s.E,
+            (lambda: L.lrmoe_score(inp_["topk_idx"], inp_["topk_w"], inp_["dY"], inp_["a"], s.E,
                                    out["score"], st, stream)) if a_sqnorm is None else
-            (lambda: L.lrmoe_score_from_norms(inp["topk_idx"], inp["topk_w"], inp["dY"], a_sqnorm,
+            (lambda: L.lrmoe_score_from_norms(inp_["topk_idx"], inp_["topk_w"], inp_["dY"], a_sqnorm,
                                               s.E, out["score"], st, stream)))
         head = (
             score_call,
-            lambda: L.lrmoe_select_quota(inp["topk_idx"], out["score"], inp["quota"], out["counts"],
+            lambda: L.lrmoe_select_quota(inp_["topk_idx"], out["score"], inp_["quota"], out["counts"],
                                          out["kept"], out["offsets"], out["perm"], out["pos"],
                                          out["workspace"], st, stream),
             # bf16: g, u are read in place at row perm[r] (and, with wgrad_gather, a, x)
-            (lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], None, inp["dY"],
+            (lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp_["topk_w"], None, inp_["dY"],
                                   None, None, None, None, out["DYp"], None, None, None, st,
                                   stream, I=s.I)) if gather and wgrad_gather else
-            (lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], inp["x"], inp["dY"],
-                                  inp["a"], None, None, out["Xp"], out["DYp"], out["Ap"], None,
+            (lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp_["topk_w"], inp_["x"], inp_["dY"],
+                                  inp_["a"], None, None, out["Xp"], out["DYp"], out["Ap"], None,
                                   None, st, stream)) if gather else
-            (lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp["topk_w"], inp["x"], inp["dY"],
-                                  inp["a"], inp["g"], inp["u"], out["Xp"], out["DYp"], out["Ap"],
+            (lambda: L.lrmoe_pack(out["perm"], out["offsets"], inp_["topk_w"], inp_["x"], inp_["dY"],
+                                  inp_["a"], inp_["g"], inp_["u"], out["Xp"], out["DYp"], out["Ap"],
                                   out["Gp"], out["Up"], st, stream)),
         )
         if not fused:  # the four grouped GEMMs as separate launches
             gemms = (
                 (lambda: L.lrmoe_grouped_dgrad_swiglu_gather(
-                    out["DYp"], inp["W_down"], out["offsets"], out["perm"], inp["g"], inp["u"],
+                    out["DYp"], inp_["W_down"], out["offsets"], out["perm"], inp_["g"], inp_["u"],
                     out["dGUp"], status=st, stream=stream)) if gather else
-                (lambda: L.lrmoe_grouped_dgrad(out["DYp"], inp["W_down"], out["offsets"],
+                (lambda: L.lrmoe_grouped_dgrad(out["DYp"], inp_["W_down"], out["offsets"],
                                                L.LRMOE_EPI_SWIGLU_BWD, out["dGUp"], Gp=out["Gp"],
                                                Up=out["Up"], status=st, stream=stream)),
                 (lambda: L.lrmoe_grouped_wgrad_gather(
-                    out["DYp"], out["perm"], inp["a"], 1, s.P, out["offsets"], out["dW_down"],
+                    out["DYp"], out["perm"], inp_["a"], 1, s.P, out["offsets"], out["dW_down"],
                     status=st, stream=stream)) if gather and wgrad_gather else
                 (lambda: L.lrmoe_grouped_wgrad(out["DYp"], out["Ap"], out["offsets"],
                                                out["dW_down"], status=st, stream=stream)),
                 (lambda: L.lrmoe_grouped_wgrad_gather(
-                    out["dGUp"], out["perm"], inp["x"], s.k, s.P, out["offsets"], out["dW_gu"],
+                    out["dGUp"], out["perm"], inp_["x"], s.k, s.P, out["offsets"], out["dW_gu"],
                     status=st, stream=stream)) if gather and wgrad_gather else
                 (lambda: L.lrmoe_grouped_wgrad(out["dGUp"], out["Xp"], out["offsets"],
                                                out["dW_gu"], status=st, stream=stream)),
-                lambda: L.lrmoe_grouped_dgrad(out["dGUp"], inp["W_gu"], out["offsets"],
+                lambda: L.lrmoe_grouped_dgrad(out["dGUp"], inp_["W_gu"], out["offsets"],
                                               L.LRMOE_EPI_STORE, out["dXp"], status=st,
                                               stream=stream),
             )
         else:  # each dgrad with the wgrad over the same gradient rows in one launch
             gemms = (
                 lambda: L.lrmoe_grouped_dgrad_wgrad(
-                    out["DYp"], inp["W_down"], out["offsets"], L.LRMOE_EPI_SWIGLU_BWD,
+                    out["DYp"], inp_["W_down"], out["offsets"], L.LRMOE_EPI_SWIGLU_BWD,
                     out["dGUp"], out["Ap"], out["dW_down"], Gp=out["Gp"], Up=out["Up"],
                     status=st, stream=stream),
                 lambda: L.lrmoe_grouped_dgrad_wgrad(
-                    out["dGUp"], inp["W_gu"], out["offsets"], L.LRMOE_EPI_STORE, out["dXp"],
+                    out["dGUp"], inp_["W_gu"], out["offsets"], L.LRMOE_EPI_STORE, out["dXp"],
                     out["Xp"], out["dW_gu"], status=st, stream=stream),
             )
         calls = head + gemms + (
@@ -828,59 +830,88 @@ def run_extras(layer, res, dev, args, dist, peaks):
 
 def run_e2e(layer, res, dev, args, dist):
     """The same metric end to end: every step uploads its inputs from pinned host
-    memory (on a copy stream, in the order the path consumes them), runs the path
-    and reads dX and the status word back, all inside the timed region."""
+    memory, runs the path and reads dX and the status word back, all inside the timed
+    region.  Steps are pipelined over two sets of device input buffers: the uploads of
+    step j+1 (two copy streams, in the order the path consumes them) run while step j
+    computes, and step j's dX goes back on a third stream.  The timed region spans the
+    whole run, from the first upload to the last read-back; the value is the retained
+    pairs of all steps over that time."""
     import torch
 
     s = layer.spec
     tdt = torch.bfloat16 if s.dtype == "bf16" else torch.float32
     host, inp, out, stream, flush_l2, step = res["runner"]
     pin = {k_: v.pin_memory() for k_, v in host.items()}
-    dX_host = torch.empty(s.T, s.H, dtype=tdt).pin_memory()
-    st_host = torch.empty(1, dtype=torch.int32).pin_memory()
+    sets = (inp, dict(inp, **{k_: torch.empty_like(inp[k_]) for k_ in pin}))
+    dX_host = [torch.empty(s.T, s.H, dtype=tdt).pin_memory() for _ in range(2)]
+    st_host = [torch.zeros(1, dtype=torch.int32).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
-    d2h = dX_host.numel() * dX_host.element_size() + 4
+    d2h = dX_host[0].numel() * dX_host[0].element_size() + 4
     n_e2e = max(3, min(args.steps, 50))
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(n_e2e)]
     # The compute stream waits only where it needs each group (score and select:
-    # routing, dY, a; pack: x; the SwiGLU dgrad: g, u).  Each group's tensors are
-    # split over two copy streams (two DMA queues in flight at once).
+    # routing, dY, a; pack: x; the SwiGLU dgrad: g, u), and its unpack (the last call,
+    # which writes dX) for the read-back of the previous step's dX.  Each group's
+    # tensors are split over two copy streams (two DMA queues in flight at once).
     copy_streams = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    back = torch.cuda.Stream(dev)
     groups = (("topk_idx", "topk_w", "quota", "dY", "a"), ("x",), ("g", "u"))
     need_at = (0, 2, 3)   # step call index before which each group must have landed
-    for i in range(n_e2e + 2):
-        timed = i >= 2
-        flush_l2()
-        if timed:
-            e2e_ev[i - 2][0].record(stream)
+    unpack_at = len(CALL_NAMES) - 1
+
+    def upload(j, after):
+        """Step j's uploads into input set j % 2, once the event `after` has passed."""
+        dst = sets[j % 2]
         for cs in copy_streams:
-            cs.wait_stream(stream)   # the previous step is done with its inputs
+            cs.wait_event(after)
         landed = []
         for grp in groups:
             evs_ = []
-            for j, cs in enumerate(copy_streams):
+            for c, cs in enumerate(copy_streams):
                 with torch.cuda.stream(cs):
                     for k_ in grp:
                         half = pin[k_].shape[0] // 2
-                        rows = slice(0, half) if j == 0 else slice(half, None)
+                        rows = slice(0, half) if c == 0 else slice(half, None)
                         if pin[k_][rows].numel():
-                            inp[k_][rows].copy_(pin[k_][rows], non_blocking=True)
+                            dst[k_][rows].copy_(pin[k_][rows], non_blocking=True)
                     ev_ = torch.cuda.Event()
                     ev_.record(cs)
                     evs_.append(ev_)
             landed.append(evs_)
-        step(waits=dict(zip(need_at, landed)))
-        dX_host.copy_(out["dX"], non_blocking=True)
-        st_host.copy_(out["status"], non_blocking=True)
-        if timed:
-            e2e_ev[i - 2][1].record(stream)
-    torch.cuda.synchronize(dev)
-    if int(st_host.item()) != 0:
-        raise SystemExit(f"device status {int(st_host.item())} after the end-to-end steps")
-    e2e_ms = max_over_ranks(statistics.fmean(a_.elapsed_time(b_) for a_, b_ in e2e_ev), dist)
+        return landed
+
+    def run(n):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        done, read, landed = [None] * n, [None] * n, {0: upload(0, t0)}
+        for j in range(n):
+            if j + 1 < n:   # set (j+1) % 2 was last read by step j-1
+                landed[j + 1] = upload(j + 1, done[j - 1] if j >= 1 else t0)
+            flush_l2()
+            waits = dict(zip(need_at, landed.pop(j)))
+            if j >= 1:
+                waits.setdefault(unpack_at, []).append(read[j - 1])
+            step(waits=waits, src=sets[j % 2])
+            done[j] = torch.cuda.Event()
+            done[j].record(stream)
+            back.wait_event(done[j])
+            with torch.cuda.stream(back):
+                dX_host[j % 2].copy_(out["dX"], non_blocking=True)
+                st_host[j % 2].copy_(out["status"], non_blocking=True)
+                read[j] = torch.cuda.Event()
+                read[j].record(back)
+        stream.wait_event(read[n - 1])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        return t0.elapsed_time(t1)
+
+    run(2)   # warm-up
+    e2e_ms = max_over_ranks(run(n_e2e) / n_e2e, dist)
+    bad = [int(h.item()) for h in st_host if int(h.item()) != 0]
+    if bad:
+        raise SystemExit(f"device status {bad[0]} after the end-to-end steps")
     return {"value": res["M_all"] / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e}
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e,
+            "pipelined": "two input sets: step j+1's uploads overlap step j"}
 
 
 def run_gpu(args):
