@@ -1,7 +1,7 @@
 """The benchmark's measurement model on CPU: the algorithmic bytes and flops that
 every roofline figure divides by, hand-counted on a small layer; the fused-launch
 entries count the shared gradient rows once; recorded DRAM traffic is dropped as
-soon as the GEMM sources change."""
+soon as the kernels' code (comments aside) changes."""
 import json
 import os
 
@@ -69,3 +69,14 @@ def test_roofline_bound_follows_the_ridge():
     r = bench.roofline_of("wgrad_gu", 0.34, by, fl, peaks, "fallback", "qwen")
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert bench.roofline_of("unpack", 0.03, by, fl, peaks, "fallback", "qwen")["bound"] == "hbm"
+
+
+def test_source_hash_ignores_comments_only():
+    """The traffic records are keyed to the kernels' code: an edit of comments or
+    whitespace keeps the key, an edit of code changes it."""
+    code = "int f(int a) {  // doubles\n  /* the\n  result */ return 2 * a;\n}\n"
+    same = "int f(int a) {\n  return 2 * a;  // twice a\n}\n"
+    other = "int f(int a) {\n  return 3 * a;\n}\n"
+    assert bench._code_only(code) == bench._code_only(same)
+    assert bench._code_only(code) != bench._code_only(other)
+    assert "//" not in bench._code_only(code) and "/*" not in bench._code_only(code)
