@@ -230,3 +230,20 @@ def test_quota_controller_rejects_bad_arguments(lib):
     assert f(NULL, 4, 2, 3, 0, -1, FAKE, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
     assert f(FAKE, 4, 2, 5000, 0, -1, FAKE, FAKE, NULL, NULL) == L.LRMOE_ERR_UNSUPPORTED
     assert f(FAKE, 0, 2, 3, 0, -1, FAKE, FAKE, NULL, NULL) == L.LRMOE_ERR_INVALID_ARG
+
+
+def test_binding_selects_the_checked_library_by_environment():
+    """LRMOE_CHECKED=1 makes the binding load liblrmoe_checked.so (read once, at import)."""
+    import subprocess
+    import sys
+    code = ("from pruned_expert_backward_lrmoe_b200 import lrmoe as L; "
+            "print(L.LIB_PATH.rsplit('/', 1)[-1])")
+    for env_val, want in (("1", "liblrmoe_checked.so"), (None, "liblrmoe.so")):
+        env = dict(os.environ)
+        env.pop("LRMOE_CHECKED", None)
+        if env_val is not None:
+            env["LRMOE_CHECKED"] = env_val
+        r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                           text=True, timeout=300)
+        assert r.returncode == 0, r.stderr[-2000:]
+        assert r.stdout.strip() == want
